@@ -1,0 +1,499 @@
+#!/usr/bin/env python
+"""Benchmark of the CoWA hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic inputs:
+cowa_fwd (schedule + forward), cowa_bwd (schedules, delta, dK/dV pass, dQ
+pass) and cowa_decode of one new token per sequence against the same K/V as
+its cache (split-KV + merge).  The default workload is the 8K
+associative-recall-scale training op (B=4, L=8192, Hq=8, Hkv=4, d=64,
+quad (64, 1024, 0, 1792)).
+
+Metric: effective TFLOP/s counted on visible pairs only -- 4*d flops per
+pair forward, 10*d backward, 4*d per visible key and query head in decode --
+over the step time; decode GB/s on visible K+V bytes is reported beside it.
+Timing: CUDA events on the launching stream, L2 flushed (a 512 MiB write)
+before every timed step, max over ranks.  Multi-GPU: every rank runs its own
+batch (data-parallel replicas, no collective on the data path; weak scaling).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle, timed on host cores
+"""
+import argparse
+import datetime
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------- counting ----
+def row_visible_counts(Lq, Lk, quad, h):
+    """Visible keys of every query row of KV head h (int64 [Lq]): the size of
+    the union of the sink, near and long key intervals of the row."""
+    S, N, G, W = (int(x) for x in quad)
+    p = np.arange(Lq, dtype=np.int64) + (Lk - Lq)
+    c = N + G + h * W
+    e = c + W
+    zero = np.zeros_like(p)
+    ivs = [
+        (zero, np.minimum(S, p + 1)),                          # sink  [0, S)
+        (np.maximum(0, p - N + 1), p + 1 if N > 0 else zero),  # near  (p-N, p]
+        (np.maximum(0, p - e + 1), np.maximum(0, p - c + 1) if W > 0 else zero),  # long
+    ]
+    lo = np.stack([np.where(a < b, a, 0) for a, b in ivs], axis=1)
+    hi = np.stack([np.where(a < b, b, 0) for a, b in ivs], axis=1)
+    hi = np.where(p[:, None] >= 0, hi, 0)
+    lo = np.where(hi > lo, lo, 0)
+    hi = np.where(hi > lo, hi, 0)
+    order = np.argsort(lo + (hi == 0) * (1 << 40), axis=1, kind="stable")
+    lo = np.take_along_axis(lo, order, axis=1)
+    hi = np.take_along_axis(hi, order, axis=1)
+    total = np.zeros_like(p)
+    reach = np.zeros_like(p)  # end of the union so far
+    for a in range(3):
+        start = np.maximum(lo[:, a], reach)
+        total += np.maximum(0, hi[:, a] - start)
+        reach = np.maximum(reach, hi[:, a])
+    return total
+
+
+def visible_pairs(B, Lq, Lk, Hq, Hkv, quad, kv_head_offset=0, rows=None):
+    """Visible (query, key) pairs over all batches and query heads."""
+    g = Hq // Hkv
+    tot = 0
+    for h in range(Hkv):
+        cnt = row_visible_counts(Lq, Lk, quad, h + kv_head_offset)
+        if rows is not None:
+            cnt = cnt[rows]
+        tot += int(cnt.sum()) * g
+    return tot * B
+
+
+def decode_visible_keys(seqlens, Hkv, quad, kv_head_offset=0):
+    """Visible keys summed over sequences and KV heads for one decode step."""
+    tot = 0
+    for L in seqlens:
+        for h in range(Hkv):
+            tot += int(row_visible_counts(1, int(L), quad, h + kv_head_offset)[0]) if L > 0 else 0
+    return tot
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise max of a list of floats over all ranks (the slowest rank
+    sets the time of a step)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+# ----------------------------------------------------------------- clocks ----
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = max(smax, float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ peaks ----
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (matched by a hash of csrc/)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            entries = json.load(f)
+    except (OSError, ValueError):
+        return None
+    import hashlib
+    csrc = os.path.join(ROOT, "structured_sparse_attention_block_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    digest = h.hexdigest()[:16]
+    for e in entries:
+        if e.get("kernel") == kernel and e.get("workload") == workload and e.get("csrc_sha") == digest:
+            return e.get("bytes_per_launch")
+    return None
+
+
+# ------------------------------------------------------------- GPU arm ----
+def run_cowa(args, rank, world, local_rank):
+    import torch.distributed as dist
+
+    import structured_sparse_attention_block_b200 as cowa
+    from structured_sparse_attention_block_b200.inputs import WORKLOADS, training_inputs
+
+    wl = WORKLOADS[args.workload]
+    if wl.kind != "train":
+        raise SystemExit("the step workload must be a training workload")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    q, k, v, do = training_inputs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, wl.d, device=dev, seed=1000 * rank)
+    quad = wl.quad
+    # decode: the last query row of every sequence against its full K/V as cache
+    qd = q[:, -1:].contiguous()
+    seqlens = torch.full((wl.B,), wl.Lk, dtype=torch.int32, device=dev)
+
+    o = torch.empty_like(q)
+    lse = torch.empty((wl.B, wl.Hq, wl.Lq), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    od = torch.empty_like(qd)
+    lsed = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device=dev)
+    ws_f = torch.empty(cowa.cowa_fwd_workspace_size(q, k, quad), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(cowa.cowa_bwd_workspace_size(q, k, quad), dtype=torch.uint8, device=dev)
+    ws_d = torch.empty(cowa.cowa_decode_workspace_size(qd, k, quad), dtype=torch.uint8, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        cowa.cowa_fwd(q, k, v, quad, out=o, lse=lse, workspace=ws_f)
+        if ev is not None:
+            ev[1].record(stream)
+        cowa.cowa_bwd(q, k, v, o, lse, do, quad, dq=dq, dk=dk, dv=dv, workspace=ws_b)
+        if ev is not None:
+            ev[2].record(stream)
+        cowa.cowa_decode(qd, k, v, seqlens, quad, out=od, lse=lsed, workspace=ws_d)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    cowa.cowa_get_device_error(dev)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = cowa.cowa_launch_count()
+    with ClockSampler(local_rank) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+    launches = cowa.cowa_launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    cowa.cowa_get_device_error(dev)
+
+    t_fwd = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    t_bwd = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    t_dec = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    t_step = sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps
+    t_step, t_fwd, t_bwd, t_dec = max_over_ranks([t_step, t_fwd, t_bwd, t_dec], world, dev)
+
+    pairs = visible_pairs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, quad)
+    dec_keys = decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, quad)
+    g = wl.Hq // wl.Hkv
+    flops_step = pairs * 14 * wl.d + dec_keys * g * 4 * wl.d
+    dec_bytes = dec_keys * 2 * wl.d * 2
+    value = flops_step * world / (t_step * 1e-3) / 1e12
+
+    # end to end through the public API from pinned host buffers
+    e2e = run_e2e(args, cowa, wl, q, k, v, do, qd, seqlens, quad, dev, stream, flush, world)
+    e2e["value"] = flops_step * world / (e2e.pop("ms") * 1e-3) / 1e12
+    e2e["unit"] = "TFLOP/s"
+
+    peaks, peak_src = load_peaks()
+    bwd_tflops = pairs * 10 * wl.d / (t_bwd * 1e-3) / 1e12
+    fwd_tflops = pairs * 4 * wl.d / (t_fwd * 1e-3) / 1e12
+    dec_gbs = dec_bytes / (t_dec * 1e-3) / 1e9
+    roofline = {
+        "kernel": "cowa_bwd (dK/dV + dQ passes)",
+        "bound": "tensor", "achieved": round(bwd_tflops, 2), "peak": peaks["bf16_tflops"],
+        "unit": "TFLOP/s", "frac": round(bwd_tflops / peaks["bf16_tflops"], 4),
+        "peak_source": "%s bf16_tflops (burst)" % peak_src,
+        "traffic": load_traffic("bwd", wl.name),
+        "algorithmic": "10*d flops per visible pair, %d pairs" % pairs,
+    }
+    result = {
+        "metric": "effective TFLOP/s on visible pairs (fwd/bwd) & decode GB/s, % of B200 roofline",
+        "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic N(0,1), seeded",
+        "config": {"workload": wl.name, "B": wl.B, "Lq": wl.Lq, "Lk": wl.Lk, "Hq": wl.Hq,
+                   "Hkv": wl.Hkv, "d": wl.d, "quad": list(quad),
+                   "step": "cowa_fwd + cowa_bwd + cowa_decode(last token, full K/V as cache)",
+                   "l2": "512 MiB write before every timed step",
+                   "parallelism": "dp%d (independent replicas)" % world},
+        "breakdown": {
+            "fwd_ms": round(t_fwd, 4), "fwd_tflops": round(fwd_tflops, 2),
+            "fwd_frac": round(fwd_tflops / peaks["bf16_tflops"], 4),
+            "bwd_ms": round(t_bwd, 4), "bwd_tflops": round(bwd_tflops, 2),
+            "bwd_frac": round(bwd_tflops / peaks["bf16_tflops"], 4),
+            "decode_ms": round(t_dec, 4), "decode_gbs": round(dec_gbs, 1),
+            "decode_frac": round(dec_gbs / peaks["hbm_gbs"], 4),
+            "visible_pairs": pairs, "decode_visible_keys": dec_keys,
+        },
+        "roofline": roofline,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+    }
+    if args.decode_workload:
+        result["decode_workload"] = run_decode_workload(args, cowa, dev, stream, flush, world, peaks, peak_src)
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = run_cpu_baseline(wl, q, k, v, do, quad, args.cpu_rows)
+    return result
+
+
+def run_e2e(args, cowa, wl, q, k, v, do, qd, seqlens, quad, dev, stream, flush, world):
+    import torch.distributed as dist
+    hq, hk, hv, hdo, hqd = (t.cpu().pin_memory() for t in (q, k, v, do, qd))
+    hsl = seqlens.cpu().pin_memory()
+    outs = {"o": torch.empty(q.shape, dtype=q.dtype).pin_memory(),
+            "dq": torch.empty(q.shape, dtype=q.dtype).pin_memory(),
+            "dk": torch.empty(k.shape, dtype=k.dtype).pin_memory(),
+            "dv": torch.empty(v.shape, dtype=v.dtype).pin_memory(),
+            "od": torch.empty(qd.shape, dtype=qd.dtype).pin_memory()}
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo, hqd, hsl))
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+
+    def e2e_step():
+        dq_, dk_, dv_, ddo, dqd = (t.to(dev, non_blocking=True) for t in (hq, hk, hv, hdo, hqd))
+        dsl = hsl.to(dev, non_blocking=True)
+        o, lse = cowa.cowa_fwd(dq_, dk_, dv_, quad)
+        g1, g2, g3 = cowa.cowa_bwd(dq_, dk_, dv_, o, lse, ddo, quad)
+        od, _ = cowa.cowa_decode(dqd, dk_, dv_, dsl, quad)
+        for name, t in (("o", o), ("dq", g1), ("dk", g2), ("dv", g3), ("od", od)):
+            outs[name].copy_(t, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        e2e_step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in evs) / args.steps], world, dev)[0]
+    return {"ms": ms, "ms_per_step": round(ms, 4),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "path": "pinned host -> device copies, cowa_fwd/bwd/decode, device -> pinned host"}
+
+
+def run_decode_workload(args, cowa, dev, stream, flush, world, peaks, peak_src):
+    """The 128K decode workload (B=16, Hq=32, Hkv=8, d=128), timed on its own."""
+    from structured_sparse_attention_block_b200.inputs import WORKLOADS, workload_inputs
+    wl = WORKLOADS["decode128k"]
+    q, kc, vc, sl = workload_inputs(wl, device=dev, seed=7)
+    out = torch.empty_like(q)
+    lse = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(cowa.cowa_decode_workspace_size(q, kc, wl.quad), dtype=torch.uint8, device=dev)
+    for _ in range(max(3, args.warmup)):
+        cowa.cowa_decode(q, kc, vc, sl, wl.quad, out=out, lse=lse, workspace=ws)
+    torch.cuda.synchronize()
+    n = max(args.steps, 10)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        flush.zero_()
+        evs[i][0].record(stream)
+        cowa.cowa_decode(q, kc, vc, sl, wl.quad, out=out, lse=lse, workspace=ws)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / n
+    keys = decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, wl.quad)
+    nbytes = keys * 2 * wl.d * 2
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del q, kc, vc
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "ms": round(ms, 4), "visible_kv_bytes": nbytes,
+            "GB/s": round(gbs, 1), "peak": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4),
+            "peak_source": "%s hbm_gbs" % peak_src,
+            "full_cache_bytes": wl.B * wl.Lk * wl.Hkv * wl.d * 2 * 2}
+
+
+# ------------------------------------------------------------ CPU oracle ----
+def oracle_sample(wl, q, k, v, do, quad, rows):
+    """The oracle on a bounded sample of the step: batch element 0, the last
+    `rows` query rows (a chunk of the same problem under bottom-right
+    alignment), forward + backward, plus one decode row per query head.
+    Returns (seconds, flops credited to the sample, threads)."""
+    from oracle import oracle
+    from structured_sparse_attention_block_b200.inputs import bf16_bits
+    Lq = wl.Lq
+    rows = min(rows, Lq)
+    qb = bf16_bits(q[:1, Lq - rows:])
+    kb, vb = bf16_bits(k[:1]), bf16_bits(v[:1])
+    db = bf16_bits(do[:1, Lq - rows:])
+    t0 = time.perf_counter()
+    oracle.fwd(qb, kb, vb, quad)
+    oracle.bwd(qb, kb, vb, db, quad)
+    oracle.decode(bf16_bits(q[:1, -1]), kb, vb, [wl.Lk], quad)
+    sec = time.perf_counter() - t0
+    pairs = visible_pairs(1, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, quad, rows=np.arange(Lq - rows, Lq))
+    dec = decode_visible_keys([wl.Lk], wl.Hkv, quad) * (wl.Hq // wl.Hkv)
+    flops = pairs * 14 * wl.d + dec * 4 * wl.d
+    return sec, flops, oracle.threads(), rows
+
+
+def run_cpu_baseline(wl, q, k, v, do, quad, rows):
+    sec, flops, thr, rows = oracle_sample(wl, q, k, v, do, quad, rows)
+    return {"value": flops / sec / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+            "seconds": round(sec, 2),
+            "sample": "batch 0, last %d of %d query rows, all heads: fp64 forward + backward "
+                      "+ one decode row per head" % (rows, wl.Lq)}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle as it stands, on host cores."""
+    if rank != 0:
+        return None
+    from structured_sparse_attention_block_b200.inputs import WORKLOADS, training_inputs
+    wl = WORKLOADS[args.workload]
+    q, k, v, do = training_inputs(1, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, wl.d, device="cpu", seed=0)
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(wl, q, k, v, do, wl.quad, rows)
+    secs, flops, thr = 0.0, 0, 1
+    for _ in range(args.steps):
+        s, f, thr, rows = oracle_sample(wl, q, k, v, do, wl.quad, rows)
+        secs += s
+        flops += f
+    value = flops / secs / 1e12
+    ms = secs / args.steps * 1e3
+    sample = ("batch 0, last %d of %d query rows, all heads: fp64 forward + backward + one "
+              "decode row per head" % (rows, wl.Lq))
+    return {
+        "impl": "reference",
+        "metric": "effective TFLOP/s on visible pairs (fwd/bwd) & decode GB/s, % of B200 roofline",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic N(0,1), seeded",
+        "config": {"workload": wl.name, "B": wl.B, "Lq": wl.Lq, "Lk": wl.Lk, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                   "d": wl.d, "quad": list(wl.quad), "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["cowa", "reference"], default="cowa")
+    ap.add_argument("--workload", default="recall8k")
+    ap.add_argument("--cpu-rows", type=int, default=4096, help="query rows in the CPU-baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=512, help="query rows per reference-arm step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode-workload", dest="decode_workload", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            raise SystemExit("--gpus %d needs torchrun with %d processes" % (args.gpus, args.gpus))
+        raise SystemExit("WORLD_SIZE=%d does not match --gpus %d" % (world, args.gpus))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_cowa(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

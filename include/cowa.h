@@ -1,0 +1,178 @@
+/*
+ * cowa.h -- C ABI of the CoWindow Attention (CoWA) library for B200 (sm_100a).
+ *
+ * CoWA is the position-defined, block-sparse causal attention of
+ * "CoWindow Attention: Full Causal Coverage Is a Collective Property"
+ * (abstract; paper digest, method key points).  Every KV head sees a shared
+ * prefix-sink window and a shared near-diagonal window, plus its own
+ * complementary long-range window; the long windows of the KV heads split the
+ * remaining history into equal-width slices, so the union over heads is the
+ * full causal prefix.  The windows are described by the quadruple
+ * (sink width S, near width N, gap G, long-range width W) and by
+ * bottom-right-aligned causal distance, used identically for training,
+ * prefill and decoding.
+ *
+ * Exact rule (the pages give no breakpoint formula; this library fixes it):
+ * for query row i of Lq and key j of Lk, p = i + Lk - Lq and d = p - j.
+ * Key j is visible to KV head h (global index) iff d >= 0 and
+ *     j < S   or   d < N   or   N+G+h*W <= d < N+G+(h+1)*W.
+ * Query head hq uses KV head floor(hq / (Hq/Hkv)) (contiguous GQA groups).
+ *
+ * Conventions for every entry point
+ *  - Tensors are bf16 in [B, L, H, d] order with the last dimension
+ *    contiguous; the other three strides are given in ELEMENTS and must be
+ *    multiples of 8 (16 bytes).  Base pointers must be 16-byte aligned.
+ *  - LSE is fp32, contiguous [B, Hq, Lq], natural logarithm; a query row
+ *    that sees no key gets O = 0 and LSE = -inf.
+ *  - d (head dimension) is 64 or 128.
+ *  - All device pointers are owned by the caller.  The library allocates no
+ *    memory: scratch space is the caller's workspace buffer, sized by the
+ *    matching *_workspace_size call, 256-byte aligned.
+ *  - Calls are asynchronous on the given CUDA stream (a cudaStream_t passed as
+ *    void*; NULL is the legacy default stream).  They return only
+ *    launch-time errors; they never abort or throw.  Kernel-side errors
+ *    (a bounded wait that ran out) are recorded in a device word that
+ *    cowa_get_device_error() reads.
+ *  - Thread safety: calls may be issued from several host threads; the
+ *    detail string of the last error is per thread.
+ */
+#ifndef COWA_H
+#define COWA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define COWA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define COWA_API __attribute__((visibility("default")))
+#else
+#define COWA_API
+#endif
+
+/* Window quadruple (sink width, near width, gap, long-range width), in keys. */
+typedef struct {
+    int32_t S, N, G, W;
+} cowa_quad_t;
+
+/*
+ * Problem shape.  Hkv is the number of KV heads present in the tensors;
+ * kv_head_offset is the global index of the first of them (0 on one GPU; a
+ * rank of a KV-head tensor-parallel group passes the index of its first head
+ * so the windows stay those of the global head, as the paper digest's
+ * execution notes describe).  Strides are in elements for (b, l, h).
+ */
+typedef struct {
+    int64_t B, Lq, Lk, Hq, Hkv, d;
+    int64_t q_stride[3];  /* Q, and dQ in cowa_bwd */
+    int64_t k_stride[3];  /* K, and dK in cowa_bwd */
+    int64_t v_stride[3];  /* V, and dV in cowa_bwd */
+    int64_t o_stride[3];  /* O, and dO in cowa_bwd */
+    int64_t kv_head_offset;
+} cowa_shape_t;
+
+typedef enum {
+    COWA_OK = 0,
+    COWA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, negative window */
+    COWA_ERR_UNSUPPORTED = 2,  /* head dim not 64/128, no sm_100 device */
+    COWA_ERR_ALIGNMENT = 3,    /* pointer or stride not 16-byte aligned */
+    COWA_ERR_WORKSPACE = 4,    /* workspace missing or too small */
+    COWA_ERR_CUDA = 5,         /* a CUDA runtime call failed */
+    COWA_ERR_TIMEOUT = 6,      /* a kernel's bounded wait ran out */
+    COWA_ERR_DEVICE = 7        /* a kernel's own consistency check failed */
+} cowa_status_t;
+
+/* Human-readable name of a status code (static string). */
+COWA_API const char *cowa_status_string(int status);
+
+/* Detail of the last error raised on this host thread ("" if none). */
+COWA_API const char *cowa_last_error_detail(void);
+
+/* ABI version of the loaded library (COWA_ABI_VERSION). */
+COWA_API int cowa_abi_version(void);
+
+/* Number of CUDA kernels this library has launched in this process. */
+COWA_API uint64_t cowa_launch_count(void);
+
+/*
+ * Default quadruple: G = 0 and W = ceil((Lk - N) / Hkv), clamped at 0, so
+ * the Hkv long windows exactly cover distances N .. Lk-1.  Hkv here is the
+ * GLOBAL number of KV heads.
+ */
+COWA_API cowa_quad_t cowa_default_quad(int64_t Lk, int64_t Hkv, int32_t S, int32_t N);
+
+/* Workspace bytes for each call (0 is never returned for a valid shape). */
+COWA_API size_t cowa_fwd_workspace_size(const cowa_shape_t *shape, cowa_quad_t quad);
+COWA_API size_t cowa_bwd_workspace_size(const cowa_shape_t *shape, cowa_quad_t quad);
+COWA_API size_t cowa_decode_workspace_size(const cowa_shape_t *shape, cowa_quad_t quad);
+
+/*
+ * Training / prefill forward (paper abstract: training forward pass).
+ *   q [B, Lq, Hq, d], k/v [B, Lk, Hkv, d] in; o [B, Lq, Hq, d] bf16 and
+ *   lse [B, Hq, Lq] fp32 out.  O_i = sum_j softmax_j(scale * q_i.k_j) v_j over
+ *   the keys visible to row i.  softmax_scale <= 0 selects 1/sqrt(d).
+ * Only key tiles that hold at least one visible pair are read ("block
+ * traversal skips invisible KV blocks", paper digest, execution notes).
+ */
+COWA_API int cowa_fwd(const cowa_shape_t *shape, cowa_quad_t quad, float softmax_scale,
+             const void *q, const void *k, const void *v, void *o, float *lse,
+             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Training backward (paper abstract: training backward pass).
+ *   Inputs q, k, v, o (the forward output), lse (the forward's), dO (o's
+ *   strides).  Outputs dq (q's strides), dk (k's strides), dv (v's strides),
+ *   bf16.  dK and dV sum the contributions of the query heads of each group.
+ *   Recomputes P = exp(scale*q.k - LSE) per visible tile; delta = rowsum(dO*O).
+ */
+COWA_API int cowa_bwd(const cowa_shape_t *shape, cowa_quad_t quad, float softmax_scale,
+             const void *q, const void *k, const void *v, const void *o,
+             const float *lse, const void *dout, void *dq, void *dk, void *dv,
+             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Single-token decode over a KV cache (paper abstract: decoding).
+ *   shape->Lq must be 1 and shape->Lk is the cache capacity Lcap.
+ *   q [B, 1, Hq, d]; k_cache / v_cache [B, Lcap, Hkv, d]; seqlens [B] int32
+ *   on the device, 0 <= seqlens[b] <= Lcap: keys 0 .. seqlens[b]-1 are valid
+ *   and the new token's own K/V is already stored at seqlens[b]-1, so the
+ *   query sits at p = seqlens[b]-1.  The quadruple is the model's (it is not
+ *   re-derived from the current length).  Out: o [B, 1, Hq, d] bf16 and
+ *   lse [B, Hq] fp32.  Only visible keys are read (split over the KV
+ *   sequence, then merged with LSE weights).
+ */
+COWA_API int cowa_decode(const cowa_shape_t *shape, cowa_quad_t quad, float softmax_scale,
+                const void *q, const void *k_cache, const void *v_cache,
+                const int32_t *seqlens, void *o, float *lse, void *workspace,
+                size_t workspace_bytes, void *stream);
+
+/*
+ * Visible-tile classes of one KV head, as the training kernels see them, for
+ * checking the schedule: writes out[qt * nkt + kt] (device, uint8) for the
+ * tiling BM x BN = (64 or 128) x 64, nqt = ceil(Lq/BM), nkt = ceil(Lk/BN):
+ *   0 = tile skipped, 1 = visited with the element mask applied,
+ *   2 = visited without a mask (every in-range pair visible).
+ * kv_head is the global KV-head index.  transposed = 0 uses the
+ * query-tile-major schedule (forward, dQ), 1 the key-tile-major schedule
+ * (dK/dV).  workspace as from cowa_schedule_workspace_size.
+ */
+COWA_API size_t cowa_schedule_workspace_size(int64_t Lq, int64_t Lk, int32_t BM, int32_t BN);
+COWA_API int cowa_tile_classes(int64_t Lq, int64_t Lk, int64_t kv_head, cowa_quad_t quad,
+                      int32_t BM, int32_t BN, int transposed, uint8_t *out,
+                      void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Reads and clears the device error word (synchronises the stream).
+ * Returns COWA_OK, COWA_ERR_TIMEOUT or COWA_ERR_DEVICE.
+ */
+COWA_API int cowa_get_device_error(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* COWA_H */

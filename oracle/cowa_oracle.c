@@ -405,3 +405,26 @@ void cowa_ref_decode(int64_t B, int64_t Lcap, int64_t Hq, int64_t Hkv,
         free(s);
     }
 }
+
+/*
+ * Brute-force visible-pair counts per tile of one window index, for checking
+ * the visible-tile schedule: out[qt * nkt + kt] = number of (i, j) with
+ * i in [qt*BM, min((qt+1)*BM, Lq)), j in [kt*BN, min((kt+1)*BN, Lk)) and key
+ * j visible to row i.
+ */
+void cowa_ref_tile_counts(int64_t Lq, int64_t Lk, int64_t w, int64_t S,
+                          int64_t N, int64_t G, int64_t W, int64_t BM,
+                          int64_t BN, int64_t *out)
+{
+    const int64_t nqt = (Lq + BM - 1) / BM, nkt = (Lk + BN - 1) / BN;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t qt = 0; qt < nqt; ++qt) {
+        for (int64_t kt = 0; kt < nkt; ++kt) out[qt * nkt + kt] = 0;
+        const int64_t i1 = (qt + 1) * BM < Lq ? (qt + 1) * BM : Lq;
+        for (int64_t i = qt * BM; i < i1; ++i) {
+            const int64_t p = i + Lk - Lq;
+            for (int64_t j = 0; j < Lk; ++j)
+                out[qt * nkt + j / BN] += cowa_ref_visible(p, j, w, S, N, G, W);
+        }
+    }
+}

@@ -41,6 +41,7 @@ def _load():
         _lib.cowa_ref_visible.argtypes = [_i64] * 7
         _lib.cowa_ref_visible.restype = ctypes.c_int
         _lib.cowa_ref_threads.restype = ctypes.c_int
+        _lib.cowa_ref_tile_counts.argtypes = [_i64] * 9 + [_ptr]
     return _lib
 
 
@@ -105,6 +106,14 @@ def mask(Lq, Lk, w, quad) -> np.ndarray:
     out = np.empty((Lq, Lk), dtype=np.uint8)
     _load().cowa_ref_mask(Lq, Lk, w, S, N, G, W, _p(out))
     return out.astype(bool)
+
+
+def tile_counts(Lq, Lk, w, quad, BM, BN) -> np.ndarray:
+    """int64 [ceil(Lq/BM), ceil(Lk/BN)]: visible pairs in each tile (brute force)."""
+    S, N, G, W = quad
+    out = np.zeros((-(-Lq // BM), -(-Lk // BN)), dtype=np.int64)
+    _load().cowa_ref_tile_counts(Lq, Lk, w, S, N, G, W, BM, BN, _p(out))
+    return out
 
 
 def fwd(q, k, v, quad, scale=None, kv_head_offset=0, widx=None):
@@ -217,5 +226,5 @@ def bits_to_f64(bits) -> np.ndarray:
     return b.view(np.float32).astype(np.float64)
 
 
-__all__ = ["threads", "default_quad", "visible", "mask", "fwd", "fwd_rows", "bwd",
+__all__ = ["threads", "default_quad", "visible", "mask", "tile_counts", "fwd", "fwd_rows", "bwd",
            "bwd_dq_rows", "bwd_dkv_cols", "decode", "bf16_bits", "bits_to_f64"]

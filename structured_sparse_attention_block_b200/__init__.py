@@ -1,0 +1,286 @@
+"""CoWindow Attention (CoWA) for B200: Python binding of ``libcowa.so``.
+
+Argument marshalling only.  Every step of the operator runs in the library's
+sm_100a kernels; PyTorch provides device memory and the current stream.
+There is no CPU or eager fallback: if the library is missing or the tensors
+are not on a CUDA device, the calls raise.
+
+Entry points (same names as the C ABI in ``include/cowa.h``):
+
+* ``cowa_fwd(q, k, v, quad)`` -> ``(o, lse)``: training / prefill forward,
+  q [B, Lq, Hq, d], k/v [B, Lk, Hkv, d] bf16; lse [B, Hq, Lq] fp32.
+* ``cowa_bwd(q, k, v, o, lse, dout, quad)`` -> ``(dq, dk, dv)``.
+* ``cowa_decode(q, k_cache, v_cache, seqlens, quad)`` -> ``(o, lse)``:
+  one new token per sequence, q [B, 1, Hq, d], caches [B, Lcap, Hkv, d],
+  seqlens int32 [B] on the device.
+* ``cowa_default_quad(Lk, Hkv, S, N)``: G = 0, W = ceil((Lk - N) / Hkv).
+* ``cowa_tile_classes(...)``: the visible-tile map the kernels use.
+
+The window quadruple ``quad`` is ``(S, N, G, W)``: sink width, near width,
+gap and long-range width ("CoWindow Attention: Full Causal Coverage Is a
+Collective Property", paper digest, method key points).
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = ["CowaError", "cowa_fwd", "cowa_bwd", "cowa_decode", "cowa_default_quad",
+           "cowa_tile_classes", "cowa_fwd_workspace_size", "cowa_bwd_workspace_size",
+           "cowa_decode_workspace_size", "cowa_get_device_error", "cowa_launch_count",
+           "library_path", "lib"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libcowa.so")
+_lib = None
+
+COWA_OK = 0
+_STATUS = {0: "COWA_OK", 1: "COWA_ERR_INVALID_ARG", 2: "COWA_ERR_UNSUPPORTED",
+           3: "COWA_ERR_ALIGNMENT", 4: "COWA_ERR_WORKSPACE", 5: "COWA_ERR_CUDA",
+           6: "COWA_ERR_TIMEOUT", 7: "COWA_ERR_DEVICE"}
+
+
+class CowaError(RuntimeError):
+    def __init__(self, status, detail):
+        self.status = status
+        super().__init__("%s: %s" % (_STATUS.get(status, status), detail))
+
+
+class Quad(ctypes.Structure):
+    _fields_ = [("S", ctypes.c_int32), ("N", ctypes.c_int32), ("G", ctypes.c_int32),
+                ("W", ctypes.c_int32)]
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("Lq", ctypes.c_int64), ("Lk", ctypes.c_int64),
+                ("Hq", ctypes.c_int64), ("Hkv", ctypes.c_int64), ("d", ctypes.c_int64),
+                ("q_stride", ctypes.c_int64 * 3), ("k_stride", ctypes.c_int64 * 3),
+                ("v_stride", ctypes.c_int64 * 3), ("o_stride", ctypes.c_int64 * 3),
+                ("kv_head_offset", ctypes.c_int64)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """The loaded ``libcowa.so``; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                "libcowa.so is missing at %s: build it with "
+                "`python -m structured_sparse_attention_block_b200.build`" % _LIB_PATH)
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, sz, i32, i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64
+        SP = ctypes.POINTER(Shape)
+        L.cowa_status_string.restype = ctypes.c_char_p
+        L.cowa_status_string.argtypes = [ctypes.c_int]
+        L.cowa_last_error_detail.restype = ctypes.c_char_p
+        L.cowa_abi_version.restype = ctypes.c_int
+        L.cowa_launch_count.restype = ctypes.c_uint64
+        L.cowa_default_quad.restype = Quad
+        L.cowa_default_quad.argtypes = [i64, i64, i32, i32]
+        for name in ("cowa_fwd_workspace_size", "cowa_bwd_workspace_size",
+                     "cowa_decode_workspace_size"):
+            f = getattr(L, name)
+            f.restype = sz
+            f.argtypes = [SP, Quad]
+        L.cowa_fwd.restype = ctypes.c_int
+        L.cowa_fwd.argtypes = [SP, Quad, ctypes.c_float, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.cowa_bwd.restype = ctypes.c_int
+        L.cowa_bwd.argtypes = [SP, Quad, ctypes.c_float] + [vp] * 9 + [vp, sz, vp]
+        L.cowa_decode.restype = ctypes.c_int
+        L.cowa_decode.argtypes = [SP, Quad, ctypes.c_float] + [vp] * 6 + [vp, sz, vp]
+        L.cowa_schedule_workspace_size.restype = sz
+        L.cowa_schedule_workspace_size.argtypes = [i64, i64, i32, i32]
+        L.cowa_tile_classes.restype = ctypes.c_int
+        L.cowa_tile_classes.argtypes = [i64, i64, i64, Quad, i32, i32, ctypes.c_int, vp, vp, sz, vp]
+        L.cowa_get_device_error.restype = ctypes.c_int
+        L.cowa_get_device_error.argtypes = [vp]
+        _lib = L
+    return _lib
+
+
+def _check(status):
+    if status != COWA_OK:
+        raise CowaError(status, lib().cowa_last_error_detail().decode())
+
+
+def _quad(quad) -> Quad:
+    if isinstance(quad, Quad):
+        return quad
+    S, N, G, W = (int(x) for x in quad)
+    return Quad(S, N, G, W)
+
+
+def cowa_default_quad(Lk, Hkv, S, N):
+    """(S, N, 0, ceil((Lk - N) / Hkv)) with W clamped at 0; Hkv is the global count."""
+    q = lib().cowa_default_quad(int(Lk), int(Hkv), int(S), int(N))
+    return (q.S, q.N, q.G, q.W)
+
+
+def _bf16_cuda(t, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != torch.bfloat16:
+        raise TypeError("%s must be bfloat16 (got %s)" % (name, t.dtype))
+    if t.dim() != 4 or (t.numel() > 0 and t.stride(3) != 1):
+        raise ValueError("%s must be [B, L, H, d] with a contiguous last dimension" % name)
+
+
+def _strides(t):
+    return (ctypes.c_int64 * 3)(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _shape(q, k, v, o, kv_head_offset):
+    B, Lq, Hq, d = q.shape
+    _, Lk, Hkv, _ = k.shape
+    return Shape(B, Lq, Lk, Hq, Hkv, d, _strides(q), _strides(k), _strides(v), _strides(o),
+                 int(kv_head_offset))
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None and t.numel() > 0 else None
+
+
+def _workspace(nbytes, device, workspace):
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError("workspace too small: need %d bytes" % nbytes)
+        return workspace
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def cowa_fwd_workspace_size(q, k, quad, kv_head_offset=0):
+    return int(lib().cowa_fwd_workspace_size(ctypes.byref(_shape(q, k, k, q, kv_head_offset)), _quad(quad)))
+
+
+def cowa_bwd_workspace_size(q, k, quad, kv_head_offset=0):
+    return int(lib().cowa_bwd_workspace_size(ctypes.byref(_shape(q, k, k, q, kv_head_offset)), _quad(quad)))
+
+
+def cowa_decode_workspace_size(q, k_cache, quad, kv_head_offset=0):
+    q4 = q if q.dim() == 4 else q.unsqueeze(1)
+    return int(lib().cowa_decode_workspace_size(
+        ctypes.byref(_shape(q4, k_cache, k_cache, q4, kv_head_offset)), _quad(quad)))
+
+
+def cowa_fwd(q, k, v, quad, softmax_scale=None, kv_head_offset=0, out=None, lse=None,
+             workspace=None):
+    """CoWA forward.  Returns ``(o, lse)``; see the module docstring."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bf16_cuda(t, n)
+    B, Lq, Hq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    _bf16_cuda(out, "out")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, Lq):
+        raise ValueError("lse must be contiguous fp32 [B, Hq, Lq]")
+    shape = _shape(q, k, v, out, kv_head_offset)
+    qd = _quad(quad)
+    L = lib()
+    need = L.cowa_fwd_workspace_size(ctypes.byref(shape), qd)
+    if need == 0:
+        _raise_size_error(L)
+    ws = _workspace(need, q.device, workspace)
+    scale = 0.0 if softmax_scale is None else float(softmax_scale)
+    _check(L.cowa_fwd(ctypes.byref(shape), qd, scale, _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                      _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)))
+    return out, lse
+
+
+def _raise_size_error(L):
+    """A workspace query returned 0: the arguments were rejected."""
+    detail = L.cowa_last_error_detail().decode()
+    raise CowaError(1, detail or "invalid arguments")
+
+
+def cowa_bwd(q, k, v, o, lse, dout, quad, softmax_scale=None, kv_head_offset=0,
+             dq=None, dk=None, dv=None, workspace=None):
+    """CoWA backward.  Returns ``(dq, dk, dv)``; dO uses o's strides, dQ q's,
+    dK k's and dV v's (pass dq/dk/dv to choose them)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _bf16_cuda(t, n)
+    if dout.stride() != o.stride():
+        raise ValueError("dout must have the strides of o")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, ref, n in ((dq, q, "dq"), (dk, k, "dk"), (dv, v, "dv")):
+        _bf16_cuda(t, n)
+        if t.stride() != ref.stride() or t.shape != ref.shape:
+            raise ValueError("%s must match the shape and strides of its input" % n)
+    B, Lq, Hq, d = q.shape
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, Lq):
+        raise ValueError("lse must be contiguous fp32 [B, Hq, Lq]")
+    shape = _shape(q, k, v, o, kv_head_offset)
+    qd = _quad(quad)
+    L = lib()
+    need = L.cowa_bwd_workspace_size(ctypes.byref(shape), qd)
+    if need == 0:
+        _raise_size_error(L)
+    ws = _workspace(need, q.device, workspace)
+    scale = 0.0 if softmax_scale is None else float(softmax_scale)
+    _check(L.cowa_bwd(ctypes.byref(shape), qd, scale, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                      _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
+                      _stream(q.device)))
+    return dq, dk, dv
+
+
+def cowa_decode(q, k_cache, v_cache, seqlens, quad, softmax_scale=None, kv_head_offset=0,
+                out=None, lse=None, workspace=None):
+    """CoWA single-token decode.  q [B, 1, Hq, d] (or [B, Hq, d]); returns
+    ``(o [B, 1, Hq, d], lse [B, Hq])``."""
+    q4 = q if q.dim() == 4 else q.unsqueeze(1)
+    for t, n in ((q4, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _bf16_cuda(t, n)
+    if seqlens.dtype != torch.int32 or not seqlens.is_cuda or not seqlens.is_contiguous():
+        raise TypeError("seqlens must be a contiguous int32 CUDA tensor")
+    B, _, Hq, d = q4.shape
+    if out is None:
+        out = torch.empty((B, 1, Hq, d), dtype=torch.bfloat16, device=q4.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q4.device)
+    _bf16_cuda(out, "out")
+    shape = _shape(q4, k_cache, v_cache, out, kv_head_offset)
+    qd = _quad(quad)
+    L = lib()
+    need = L.cowa_decode_workspace_size(ctypes.byref(shape), qd)
+    if need == 0:
+        _raise_size_error(L)
+    ws = _workspace(need, q4.device, workspace)
+    scale = 0.0 if softmax_scale is None else float(softmax_scale)
+    _check(L.cowa_decode(ctypes.byref(shape), qd, scale, _ptr(q4), _ptr(k_cache), _ptr(v_cache),
+                         _ptr(seqlens), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                         _stream(q4.device)))
+    return out, lse
+
+
+def cowa_tile_classes(Lq, Lk, kv_head, quad, BM, BN=64, transposed=False, device="cuda"):
+    """uint8 [ceil(Lq/BM), ceil(Lk/BN)]: 0 skipped, 1 masked, 2 unmasked tile."""
+    L = lib()
+    nqt, nkt = -(-Lq // BM), -(-Lk // BN)
+    out = torch.empty((nqt, nkt), dtype=torch.uint8, device=device)
+    need = L.cowa_schedule_workspace_size(Lq, Lk, BM, BN)
+    ws = torch.empty(max(int(need), 1), dtype=torch.uint8, device=device)
+    _check(L.cowa_tile_classes(Lq, Lk, kv_head, _quad(quad), BM, BN, int(bool(transposed)),
+                               _ptr(out), _ptr(ws), ws.numel(), _stream(torch.device(device))))
+    return out
+
+
+def cowa_launch_count() -> int:
+    """Kernels the library has launched in this process (all devices)."""
+    return int(lib().cowa_launch_count())
+
+
+def cowa_get_device_error(device=None):
+    """Synchronise and raise if a kernel recorded a device-side error."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    _check(lib().cowa_get_device_error(_stream(dev)))

@@ -1,0 +1,388 @@
+// C ABI of the CoWA library: argument checks, workspace carving and kernel
+// launches.  Declarations and contracts are in include/cowa.h.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/cowa.h"
+#include "common.cuh"
+#include "kernels.cuh"
+
+#include <atomic>
+
+namespace cowa {
+__device__ int g_cowa_device_error = 0;
+
+static std::atomic<unsigned long long> g_launches{0};
+void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+}
+
+namespace {
+
+thread_local char tl_detail[256] = "";
+
+int fail(int status, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(tl_detail, sizeof tl_detail, fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(COWA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+struct DeviceInfo {
+    int checked = 0, ok = 0, sms = 148;
+    int *err = nullptr;  // device address of the error word on this device
+};
+DeviceInfo g_dev[64];
+
+int check_device(int *sms)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    DeviceInfo &di = g_dev[dev & 63];
+    if (!di.checked) {
+        int major = 0, minor = 0, sm = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        cudaDeviceGetAttribute(&sm, cudaDevAttrMultiProcessorCount, dev);
+        di.ok = (major == 10 && minor == 0);
+        di.sms = sm > 0 ? sm : 148;
+        if (di.ok) {
+            e = cudaGetSymbolAddress((void **)&di.err, cowa::g_cowa_device_error);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+        }
+        di.checked = 1;
+    }
+    if (!di.ok) return fail(COWA_ERR_UNSUPPORTED, "device %d is not sm_100 (B200)", dev);
+    if (sms) *sms = di.sms;
+    return COWA_OK;
+}
+
+int *device_error_word()
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return g_dev[dev & 63].err;
+}
+
+constexpr long long kMaxLen = 1ll << 30;
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int check_quad(cowa_quad_t q)
+{
+    if (q.S < 0 || q.N < 0 || q.G < 0 || q.W < 0)
+        return fail(COWA_ERR_INVALID_ARG, "window quadruple (%d,%d,%d,%d) has a negative field",
+                    q.S, q.N, q.G, q.W);
+    return COWA_OK;
+}
+
+int check_strides(const int64_t *st, const char *name)
+{
+    for (int a = 0; a < 3; ++a)
+        if (st[a] < 0 || st[a] % 8)
+            return fail(COWA_ERR_ALIGNMENT, "%s stride[%d] = %lld is not a non-negative multiple of 8 elements",
+                        name, a, (long long)st[a]);
+    return COWA_OK;
+}
+
+int check_ptr(const void *p, bool needed, const char *name)
+{
+    if (!needed) return COWA_OK;
+    if (!p) return fail(COWA_ERR_INVALID_ARG, "%s is NULL", name);
+    if ((uintptr_t)p % 16) return fail(COWA_ERR_ALIGNMENT, "%s is not 16-byte aligned", name);
+    return COWA_OK;
+}
+
+int check_shape(const cowa_shape_t *s, cowa_quad_t q, bool decode)
+{
+    if (!s) return fail(COWA_ERR_INVALID_ARG, "shape is NULL");
+    if (s->B < 0 || s->Lq < 0 || s->Lk < 0 || s->Hq < 0 || s->Hkv < 0 || s->kv_head_offset < 0)
+        return fail(COWA_ERR_INVALID_ARG, "negative size in shape");
+    if (s->Lq >= kMaxLen || s->Lk >= kMaxLen || s->B > 65535 || s->Hq > 65535 || s->Hkv > 65535)
+        return fail(COWA_ERR_UNSUPPORTED, "sequence length must be < 2^30, B/heads <= 65535");
+    if (s->Hq > 0 && (s->Hkv == 0 || s->Hq % s->Hkv))
+        return fail(COWA_ERR_INVALID_ARG, "Hq=%lld is not a multiple of Hkv=%lld", (long long)s->Hq,
+                    (long long)s->Hkv);
+    if (s->d != 64 && s->d != 128)
+        return fail(COWA_ERR_UNSUPPORTED, "head dim %lld (supported: 64, 128)", (long long)s->d);
+    if (s->kv_head_offset + s->Hkv > kMaxLen)
+        return fail(COWA_ERR_INVALID_ARG, "kv_head_offset too large");
+    int r = check_quad(q);
+    if (r) return r;
+    if ((r = check_strides(s->q_stride, "q")) || (r = check_strides(s->k_stride, "k")) ||
+        (r = check_strides(s->v_stride, "v")) || (r = check_strides(s->o_stride, "o")))
+        return r;
+    if (decode) {
+        if (s->Lq != 1) return fail(COWA_ERR_INVALID_ARG, "decode needs Lq == 1 (got %lld)", (long long)s->Lq);
+        if (s->Hkv > 0 && s->Hq / s->Hkv > 16)
+            return fail(COWA_ERR_UNSUPPORTED, "decode supports up to 16 query heads per KV head");
+    }
+    return COWA_OK;
+}
+
+float resolve_scale(float scale, int64_t d) { return scale > 0.f ? scale : 1.0f / sqrtf((float)d); }
+
+template <typename P>
+void fill_common(P &p, const cowa_shape_t *s, cowa_quad_t q, float scale)
+{
+    for (int a = 0; a < 3; ++a) {
+        p.qs[a] = s->q_stride[a];
+        p.ks[a] = s->k_stride[a];
+        p.vs[a] = s->v_stride[a];
+        p.os[a] = s->o_stride[a];
+    }
+    p.Hq = (int)s->Hq;
+    p.Hkv = (int)s->Hkv;
+    p.g = s->Hkv > 0 ? (int)(s->Hq / s->Hkv) : 1;
+    p.S = q.S; p.N = q.N; p.G = q.G; p.W = q.W;
+    p.kv_head_offset = (int)s->kv_head_offset;
+    p.scale = resolve_scale(scale, s->d);
+    p.scale_log2 = p.scale * 1.4426950408889634f;
+    p.err = device_error_word();
+}
+
+size_t sched_bytes(long long heads, long long tiles) { return align256((size_t)(heads * tiles) * 8 * sizeof(int)); }
+
+long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+int decode_splits(const cowa_shape_t *s, cowa_quad_t q, int sms)
+{
+    const long long pairs = s->B * s->Hkv;
+    if (pairs <= 0) return 1;
+    long long keys = (long long)q.S + q.N + q.W;
+    if (keys > s->Lk) keys = s->Lk;
+    const long long tiles = cdiv(keys, cowa::kDecBN) + 3;
+    long long sp = cdiv(4ll * sms, pairs);
+    if (sp > tiles) sp = tiles;
+    if (sp > 64) sp = 64;
+    if (sp < 1) sp = 1;
+    return (int)sp;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *cowa_status_string(int status)
+{
+    switch (status) {
+    case COWA_OK: return "COWA_OK";
+    case COWA_ERR_INVALID_ARG: return "COWA_ERR_INVALID_ARG";
+    case COWA_ERR_UNSUPPORTED: return "COWA_ERR_UNSUPPORTED";
+    case COWA_ERR_ALIGNMENT: return "COWA_ERR_ALIGNMENT";
+    case COWA_ERR_WORKSPACE: return "COWA_ERR_WORKSPACE";
+    case COWA_ERR_CUDA: return "COWA_ERR_CUDA";
+    case COWA_ERR_TIMEOUT: return "COWA_ERR_TIMEOUT";
+    case COWA_ERR_DEVICE: return "COWA_ERR_DEVICE";
+    default: return "COWA_ERR_UNKNOWN";
+    }
+}
+
+const char *cowa_last_error_detail(void) { return tl_detail; }
+
+int cowa_abi_version(void) { return COWA_ABI_VERSION; }
+
+uint64_t cowa_launch_count(void) { return cowa::g_launches.load(std::memory_order_relaxed); }
+
+cowa_quad_t cowa_default_quad(int64_t Lk, int64_t Hkv, int32_t S, int32_t N)
+{
+    cowa_quad_t q;
+    q.S = S;
+    q.N = N;
+    q.G = 0;
+    long long rest = (long long)Lk - N;
+    long long W = (Hkv > 0 && rest > 0) ? cdiv(rest, Hkv) : 0;
+    q.W = (int32_t)(W > 0x7fffffff ? 0x7fffffff : W);
+    return q;
+}
+
+size_t cowa_fwd_workspace_size(const cowa_shape_t *s, cowa_quad_t q)
+{
+    if (check_shape(s, q, false)) return 0;
+    return sched_bytes(s->Hkv, cdiv(s->Lq, cowa::kFwdBM)) + 256;
+}
+
+size_t cowa_bwd_workspace_size(const cowa_shape_t *s, cowa_quad_t q)
+{
+    if (check_shape(s, q, false)) return 0;
+    return align256((size_t)(s->B * s->Hq * s->Lq) * sizeof(float)) +
+           sched_bytes(s->Hkv, cdiv(s->Lq, cowa::kBwdBM)) +
+           sched_bytes(s->Hkv, cdiv(s->Lk, cowa::kBwdBN)) + 256;
+}
+
+size_t cowa_decode_workspace_size(const cowa_shape_t *s, cowa_quad_t q)
+{
+    if (check_shape(s, q, true)) return 0;
+    int sms = 148;
+    if (check_device(&sms)) return 0;
+    const long long sp = decode_splits(s, q, sms);
+    const long long rows = s->B * s->Hq * sp;
+    return align256((size_t)(rows * s->d) * sizeof(float)) + align256((size_t)rows * sizeof(float)) + 256;
+}
+
+int cowa_fwd(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const void *q, const void *k,
+             const void *v, void *o, float *lse, void *ws, size_t ws_bytes, void *stream)
+{
+    int r = check_shape(s, quad, false);
+    if (r) return r;
+    const bool qrows = s->B * s->Lq * s->Hq > 0, krows = s->B * s->Lk * s->Hkv > 0;
+    if ((r = check_ptr(q, qrows, "q")) || (r = check_ptr(k, qrows && krows, "k")) ||
+        (r = check_ptr(v, qrows && krows, "v")) || (r = check_ptr(o, qrows, "o")) ||
+        (r = check_ptr(lse, qrows, "lse")))
+        return r;
+    if (!qrows) return COWA_OK;
+    if ((r = check_device(nullptr))) return r;
+    const size_t need = cowa_fwd_workspace_size(s, quad);
+    if (!ws || ws_bytes < need || (uintptr_t)ws % 256)
+        return fail(COWA_ERR_WORKSPACE, "fwd workspace needs %zu bytes, 256-byte aligned (got %zu)", need, ws_bytes);
+    cudaStream_t st = (cudaStream_t)stream;
+    cowa::AttnParams p{};
+    fill_common(p, s, quad, softmax_scale);
+    p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
+    p.B = (int)s->B; p.Lq = (int)s->Lq; p.Lk = (int)s->Lk;
+    p.nqt = (int)cdiv(s->Lq, cowa::kFwdBM);
+    p.nkt = (int)cdiv(s->Lk, cowa::kFwdBN);
+    int *sched = (int *)ws;
+    p.sched = sched;
+    cudaError_t e = cowa::launch_schedule(sched, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W,
+                                          cowa::kFwdBM, cowa::kFwdBN, 0, st);
+    if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+    e = cowa::launch_fwd_mma(p, (int)s->d, st);
+    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    return COWA_OK;
+}
+
+int cowa_bwd(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const void *q, const void *k,
+             const void *v, const void *o, const float *lse, const void *dout, void *dq, void *dk, void *dv,
+             void *ws, size_t ws_bytes, void *stream)
+{
+    int r = check_shape(s, quad, false);
+    if (r) return r;
+    const bool qrows = s->B * s->Lq * s->Hq > 0, krows = s->B * s->Lk * s->Hkv > 0;
+    if ((r = check_ptr(q, qrows, "q")) || (r = check_ptr(k, krows, "k")) || (r = check_ptr(v, krows, "v")) ||
+        (r = check_ptr(o, qrows, "o")) || (r = check_ptr(lse, qrows, "lse")) ||
+        (r = check_ptr(dout, qrows, "dout")) || (r = check_ptr(dq, qrows, "dq")) ||
+        (r = check_ptr(dk, krows, "dk")) || (r = check_ptr(dv, krows, "dv")))
+        return r;
+    if (!qrows && !krows) return COWA_OK;
+    if ((r = check_device(nullptr))) return r;
+    const size_t need = cowa_bwd_workspace_size(s, quad);
+    if (!ws || ws_bytes < need || (uintptr_t)ws % 256)
+        return fail(COWA_ERR_WORKSPACE, "bwd workspace needs %zu bytes, 256-byte aligned (got %zu)", need, ws_bytes);
+    cudaStream_t st = (cudaStream_t)stream;
+    cowa::AttnParams p{};
+    fill_common(p, s, quad, softmax_scale);
+    p.q = q; p.k = k; p.v = v; p.o = (void *)o; p.lse_in = lse; p.dout = dout;
+    p.dq = dq; p.dk = dk; p.dv = dv;
+    p.B = (int)s->B; p.Lq = (int)s->Lq; p.Lk = (int)s->Lk;
+    const int QB = cowa::bwd_kv_qtile((int)s->d);
+    p.nqt = (int)cdiv(s->Lq, cowa::kBwdBM);
+    p.nkt = (int)cdiv(s->Lk, cowa::kBwdBN);
+    char *w = (char *)ws;
+    p.delta = (float *)w;
+    w += align256((size_t)(s->B * s->Hq * s->Lq) * sizeof(float));
+    int *sched_q = (int *)w;
+    w += sched_bytes(s->Hkv, p.nqt);
+    int *sched_t = (int *)w;
+    p.sched = sched_q;
+    p.sched_t = sched_t;
+    cudaError_t e = cowa::launch_schedule(sched_q, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W,
+                                          cowa::kBwdBM, cowa::kBwdBN, 0, st);
+    if (e == cudaSuccess)
+        e = cowa::launch_schedule(sched_t, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W, QB,
+                                  cowa::kBwdBN, 1, st);
+    if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+    e = cowa::launch_bwd_mma(p, (int)s->d, st);
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    return COWA_OK;
+}
+
+int cowa_decode(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const void *q, const void *k_cache,
+                const void *v_cache, const int32_t *seqlens, void *o, float *lse, void *ws, size_t ws_bytes,
+                void *stream)
+{
+    int r = check_shape(s, quad, true);
+    if (r) return r;
+    const bool rows = s->B * s->Hq > 0, cache = s->B * s->Lk * s->Hkv > 0;
+    if ((r = check_ptr(q, rows, "q")) || (r = check_ptr(k_cache, rows && cache, "k_cache")) ||
+        (r = check_ptr(v_cache, rows && cache, "v_cache")) || (r = check_ptr(o, rows, "o")) ||
+        (r = check_ptr(lse, rows, "lse")))
+        return r;
+    if (rows && !seqlens) return fail(COWA_ERR_INVALID_ARG, "seqlens is NULL");
+    if (!rows) return COWA_OK;
+    int sms = 148;
+    if ((r = check_device(&sms))) return r;
+    const size_t need = cowa_decode_workspace_size(s, quad);
+    if (!ws || ws_bytes < need || (uintptr_t)ws % 256)
+        return fail(COWA_ERR_WORKSPACE, "decode workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
+                    ws_bytes);
+    cowa::DecodeParams p{};
+    fill_common(p, s, quad, softmax_scale);
+    p.q = q; p.kc = k_cache; p.vc = v_cache; p.seqlens = seqlens; p.o = o; p.lse = lse;
+    p.B = (int)s->B;
+    p.Lcap = (int)s->Lk;
+    p.splits = decode_splits(s, quad, sms);
+    const size_t rows_p = (size_t)(s->B * s->Hq * p.splits);
+    p.part_o = (float *)ws;
+    p.part_lse = (float *)((char *)ws + align256(rows_p * s->d * sizeof(float)));
+    cudaError_t e = cowa::launch_decode(p, (int)s->d, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return COWA_OK;
+}
+
+size_t cowa_schedule_workspace_size(int64_t Lq, int64_t Lk, int32_t BM, int32_t BN)
+{
+    if (Lq < 0 || Lk < 0 || BM <= 0 || BN <= 0) return 0;
+    const long long n = cdiv(Lq, BM) > cdiv(Lk, BN) ? cdiv(Lq, BM) : cdiv(Lk, BN);
+    return sched_bytes(1, n) + 256;
+}
+
+int cowa_tile_classes(int64_t Lq, int64_t Lk, int64_t kv_head, cowa_quad_t quad, int32_t BM, int32_t BN,
+                      int transposed, uint8_t *out, void *ws, size_t ws_bytes, void *stream)
+{
+    int r = check_quad(quad);
+    if (r) return r;
+    if (Lq < 0 || Lk < 0 || Lq >= kMaxLen || Lk >= kMaxLen || kv_head < 0 || kv_head >= kMaxLen)
+        return fail(COWA_ERR_INVALID_ARG, "bad length or head");
+    if ((BM != 64 && BM != 128 && BM != 32) || BN != 64)
+        return fail(COWA_ERR_UNSUPPORTED, "tiling %dx%d (supported: 32/64/128 x 64)", BM, BN);
+    if (Lq == 0 || Lk == 0) return COWA_OK;
+    if (!out) return fail(COWA_ERR_INVALID_ARG, "out is NULL");
+    if ((r = check_device(nullptr))) return r;
+    const size_t need = cowa_schedule_workspace_size(Lq, Lk, BM, BN);
+    if (!ws || ws_bytes < need || (uintptr_t)ws % 256)
+        return fail(COWA_ERR_WORKSPACE, "schedule workspace needs %zu bytes", need);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cowa::launch_schedule((int *)ws, 1, (int)kv_head, (int)Lq, (int)Lk, quad.S, quad.N, quad.G,
+                                          quad.W, BM, BN, transposed ? 1 : 0, st);
+    if (e == cudaSuccess)
+        e = cowa::launch_tile_classes((const int *)ws, out, (int)kv_head, (int)Lq, (int)Lk, quad.S, quad.N, quad.G,
+                                      quad.W, BM, BN, transposed ? 1 : 0, st);
+    if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+    return COWA_OK;
+}
+
+int cowa_get_device_error(void *stream)
+{
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, cowa::g_cowa_device_error, sizeof v);
+    if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+    e = cudaMemcpyToSymbol(cowa::g_cowa_device_error, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+    if (v == COWA_ERR_TIMEOUT) return fail(COWA_ERR_TIMEOUT, "a kernel's bounded wait ran out");
+    if (v) return fail(COWA_ERR_DEVICE, "a kernel's device-side check failed (code %d)", v);
+    return COWA_OK;
+}
+
+}  // extern "C"

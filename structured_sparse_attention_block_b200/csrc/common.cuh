@@ -1,0 +1,241 @@
+// Device-side building blocks of the CoWA library: window geometry, the
+// visible-tile schedule, and thin wrappers over PTX instructions.
+//
+// Window rule ("CoWindow Attention: Full Causal Coverage Is a Collective
+// Property", paper digest, method key points; breakpoints fixed by this
+// library): for aligned query position p = i + Lk - Lq and key j,
+// d = p - j; visible iff d >= 0 and (j < S or d < N or c <= d < e) with
+// c = N + G + h*W, e = c + W for the global KV head h.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace cowa {
+
+constexpr int kMaxRanges = 3;
+constexpr int kSchedInts = 8;  // n, lo0, hi0, lo1, hi1, lo2, hi2, pad
+
+// Per-head window geometry in 32-bit key units; [c, e) is the long window's
+// distance range, clamped so that nothing overflows (a window starting past
+// any reachable distance is empty).
+struct Win {
+    int S, N, c, e;
+};
+
+__host__ __device__ inline Win make_win(int S, int N, int G, int W, long long h)
+{
+    const long long big = 1ll << 30;
+    long long c = (long long)N + G + h * (long long)W;
+    long long e = c + W;
+    Win w;
+    w.S = S < big ? S : (int)big;
+    w.N = N < big ? N : (int)big;
+    w.c = (int)(c < big ? c : big);
+    w.e = (int)(e < big ? e : big);
+    return w;
+}
+
+__host__ __device__ __forceinline__ bool visible(int p, int j, const Win &w)
+{
+    const int d = p - j;
+    return d >= 0 && (j < w.S || d < w.N || (d >= w.c && d < w.e));
+}
+
+struct Ranges {
+    int n;
+    int lo[kMaxRanges], hi[kMaxRanges];
+};
+
+// Sort up to three half-open tile ranges and merge those that overlap or touch.
+__host__ __device__ inline void merge_ranges(Ranges &r)
+{
+    for (int a = 0; a < r.n; ++a)
+        for (int b = a + 1; b < r.n; ++b)
+            if (r.lo[b] < r.lo[a]) {
+                int t = r.lo[a]; r.lo[a] = r.lo[b]; r.lo[b] = t;
+                t = r.hi[a]; r.hi[a] = r.hi[b]; r.hi[b] = t;
+            }
+    int m = 0;
+    for (int a = 0; a < r.n; ++a) {
+        if (m > 0 && r.lo[a] <= r.hi[m - 1]) {
+            if (r.hi[a] > r.hi[m - 1]) r.hi[m - 1] = r.hi[a];
+        } else {
+            r.lo[m] = r.lo[a];
+            r.hi[m] = r.hi[a];
+            ++m;
+        }
+    }
+    r.n = m;
+}
+
+__host__ __device__ __forceinline__ void push_keys(Ranges &r, int a, int b, int BN)
+{
+    // key interval [a, b] inclusive -> tile range
+    if (a <= b) {
+        r.lo[r.n] = a / BN;
+        r.hi[r.n] = b / BN + 1;
+        ++r.n;
+    }
+}
+
+// Key tiles visited by a query tile whose in-range rows have aligned
+// positions pa..pb: the union over rows of the sink, near and long key
+// intervals, each contiguous, so every listed tile holds a visible pair.
+__host__ __device__ inline Ranges query_tile_ranges(int pa, int pb, const Win &w, int BN)
+{
+    Ranges r;
+    r.n = 0;
+    if (pb < 0) return r;
+    const int pa0 = pa > 0 ? pa : 0;
+    if (w.S > 0) push_keys(r, 0, w.S - 1 < pb ? w.S - 1 : pb, BN);
+    if (w.N > 0) push_keys(r, pa0 - w.N + 1 > 0 ? pa0 - w.N + 1 : 0, pb, BN);
+    if (w.e > w.c && pb - w.c >= 0) {
+        const int a = pa0 - (w.e - 1);
+        push_keys(r, a > 0 ? a : 0, pb - w.c, BN);
+    }
+    merge_ranges(r);
+    return r;
+}
+
+__host__ __device__ __forceinline__ void push_rows(Ranges &r, long long lo, long long hi,
+                                                   long long pmin, long long pmax,
+                                                   long long delta, int BM)
+{
+    // aligned-position interval [lo, hi] -> query tile range
+    if (lo < pmin) lo = pmin;
+    if (hi > pmax) hi = pmax;
+    if (lo <= hi) {
+        r.lo[r.n] = (int)((lo - delta) / BM);
+        r.hi[r.n] = (int)((hi - delta) / BM) + 1;
+        ++r.n;
+    }
+}
+
+// Query tiles that see key tile [c0, c1] (c1 clipped to Lk-1).  Rows sit at
+// p = i + delta with delta = Lk - Lq; valid p is [max(delta, 0), Lk-1].
+__host__ __device__ inline Ranges key_tile_ranges(int c0, int c1, int Lq, int Lk,
+                                                  const Win &w, int BM)
+{
+    Ranges r;
+    r.n = 0;
+    const long long delta = (long long)Lk - Lq;
+    const long long pmin = delta > 0 ? delta : 0, pmax = (long long)Lk - 1;
+    if (c0 < w.S) push_rows(r, c0, pmax, pmin, pmax, delta, BM);
+    if (w.N > 0) push_rows(r, c0, (long long)c1 + w.N - 1, pmin, pmax, delta, BM);
+    if (w.e > w.c) push_rows(r, (long long)c0 + w.c, (long long)c1 + w.e - 1, pmin, pmax, delta, BM);
+    merge_ranges(r);
+    return r;
+}
+
+// True when every pair of the tile (rows pa..pb, all in range; columns
+// c0..c0+BN-1) is visible, so the tile needs no element mask.  Per column
+// j >= S the rows that see it form j + D with D = [0,N) u [c,e); a row
+// range fits one connected part [a,b] of D iff j lies in [pb-b, pa-a].  Sink
+// columns j < S need j <= pa.  The tile is full iff its columns are covered
+// by the union of those column intervals.
+__host__ __device__ inline bool tile_full(int pa, int pb, int c0, int BN, int Lk, const Win &w)
+{
+    const int c1 = c0 + BN - 1;
+    if (c1 >= Lk || pa < 0) return false;
+    int lo[3], hi[3], n = 0;
+    if (w.S > 0) { lo[n] = 0; hi[n] = w.S - 1 < pa ? w.S - 1 : pa; ++n; }
+    const bool has_near = w.N > 0, has_long = w.e > w.c;
+    if (has_near && has_long && w.c <= w.N) {  // near and long windows touch
+        lo[n] = pb - (w.e - 1); hi[n] = pa; ++n;
+    } else {
+        if (has_near) { lo[n] = pb - (w.N - 1); hi[n] = pa; ++n; }
+        if (has_long) { lo[n] = pb - (w.e - 1); hi[n] = pa - w.c; ++n; }
+    }
+    for (int a = (w.S > 0 ? 1 : 0); a < n; ++a)
+        if (lo[a] < w.S) lo[a] = w.S;
+    // greedy cover of [c0, c1]
+    int x = c0;
+    for (int pass = 0; pass < 3; ++pass)
+        for (int a = 0; a < n; ++a)
+            if (lo[a] <= hi[a] && lo[a] <= x && x <= hi[a]) x = hi[a] + 1;
+    return x > c1;
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers (sm_80+ forms that sm_100a keeps: cp.async, ldmatrix, mma.sync)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid)
+{
+    const int n = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t r[4], uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t r[4], uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + D, fp32 accumulate.
+__device__ __forceinline__ void mma16816(float c[4], const uint32_t a[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
+        "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Offset (in elements) of element (r, c) of a [rows][D] bf16 tile whose
+// 16-byte chunks are XOR-swizzled by the row index, so that ldmatrix of 8
+// consecutive rows at one column touches 8 distinct bank groups.
+template <int D>
+__device__ __forceinline__ int swz(int r, int c)
+{
+    return r * D + ((((c >> 3) ^ (r & 7))) << 3) + (c & 7);
+}
+
+// Copy a [rows][D] bf16 tile from global memory (row pointer stride in
+// elements) into a swizzled shared tile; rows >= nvalid are zero-filled.
+template <int D, int ROWS, int NTHREADS>
+__device__ __forceinline__ void load_tile(__nv_bfloat16 *sm, const __nv_bfloat16 *g,
+                                          long long row_stride, int nvalid, int tid)
+{
+    constexpr int CPR = D / 8;  // 16-byte chunks per row
+    constexpr int TOTAL = ROWS * CPR;
+    const uint32_t base = smem_u32(sm);
+#pragma unroll
+    for (int it = 0; it < (TOTAL + NTHREADS - 1) / NTHREADS; ++it) {
+        const int idx = it * NTHREADS + tid;
+        if (TOTAL % NTHREADS == 0 || idx < TOTAL) {
+            const int r = idx / CPR, ch = idx % CPR;
+            const bool ok = r < nvalid;
+            const __nv_bfloat16 *src = g + (ok ? (long long)r * row_stride : 0) + ch * 8;
+            cp_async16(base + 2u * (uint32_t)swz<D>(r, ch * 8), src, ok);
+        }
+    }
+}
+
+}  // namespace cowa

@@ -1,0 +1,297 @@
+// CoWA single-token decode: split-KV over the visible keys, then an
+// LSE-weighted merge.
+//
+// The new token sits at p = seqlens[b] - 1 of its sequence.  The keys it sees
+// under KV head h are at most three intervals (sink [0, S), near (p-N, p],
+// long [p-e+1, p-c]); they are merged, cut into 64-key tiles that start at
+// each interval's first key, and the tiles are shared out over `splits` CTAs
+// per (batch, KV head).  Invisible keys are never read, which is where the
+// decode saving of the paper's operator benchmark comes from.  The g query
+// heads of the KV head share every K/V tile: they form the rows of a
+// 16-row MMA block (rows g..15 are zero).  Each of the 4 warps owns 16 keys of
+// a tile and keeps its own online-softmax state; the warps and then the
+// splits are merged with their LSEs.
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace cowa {
+
+__device__ __forceinline__ float ex2d(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+
+struct KeySpans {
+    int n;
+    int lo[3], len[3];
+    int tiles[3];
+    int total_tiles;
+};
+
+__device__ inline KeySpans decode_spans(int p, const Win &w)
+{
+    KeySpans ks;
+    Ranges r;
+    r.n = 0;
+    if (p >= 0) {
+        // exact key intervals, half-open, kept in key units (BN = 1 below)
+        if (w.S > 0) { r.lo[r.n] = 0; r.hi[r.n] = min(w.S, p + 1); ++r.n; }
+        if (w.N > 0) { r.lo[r.n] = max(0, p - w.N + 1); r.hi[r.n] = p + 1; ++r.n; }
+        if (w.e > w.c && p - w.c >= 0) { r.lo[r.n] = max(0, p - w.e + 1); r.hi[r.n] = p - w.c + 1; ++r.n; }
+        merge_ranges(r);
+    }
+    ks.n = r.n;
+    ks.total_tiles = 0;
+    for (int a = 0; a < 3; ++a) {
+        ks.lo[a] = a < r.n ? r.lo[a] : 0;
+        ks.len[a] = a < r.n ? r.hi[a] - r.lo[a] : 0;
+        ks.tiles[a] = (ks.len[a] + kDecBN - 1) / kDecBN;
+        ks.total_tiles += ks.tiles[a];
+    }
+    return ks;
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
+{
+    constexpr int BN = kDecBN, NT = 128, KS = D / 16, ND = D / 8, STAGES = 3;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __nv_bfloat16 *sK = reinterpret_cast<__nv_bfloat16 *>(smem_raw);   // [STAGES][BN][D]
+    __nv_bfloat16 *sV = sK + STAGES * BN * D;                           // [STAGES][BN][D]
+    __nv_bfloat16 *sQ = sV + STAGES * BN * D;                           // [16][D]
+    // after the key loop the K/V stages are reused as the warp-merge scratch
+    float *sRed = reinterpret_cast<float *>(smem_raw);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int split = blockIdx.x, hl = blockIdx.y, b = blockIdx.z;
+    const int g = p.g;
+    int seq = p.seqlens[b];
+    if (seq < 0 || seq > p.Lcap) {  // never read outside the cache
+        if (tid == 0 && split == 0) atomicExch(p.err, 7);
+        seq = 0;
+    }
+    const int pq = seq - 1;
+    const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
+    const KeySpans ks = decode_spans(pq, w);
+    const int t_begin = (int)((long long)ks.total_tiles * split / p.splits);
+    const int t_end = (int)((long long)ks.total_tiles * (split + 1) / p.splits);
+    const int ntiles = t_end - t_begin;
+
+    // tile index -> (first key, valid keys)
+    auto tile_at = [&](int t, int &k0, int &nk) {
+        int a = 0;
+        while (a < 2 && t >= ks.tiles[a]) { t -= ks.tiles[a]; ++a; }
+        k0 = ks.lo[a] + t * BN;
+        nk = min(BN, ks.lo[a] + ks.len[a] - k0);
+    };
+
+    const __nv_bfloat16 *kg = reinterpret_cast<const __nv_bfloat16 *>(p.kc) + b * p.ks[0] + hl * p.ks[2];
+    const __nv_bfloat16 *vg = reinterpret_cast<const __nv_bfloat16 *>(p.vc) + b * p.vs[0] + hl * p.vs[2];
+    auto load_kv = [&](int t, int stage) {
+        int k0, nk;
+        tile_at(t, k0, nk);
+        load_tile<D, BN, NT>(sK + stage * BN * D, kg + (long long)k0 * p.ks[1], p.ks[1], nk, tid);
+        load_tile<D, BN, NT>(sV + stage * BN * D, vg + (long long)k0 * p.vs[1], p.vs[1], nk, tid);
+    };
+
+    // query rows of this group (rows >= g are zero)
+    const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(p.q) + b * p.qs[0] + (long long)hl * g * p.qs[2];
+    load_tile<D, 16, NT>(sQ, qg, p.qs[2], g, tid);
+    cp_async_commit();
+#pragma unroll
+    for (int s = 0; s < STAGES - 1; ++s) {
+        if (s < ntiles) load_kv(t_begin + s, s);
+        cp_async_commit();
+    }
+
+    cp_async_wait<STAGES - 1>();  // the query group
+    __syncthreads();
+    uint32_t qa[KS][4];
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk)
+        ldsm_x4(qa[kk], smem_u32(sQ + swz<D>(lane & 15, kk * 16 + (lane >> 4) * 8)));
+
+    float acc[ND][4];
+#pragma unroll
+    for (int n = 0; n < ND; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    float mx[2] = {-CUDART_INF_F, -CUDART_INF_F}, l[2] = {0.f, 0.f};
+    const int kw = warp * 16;  // this warp's keys within a tile
+
+    for (int t = 0; t < ntiles; ++t) {
+        const int stage = t % STAGES;
+        if (t + STAGES - 1 < ntiles) load_kv(t_begin + t + STAGES - 1, (t + STAGES - 1) % STAGES);
+        cp_async_commit();
+        cp_async_wait<STAGES - 1>();
+        __syncthreads();
+        int k0, nk;
+        tile_at(t_begin + t, k0, nk);
+        const __nv_bfloat16 *cK = sK + stage * BN * D;
+        const __nv_bfloat16 *cV = sV + stage * BN * D;
+
+        float s[2][4];
+#pragma unroll
+        for (int n = 0; n < 2; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            uint32_t bf[4];
+            const int key = kw + (lane & 7) + (lane >> 4) * 8;
+            const int col = kk * 16 + ((lane >> 3) & 1) * 8;
+            ldsm_x4(bf, smem_u32(cK + swz<D>(key, col)));
+            mma16816(s[0], qa[kk], bf[0], bf[1]);
+            mma16816(s[1], qa[kk], bf[2], bf[3]);
+        }
+        float tm[2] = {-CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int key = kw + n * 8 + (lane & 3) * 2 + (c & 1);
+                const float x = key < nk ? s[n][c] * p.scale_log2 : -CUDART_INF_F;
+                s[n][c] = x;
+                tm[c >> 1] = fmaxf(tm[c >> 1], x);
+            }
+        float alpha[2], msafe[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            tm[r] = fmaxf(tm[r], __shfl_xor_sync(0xffffffffu, tm[r], 1));
+            tm[r] = fmaxf(tm[r], __shfl_xor_sync(0xffffffffu, tm[r], 2));
+            const float mnew = fmaxf(mx[r], tm[r]);
+            msafe[r] = mnew == -CUDART_INF_F ? 0.f : mnew;
+            alpha[r] = ex2d(mx[r] - msafe[r]);
+            mx[r] = mnew;
+            l[r] *= alpha[r];
+        }
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float e = ex2d(s[n][c] - msafe[c >> 1]);
+                s[n][c] = e;
+                l[c >> 1] += e;
+            }
+#pragma unroll
+        for (int n = 0; n < ND; ++n) {
+            acc[n][0] *= alpha[0]; acc[n][1] *= alpha[0];
+            acc[n][2] *= alpha[1]; acc[n][3] *= alpha[1];
+        }
+        uint32_t pa_[4];
+        pa_[0] = pack_bf16(s[0][0], s[0][1]);
+        pa_[1] = pack_bf16(s[0][2], s[0][3]);
+        pa_[2] = pack_bf16(s[1][0], s[1][1]);
+        pa_[3] = pack_bf16(s[1][2], s[1][3]);
+#pragma unroll
+        for (int d2 = 0; d2 < D / 16; ++d2) {
+            uint32_t bf[4];
+            const int key = kw + (lane & 7) + ((lane >> 3) & 1) * 8;
+            const int col = d2 * 16 + (lane >> 4) * 8;
+            ldsm_x4_t(bf, smem_u32(cV + swz<D>(key, col)));
+            mma16816(acc[2 * d2], pa_, bf[0], bf[1]);
+            mma16816(acc[2 * d2 + 1], pa_, bf[2], bf[3]);
+        }
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+
+    // merge the four warps: rows 0..7 live in (lane>>2), c = 0,1 (row r = 0)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
+        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+    }
+    float *wm = sRed;              // [4][16] running max per warp and row
+    float *wl = wm + 64;           // [4][16] sums
+    float *wo = wl + 64;           // [4][16][D] unnormalised O (only rows < g used)
+    if ((lane & 3) == 0) {
+        const int row = lane >> 2;
+        wm[warp * 16 + row] = mx[0];
+        wl[warp * 16 + row] = l[0];
+        wm[warp * 16 + row + 8] = mx[1];
+        wl[warp * 16 + row + 8] = l[1];
+    }
+#pragma unroll
+    for (int n = 0; n < ND; ++n) {
+        const int col = n * 8 + (lane & 3) * 2;
+        const int row = lane >> 2;
+        wo[(warp * 16 + row) * D + col] = acc[n][0];
+        wo[(warp * 16 + row) * D + col + 1] = acc[n][1];
+        wo[(warp * 16 + row + 8) * D + col] = acc[n][2];
+        wo[(warp * 16 + row + 8) * D + col + 1] = acc[n][3];
+    }
+    __syncthreads();
+    const long long pbase = (((long long)b * p.Hq + (long long)hl * g) * p.splits + split);
+    for (int idx = tid; idx < g * D; idx += NT) {
+        const int row = idx / D, col = idx % D;
+        float m = -CUDART_INF_F;
+        for (int u = 0; u < 4; ++u) m = fmaxf(m, wm[u * 16 + row]);
+        const float ms = m == -CUDART_INF_F ? 0.f : m;
+        float lsum = 0.f, o = 0.f;
+        for (int u = 0; u < 4; ++u) {
+            const float f = ex2d(wm[u * 16 + row] - ms);
+            lsum += f * wl[u * 16 + row];
+            o += f * wo[(u * 16 + row) * D + col];
+        }
+        const long long pi = pbase + (long long)row * p.splits;
+        p.part_o[pi * D + col] = lsum > 0.f ? o / lsum : 0.f;
+        if (col == 0)  // log2-domain LSE of this split
+            p.part_lse[pi] = lsum > 0.f ? m + __log2f(lsum) : -CUDART_INF_F;
+    }
+}
+
+template <int D>
+__global__ void decode_combine_kernel(const DecodeParams p)
+{
+    const int row = blockIdx.x;  // b * Hq + hq
+    const int b = row / p.Hq, hq = row % p.Hq;
+    const float *pl = p.part_lse + (long long)row * p.splits;
+    const float *po = p.part_o + (long long)row * p.splits * D;
+    float m = -CUDART_INF_F;
+    for (int s = 0; s < p.splits; ++s) m = fmaxf(m, pl[s]);
+    const float ms = m == -CUDART_INF_F ? 0.f : m;
+    float lsum = 0.f;
+    for (int s = 0; s < p.splits; ++s) lsum += ex2d(pl[s] - ms);
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + b * p.os[0] + hq * p.os[2];
+    for (int col = threadIdx.x; col < D; col += blockDim.x) {
+        float acc = 0.f;
+        for (int s = 0; s < p.splits; ++s) acc += ex2d(pl[s] - ms) * po[(long long)s * D + col];
+        o[col] = __float2bfloat16_rn(lsum > 0.f ? acc / lsum : 0.f);
+    }
+    if (threadIdx.x == 0)
+        p.lse[row] = lsum > 0.f ? (m + __log2f(lsum)) * 0.69314718055994531f : -CUDART_INF_F;
+}
+
+template <int D>
+static cudaError_t launch_decode_d(const DecodeParams &p, cudaStream_t st)
+{
+    constexpr int smem = (6 * kDecBN * D + 16 * D) * 2;
+    static_assert((128 + 64 * D) * 4 <= 6 * kDecBN * D * 2, "merge scratch must fit the K/V stages");
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!configured[dev & 63]) {
+        cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured[dev & 63] = true;
+    }
+    dim3 grid(p.splits, p.Hkv, p.B);
+    decode_split_kernel<D><<<grid, 128, smem, st>>>(p);
+    note_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    decode_combine_kernel<D><<<p.B * p.Hq, 128, 0, st>>>(p);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const DecodeParams &p, int D, cudaStream_t st)
+{
+    if (p.B == 0 || p.Hq == 0) return cudaSuccess;
+    return D == 128 ? launch_decode_d<128>(p, st) : launch_decode_d<64>(p, st);
+}
+
+}  // namespace cowa

@@ -1,0 +1,67 @@
+// Kernel parameter blocks and launcher declarations shared by api.cu and the
+// kernel translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace cowa {
+
+struct AttnParams {
+    const void *q, *k, *v;
+    void *o;
+    float *lse;
+    const void *dout;
+    const float *lse_in;
+    void *dq, *dk, *dv;
+    float *delta;
+    const int *sched;       // query-tile-major schedule [Hkv][nqt][8]
+    const int *sched_t;     // key-tile-major schedule [Hkv][nkt][8]
+    long long qs[3], ks[3], vs[3], os[3];
+    int B, Lq, Lk, Hq, Hkv, g;
+    int S, N, G, W;
+    int kv_head_offset;
+    int nqt, nkt;           // tiles of the schedule in use
+    float scale, scale_log2;
+    int *err;               // device error word (status code of a failed device check)
+};
+
+struct DecodeParams {
+    const void *q, *kc, *vc;
+    const int *seqlens;
+    void *o;
+    float *lse;
+    float *part_o, *part_lse;
+    long long qs[3], ks[3], vs[3], os[3];
+    int B, Lcap, Hq, Hkv, g, splits;
+    int S, N, G, W;
+    int kv_head_offset;
+    float scale, scale_log2;
+    int *err;
+};
+
+// api.cu: process-wide count of kernels this library has launched
+void note_launches(int n);
+
+// schedule.cu
+cudaError_t launch_schedule(int *sched, int Hkv, int kv_head_offset, int Lq,
+                            int Lk, int S, int N, int G, int W, int BM, int BN, int transposed,
+                            cudaStream_t st);
+cudaError_t launch_tile_classes(const int *sched, uint8_t *out, int kv_head, int Lq, int Lk,
+                                int S, int N, int G, int W, int BM, int BN, int transposed,
+                                cudaStream_t st);
+
+// fwd_mma.cu
+cudaError_t launch_fwd_mma(const AttnParams &p, int D, cudaStream_t st);
+constexpr int kFwdBM = 128, kFwdBN = 64;
+
+// bwd_mma.cu
+cudaError_t launch_bwd_mma(const AttnParams &p, int D, cudaStream_t st);
+constexpr int kBwdBM = 64, kBwdBN = 64;
+inline int bwd_kv_qtile(int D) { return D == 128 ? 32 : 64; }
+
+// decode.cu
+cudaError_t launch_decode(const DecodeParams &p, int D, cudaStream_t st);
+constexpr int kDecBN = 64;
+
+}  // namespace cowa

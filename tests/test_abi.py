@@ -1,0 +1,101 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects
+bad arguments with the documented status codes before touching a device.
+Runs without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def cowa():
+    from structured_sparse_attention_block_b200 import build
+    build.build()
+    import structured_sparse_attention_block_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "cowa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(cowa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(cowa):
+    names = declared_functions()
+    assert "cowa_fwd" in names and "cowa_bwd" in names and "cowa_decode" in names
+    lib = ctypes.CDLL(cowa.library_path())
+    for n in names:
+        assert hasattr(lib, n), "missing export %s" % n
+
+
+def test_status_strings_and_version(cowa):
+    lib = cowa.lib()
+    assert lib.cowa_abi_version() == 1
+    for code, name in cowa._STATUS.items():
+        assert lib.cowa_status_string(code).decode() == name
+
+
+@pytest.mark.parametrize("Lk,Hkv,S,N,W", [(512, 2, 16, 64, 224), (8192, 4, 64, 1024, 1792),
+                                          (32768, 8, 128, 4096, 3584), (131072, 8, 128, 8192, 15360),
+                                          (100, 4, 0, 200, 0), (65, 8, 0, 0, 9)])
+def test_default_quad(cowa, Lk, Hkv, S, N, W):
+    assert cowa.cowa_default_quad(Lk, Hkv, S, N) == (S, N, 0, W)
+
+
+def make_shape(cowa, B=1, Lq=128, Lk=128, Hq=4, Hkv=2, d=64, off=0, strides=None):
+    st = strides or {}
+    def s(name, H):
+        v = st.get(name, (Lq if name in "qo" else Lk) * H * d)
+        return (ctypes.c_int64 * 3)(v, H * d, d)
+    return cowa.Shape(B, Lq, Lk, Hq, Hkv, d, s("q", Hq), s("k", Hkv), s("v", Hkv), s("o", Hq), off)
+
+
+def call_fwd(cowa, shape, quad=(1, 2, 0, 3), ptr=16):
+    lib = cowa.lib()
+    p = ctypes.c_void_p(ptr)
+    return lib.cowa_fwd(ctypes.byref(shape), cowa.Quad(*quad), 0.0, p, p, p, p, p, p, 1 << 20, None)
+
+
+def test_argument_errors(cowa):
+    assert call_fwd(cowa, make_shape(cowa), quad=(-1, 2, 0, 3)) == 1
+    assert call_fwd(cowa, make_shape(cowa, d=96)) == 2
+    assert call_fwd(cowa, make_shape(cowa, Hq=3, Hkv=2)) == 1
+    assert call_fwd(cowa, make_shape(cowa, strides={"k": 1001})) == 3
+    assert call_fwd(cowa, make_shape(cowa), ptr=0) == 1
+    assert call_fwd(cowa, make_shape(cowa), ptr=24) == 3
+    assert "not 16-byte aligned" in cowa.lib().cowa_last_error_detail().decode()
+    lib = cowa.lib()
+    shp = make_shape(cowa, Lq=2)
+    p = ctypes.c_void_p(16)
+    st = lib.cowa_decode(ctypes.byref(shp), cowa.Quad(1, 2, 0, 3), 0.0, p, p, p, p, p, p, p, 1 << 20, None)
+    assert st == 1  # decode needs Lq == 1
+
+
+def test_empty_problem_is_a_no_op(cowa):
+    # nothing to compute: returns OK without needing a device or pointers
+    shape = make_shape(cowa, B=0)
+    lib = cowa.lib()
+    assert lib.cowa_fwd(ctypes.byref(shape), cowa.Quad(1, 2, 0, 3), 0.0, *([None] * 5), None, 0, None) == 0
+
+
+def test_workspace_sizes(cowa):
+    lib = cowa.lib()
+    shape = make_shape(cowa, Lq=1000, Lk=1000)
+    assert lib.cowa_fwd_workspace_size(ctypes.byref(shape), cowa.Quad(1, 2, 0, 3)) >= 2 * 8 * 8 * 4
+    assert lib.cowa_bwd_workspace_size(ctypes.byref(shape), cowa.Quad(1, 2, 0, 3)) >= 4 * 1000 * 4
+    assert lib.cowa_fwd_workspace_size(ctypes.byref(shape), cowa.Quad(-1, 2, 0, 3)) == 0
+
+
+def test_oracle_is_not_reachable_from_the_product():
+    """The package never imports the oracle (test infrastructure only)."""
+    pkg = os.path.join(ROOT, "structured_sparse_attention_block_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle|#include\s+\S*oracle|cowa_ref_",
+                                     text, flags=re.M), f

@@ -137,3 +137,15 @@ def test_empty_rows_and_degenerate_quads(oracle_mod):
     # N >= Lk: every head is dense causal regardless of W
     for h in range(3):
         assert (oracle_mod.mask(9, 9, h, (0, 9, 0, 0)) == causal(9, 9)).all()
+
+
+def test_tile_counts_match_the_dense_mask(oracle_mod):
+    for (Lq, Lk, BM, BN) in [(100, 100, 32, 64), (70, 130, 64, 64), (130, 70, 128, 64)]:
+        quad = (5, 17, 3, 11)
+        for w in range(3):
+            m = oracle_mod.mask(Lq, Lk, w, quad)
+            counts = oracle_mod.tile_counts(Lq, Lk, w, quad, BM, BN)
+            for qt in range(counts.shape[0]):
+                for kt in range(counts.shape[1]):
+                    blk = m[qt * BM:(qt + 1) * BM, kt * BN:(kt + 1) * BN]
+                    assert counts[qt, kt] == blk.sum()
