@@ -210,9 +210,10 @@ def cowa_bwd(q, k, v, o, lse, dout, quad, softmax_scale=None, kv_head_offset=0,
         _bf16_cuda(t, n)
     if dout.stride() != o.stride():
         raise ValueError("dout must have the strides of o")
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
+    # the C ABI gives each gradient the strides of its input
+    dq = torch.empty_strided(q.shape, q.stride(), dtype=q.dtype, device=q.device) if dq is None else dq
+    dk = torch.empty_strided(k.shape, k.stride(), dtype=k.dtype, device=k.device) if dk is None else dk
+    dv = torch.empty_strided(v.shape, v.stride(), dtype=v.dtype, device=v.device) if dv is None else dv
     for t, ref, n in ((dq, q, "dq"), (dk, k, "dk"), (dv, v, "dv")):
         _bf16_cuda(t, n)
         if t.stride() != ref.stride() or t.shape != ref.shape:
