@@ -151,6 +151,31 @@ COWA_API int cowa_decode(const cowa_shape_t *shape, cowa_quad_t quad, float soft
                 size_t workspace_bytes, void *stream);
 
 /*
+ * Decode that allocates nothing (no counterpart in the paper: it exists for
+ * callers that cannot allocate device memory, such as a plugin inside another
+ * runtime that owns all device memory and passes only input and output
+ * buffers, or a serving loop where cudaMalloc, which may synchronise the
+ * device, is not allowed).
+ *   Same arguments and results as cowa_decode, without the workspace: the
+ *   split-KV partials live in a static device array of
+ *   COWA_DECODE_NOALLOC_SCRATCH_BYTES bytes inside the library, which every
+ *   GPU that loads the library holds until the process exits.  Shapes whose
+ *   partials (cowa_decode_workspace_size) exceed it are refused with
+ *   COWA_ERR_WORKSPACE and a detail message; nothing is launched then.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.  Every call on a device shares the one array:
+ *   calls whose kernels overlap on the GPU (different streams, no ordering
+ *   between them) race on it and must not be issued.  The array keeps the
+ *   last call's partials; each call overwrites every partial it reads.
+ *   No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+#define COWA_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+COWA_API int cowa_decode_noalloc(const cowa_shape_t *shape, cowa_quad_t quad, float softmax_scale,
+                                 const void *q, const void *k_cache, const void *v_cache,
+                                 const int32_t *seqlens, void *o, float *lse, void *stream);
+
+/*
  * Visible-tile classes of one KV head, as the training kernels see them, for
  * checking the schedule: writes out[qt * nkt + kt] (device, uint8) for the
  * tiling BM x BN = (64 or 128) x 64, nqt = ceil(Lq/BM), nkt = ceil(Lk/BN):

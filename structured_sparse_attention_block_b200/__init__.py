@@ -28,6 +28,7 @@ import torch
 __all__ = ["CowaError", "cowa_fwd", "cowa_bwd", "cowa_decode", "cowa_default_quad",
            "cowa_tile_classes", "cowa_fwd_workspace_size", "cowa_bwd_workspace_size",
            "cowa_decode_workspace_size", "cowa_get_device_error", "cowa_launch_count",
+           "cowa_decode_noalloc",
            "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -92,6 +93,8 @@ def lib():
         L.cowa_bwd.argtypes = [SP, Quad, ctypes.c_float] + [vp] * 9 + [vp, sz, vp]
         L.cowa_decode.restype = ctypes.c_int
         L.cowa_decode.argtypes = [SP, Quad, ctypes.c_float] + [vp] * 6 + [vp, sz, vp]
+        L.cowa_decode_noalloc.restype = ctypes.c_int
+        L.cowa_decode_noalloc.argtypes = [SP, Quad, ctypes.c_float] + [vp] * 6 + [vp]
         L.cowa_schedule_workspace_size.restype = sz
         L.cowa_schedule_workspace_size.argtypes = [i64, i64, i32, i32]
         L.cowa_tile_classes.restype = ctypes.c_int
@@ -261,6 +264,30 @@ def cowa_decode(q, k_cache, v_cache, seqlens, quad, softmax_scale=None, kv_head_
     _check(L.cowa_decode(ctypes.byref(shape), qd, scale, _ptr(q4), _ptr(k_cache), _ptr(v_cache),
                          _ptr(seqlens), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                          _stream(q4.device)))
+    return out, lse
+
+
+def cowa_decode_noalloc(q, k_cache, v_cache, seqlens, quad, out, lse, softmax_scale=None,
+                        kv_head_offset=0):
+    """Decode that allocates no device memory, for callers that cannot
+    allocate (for example a plugin inside a runtime that owns all device
+    memory).  The caller passes every buffer, out [B, 1, Hq, d] bf16 and
+    lse [B, Hq] fp32 included; the split scratch is a fixed array inside the
+    library (``COWA_DECODE_NOALLOC_SCRATCH_BYTES``, 4 MiB per GPU).  Calls on
+    one device must not overlap on the GPU.  Returns ``(out, lse)``."""
+    q4 = q if q.dim() == 4 else q.unsqueeze(1)
+    for t, n in ((q4, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (out, "out")):
+        _bf16_cuda(t, n)
+    if seqlens.dtype != torch.int32 or not seqlens.is_cuda or not seqlens.is_contiguous():
+        raise TypeError("seqlens must be a contiguous int32 CUDA tensor")
+    B, _, Hq, d = q4.shape
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq):
+        raise ValueError("lse must be contiguous fp32 [B, Hq]")
+    shape = _shape(q4, k_cache, v_cache, out, kv_head_offset)
+    scale = 0.0 if softmax_scale is None else float(softmax_scale)
+    _check(lib().cowa_decode_noalloc(ctypes.byref(shape), _quad(quad), scale, _ptr(q4), _ptr(k_cache),
+                                     _ptr(v_cache), _ptr(seqlens), _ptr(out), _ptr(lse),
+                                     _stream(q4.device)))
     return out, lse
 
 

@@ -14,6 +14,10 @@
 namespace cowa {
 __device__ int g_cowa_device_error = 0;
 
+// Records a status and its detail for cowa_last_error_detail() from code
+// outside this file.
+int set_error_detail(int status, const char *detail);
+
 static std::atomic<unsigned long long> g_launches{0};
 void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 }
@@ -169,6 +173,8 @@ int decode_splits(const cowa_shape_t *s, cowa_quad_t q, int sms)
 }
 
 }  // namespace
+
+int cowa::set_error_detail(int status, const char *detail) { return fail(status, "%s", detail); }
 
 extern "C" {
 

@@ -1,0 +1,60 @@
+"""cowa_decode_noalloc: decode for callers that cannot allocate device memory.
+
+Such callers (a plugin inside a runtime that owns all device memory and hands
+over only input and output buffers, or a serving loop where cudaMalloc is not
+allowed) get a decode whose split scratch is a fixed array inside the
+library.  These tests call it through the C ABI and compare it with
+cowa_decode, which takes a caller workspace, on two calls in a row (the
+second call finds the first call's partials still in the array), and check
+that a shape too large for the array is refused before anything runs.
+"""
+import ctypes
+
+import pytest
+import torch
+
+from helpers import LSE_ABS, assert_o, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def noalloc_status(cowa, q, kc, vc, sl, quad, out, lse):
+    shape = cowa._shape(q, kc, vc, out, 0)
+    return cowa.lib().cowa_decode_noalloc(
+        ctypes.byref(shape), cowa._quad(quad), ctypes.c_float(0.0), cowa._ptr(q), cowa._ptr(kc),
+        cowa._ptr(vc), cowa._ptr(sl), cowa._ptr(out), cowa._ptr(lse),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+def test_noalloc_matches_decode_on_two_calls_in_a_row():
+    import structured_sparse_attention_block_b200 as cowa
+    from structured_sparse_attention_block_b200.inputs import decode_inputs
+    quad = (64, 512, 0, 896)
+    runs = [(0, [4096, 4000, 129, 1]), (1, [77, 4096, 2048, 3000])]
+    for seed, seqlens in runs:
+        q, kc, vc, sl = decode_inputs(4, 4096, 16, 4, 128, seed=seed, seqlens=seqlens)
+        o_ref, lse_ref = cowa.cowa_decode(q, kc, vc, sl, quad)
+        out = torch.full_like(o_ref, float("nan"))
+        lse = torch.full_like(lse_ref, float("nan"))
+        assert noalloc_status(cowa, q, kc, vc, sl, quad, out, lse) == 0
+        torch.cuda.synchronize()
+        cowa.cowa_get_device_error()
+        assert_o(out[:, 0], to64(o_ref[:, 0]), what="noalloc O")
+        diff = (lse - lse_ref).abs().max().item()
+        assert diff <= LSE_ABS
+
+
+def test_noalloc_refuses_shapes_beyond_the_static_scratch():
+    import structured_sparse_attention_block_b200 as cowa
+    # 64 sequences x 64 query heads x d=128 need more split scratch than 4 MiB
+    shape = cowa.Shape(64, 1, 1 << 16, 64, 8, 128, (ctypes.c_int64 * 3)(64 * 128, 64 * 128, 128),
+                       (ctypes.c_int64 * 3)((1 << 16) * 8 * 128, 8 * 128, 128),
+                       (ctypes.c_int64 * 3)((1 << 16) * 8 * 128, 8 * 128, 128),
+                       (ctypes.c_int64 * 3)(64 * 128, 64 * 128, 128), 0)
+    quad = cowa.Quad(128, 8192, 0, 7168)
+    lib = cowa.lib()
+    torch.cuda.init()
+    assert lib.cowa_decode_workspace_size(ctypes.byref(shape), quad) > (4 << 20)
+    st = lib.cowa_decode_noalloc(ctypes.byref(shape), quad, 0.0, *([None] * 6), None)
+    assert st == 4
+    assert "static limit" in lib.cowa_last_error_detail().decode()
