@@ -178,7 +178,10 @@ COWA_API int cowa_decode_noalloc(const cowa_shape_t *shape, cowa_quad_t quad, fl
 /*
  * Visible-tile classes of one KV head, as the training kernels see them, for
  * checking the schedule: writes out[qt * nkt + kt] (device, uint8) for the
- * tiling BM x BN = (64 or 128) x 64, nqt = ceil(Lq/BM), nkt = ceil(Lk/BN):
+ * tiling BM x BN, BM in {32, 64, 128} and BN in {64, 96, 128} (the forward
+ * uses 128 x 96 for d = 64 and 128 x 64 for d = 128, the backward 64 x 64
+ * and, key-tile major, 32 or 64 x 64),
+ * nqt = ceil(Lq/BM), nkt = ceil(Lk/BN):
  *   0 = tile skipped, 1 = visited with the element mask applied,
  *   2 = visited without a mask (every in-range pair visible).
  * kv_head is the global KV-head index.  transposed = 0 uses the

@@ -255,14 +255,19 @@ int cowa_fwd(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const
     fill_common(p, s, quad, softmax_scale);
     p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
     p.B = (int)s->B; p.Lq = (int)s->Lq; p.Lk = (int)s->Lk;
+    // tensor-core path (TMA + tcgen05); with no keys at all there is nothing
+    // to map, and the warp-level kernel writes the empty rows
+    const bool tc = s->Lk > 0;
+    const int BN = tc ? cowa::fwd5_bn((int)s->d) : cowa::kFwdBN;
     p.nqt = (int)cdiv(s->Lq, cowa::kFwdBM);
-    p.nkt = (int)cdiv(s->Lk, cowa::kFwdBN);
+    p.nkt = (int)cdiv(s->Lk, BN);
     int *sched = (int *)ws;
     p.sched = sched;
     cudaError_t e = cowa::launch_schedule(sched, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W,
-                                          cowa::kFwdBM, cowa::kFwdBN, 0, st);
+                                          cowa::kFwdBM, BN, 0, st);
     if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
-    e = cowa::launch_fwd_mma(p, (int)s->d, st);
+    e = tc ? cowa::launch_fwd_sm100(p, (int)s->d, st) : cowa::launch_fwd_mma(p, (int)s->d, st);
+    if (e == cudaErrorInvalidValue && tc) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
     if (e != cudaSuccess) return cuda_fail(e, "forward launch");
     return COWA_OK;
 }
@@ -359,8 +364,8 @@ int cowa_tile_classes(int64_t Lq, int64_t Lk, int64_t kv_head, cowa_quad_t quad,
     if (r) return r;
     if (Lq < 0 || Lk < 0 || Lq >= kMaxLen || Lk >= kMaxLen || kv_head < 0 || kv_head >= kMaxLen)
         return fail(COWA_ERR_INVALID_ARG, "bad length or head");
-    if ((BM != 64 && BM != 128 && BM != 32) || BN != 64)
-        return fail(COWA_ERR_UNSUPPORTED, "tiling %dx%d (supported: 32/64/128 x 64)", BM, BN);
+    if ((BM != 64 && BM != 128 && BM != 32) || (BN != 64 && BN != 96 && BN != 128))
+        return fail(COWA_ERR_UNSUPPORTED, "tiling %dx%d (supported: 32/64/128 x 64/96/128)", BM, BN);
     if (Lq == 0 || Lk == 0) return COWA_OK;
     if (!out) return fail(COWA_ERR_INVALID_ARG, "out is NULL");
     if ((r = check_device(nullptr))) return r;

@@ -1,0 +1,446 @@
+// CoWA training / prefill forward on the 5th-generation tensor cores.
+//
+// One CTA per (query tile of 128 rows, pair of query heads of one GQA group,
+// batch).  Two query heads of a group have the same KV head, hence the same
+// window mask and the same visible key tiles, so the CTA streams each K/V
+// tile once for both and neither head wastes work.  Ten warps:
+//   warp 8     TMA producer: both Q tiles once, then the K and V tiles the
+//              schedule lists (sink, near and long bands only) into a ring of
+//              shared-memory stages;
+//   warp 9     MMA issuer (one thread) and tensor-memory owner.  For head slot
+//              x in {0, 1}: S_x(t) = Q_x K_t^T into S_x, and O_x += P_x(t) V_t
+//              with P_x(t) read from its own tensor-memory region (a later MMA
+//              writing S_x is not ordered after an earlier MMA's read of P from
+//              the same columns, so P never shares columns with S).  Order:
+//              S_0(0) S_1(0), then per tile  PV_0(t) S_0(t+1) PV_1(t) S_1(t+1),
+//              so each softmax warpgroup only waits on its own MMAs and the two
+//              warpgroups overlap;
+//   warps 0-3  softmax of slot 0, warps 4-7 softmax of slot 1: thread r of a
+//              warpgroup owns query row r.  Pass 1 reads the row of S in
+//              32-column chunks and takes the max (edge tiles only apply the
+//              element mask); pass 2 re-reads S, writes P = 2^(s*scale - m) as
+//              bf16 to P_x, and sums P twice: in fp32 for the LSE and as the
+//              rounded bf16 values for the normalisation of O, so O is divided
+//              by exactly the weights the PV product used.  The O row is
+//              rescaled in tensor memory only when the max grows by more than
+//              2^8 (until then the stale max is a valid reference point).
+// Key tiles are 96 wide for d = 64 and 64 wide for d = 128: a softmax thread
+// reads its whole row of S_x with one tensor-memory round trip and keeps it in
+// registers.  Tensor-memory columns: S_x at x*128 (d = 64) or x*64 (d = 128),
+// P_x at 256 + 64x or 128 + 32x, O_x at 384 + 64x or 256 + 128x.  A tcgen05.commit tracks every earlier MMA of the issuing
+// thread, so S_x(t+1) complete implies PV_x(t) complete: P_x and O_x are free
+// to rewrite once the softmax holds S_x(t+1).
+// Every mbarrier wait is bounded; a wait that runs out records a timeout in
+// the device error word and the CTA winds down.
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace cowa {
+
+using namespace sm100;
+
+struct FwdArgs {
+    CUtensorMap tq, tk, tv;
+    AttnParams p;
+    int npair;  // head pairs per KV head: ceil(g / 2)
+};
+
+template <int D>
+struct FwdCfg {
+    static constexpr int BM = 128, BN = fwd5_bn(D);
+    static constexpr int STAGES = 4;
+    // tensor-memory column offsets and per-slot strides (32-column aligned)
+    static constexpr int S_STR = D == 128 ? 64 : 128, P_STR = S_STR / 2;
+    static constexpr int T_S = 0, T_P = 2 * S_STR, T_O = D == 128 ? 256 : 384;
+    static constexpr int KB = D / 64;                 // 128-byte blocks along d
+    static constexpr int Q_BYTES = BM * D * 2;        // one head's query tile
+    static constexpr int KV_BYTES = BN * D * 2;       // one of K or V
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+    static constexpr int NBAR = 10 + 2 * STAGES;
+    static constexpr int SMEM = 1024 + 2 * Q_BYTES + STAGES * STAGE_BYTES + 8 * NBAR + 16;
+    static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
+    static constexpr uint32_t IDESC_O = idesc_bf16(128, D, 0, 1);
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant__ FwdArgs a)
+{
+    using C = FwdCfg<D>;
+    constexpr int BM = C::BM, BN = C::BN, ST = C::STAGES, KB = C::KB;
+    const AttnParams &p = a.p;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char *sm = smem_raw + (base - raw);
+    const uint32_t sQ = base;  // slot x at sQ + x * Q_BYTES
+    const uint32_t sStage = base + 2 * C::Q_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 2 * C::Q_BYTES + ST * C::STAGE_BYTES);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const uint32_t bar0 = smem_addr(bars);
+    const uint32_t BAR_Q = bar0;
+    auto KV_FULL = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto KV_EMPTY = [&](int s) { return bar0 + 8u * (1 + ST + s); };
+    auto S_FULL = [&](int x) { return bar0 + 8u * (1 + 2 * ST + x); };
+    auto P_FULL = [&](int x) { return bar0 + 8u * (3 + 2 * ST + x); };
+    auto O_DONE = [&](int x) { return bar0 + 8u * (5 + 2 * ST + x); };
+    const uint32_t FIN = bar0 + 8u * (7 + 2 * ST);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qt = gridDim.x - 1 - blockIdx.x;  // long rows first
+    const int hl = blockIdx.y / a.npair, pair = blockIdx.y % a.npair;
+    const int hq0 = hl * p.g + 2 * pair;
+    const int nslot = (2 * pair + 1 < p.g) ? 2 : 1;  // an odd group leaves the last head alone
+    const int b = blockIdx.z;
+    const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
+    const int delta = p.Lk - p.Lq;
+    const int i0 = qt * BM;
+    const int nrows = min(BM, p.Lq - i0);
+    const int pa = i0 + delta, pb = i0 + nrows - 1 + delta;
+
+    const int4 *e4 = reinterpret_cast<const int4 *>(p.sched + ((size_t)hl * p.nqt + qt) * kSchedInts);
+    const int4 e0 = e4[0], e1 = e4[1];
+    const int nr = e0.x;
+    const int lo0 = e0.y, lo1 = e0.w, lo2 = e1.y;
+    const int len0 = e0.z - e0.y, len1 = e1.x - e0.w, len2 = e1.z - e1.y;
+    const int ntiles = (nr > 0 ? len0 : 0) + (nr > 1 ? len1 : 0) + (nr > 2 ? len2 : 0);
+    auto tile_of = [&](int t) {
+        if (t < len0 || nr == 1) return lo0 + t;
+        t -= len0;
+        if (t < len1 || nr == 2) return lo1 + t;
+        return lo2 + t - len1;
+    };
+
+    if (tid == 0) {
+        mbar_init(BAR_Q, 1);
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(KV_FULL(s), 1);
+            mbar_init(KV_EMPTY(s), 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(S_FULL(x), 1);
+            mbar_init(P_FULL(x), 128);
+            mbar_init(O_DONE(x), 1);
+        }
+        mbar_init(FIN, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_addr(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tmap(&a.tq);
+        prefetch_tmap(&a.tk);
+        prefetch_tmap(&a.tv);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ TMA
+        if (lane == 0) {
+            mbar_expect_tx(BAR_Q, nslot * C::Q_BYTES);
+            for (int x = 0; x < nslot; ++x)
+                for (int kb = 0; kb < KB; ++kb)
+                    tma_load_4d(sQ + x * C::Q_BYTES + kb * BM * 128, &a.tq, BAR_Q, kb * 64, i0, hq0 + x, b);
+            int issued = 0;
+            for (int t = 0; t < ntiles; ++t) {
+                const int s = t % ST;
+                if (t >= ST && !mbar_wait(KV_EMPTY(s), ((t / ST) - 1) & 1, p.err, abort_flag)) break;
+                const int kt = tile_of(t);
+                mbar_expect_tx(KV_FULL(s), C::STAGE_BYTES);
+                const uint32_t sk = sStage + s * C::STAGE_BYTES, sv = sk + C::KV_BYTES;
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_4d(sk + kb * BN * 128, &a.tk, KV_FULL(s), kb * 64, kt * BN, hl, b);
+                    tma_load_4d(sv + kb * BN * 128, &a.tv, KV_FULL(s), kb * 64, kt * BN, hl, b);
+                }
+                issued = t + 1;
+            }
+            // every load this thread issued has landed before the CTA ends
+            mbar_wait(BAR_Q, 0, p.err, abort_flag);
+            for (int t = issued > ST ? issued - ST : 0; t < issued; ++t)
+                mbar_wait(KV_FULL(t % ST), (t / ST) & 1, p.err, abort_flag);
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ MMA
+        if (lane == 0) {
+            bool ok = mbar_wait(BAR_Q, 0, p.err, abort_flag);
+            auto qk = [&](int x, int t) {  // S_x(t) = Q_x K_t^T
+                const uint32_t sk = sStage + (t % ST) * C::STAGE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t ad = sdesc(sQ + x * C::Q_BYTES + (kk >> 2) * BM * 128 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sdesc(sk + (kk >> 2) * BN * 128 + (kk & 3) * 32, 16, 1024);
+                    mma_ss(tmem + C::T_S + x * C::S_STR, ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(S_FULL(x));
+            };
+            auto pv = [&](int x, int t) -> bool {  // O_x += P_x(t) V_t
+                if (!mbar_wait(P_FULL(x), t & 1, p.err, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t sv = sStage + (t % ST) * C::STAGE_BYTES + C::KV_BYTES;
+#pragma unroll
+                for (int k2 = 0; k2 < BN / 16; ++k2) {
+                    const uint64_t bd = sdesc(sv + k2 * 2048, BN * 128, 1024);
+                    mma_ts(tmem + C::T_O + x * D, tmem + C::T_P + x * C::P_STR + k2 * 8, bd, C::IDESC_O,
+                           (t > 0 || k2 > 0) ? 1u : 0u);
+                }
+                mma_commit(O_DONE(x));
+                return true;
+            };
+            if (ok && ntiles > 0) {
+                ok = mbar_wait(KV_FULL(0), 0, p.err, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    for (int x = 0; x < nslot; ++x) qk(x, 0);
+                }
+            }
+            for (int t = 0; ok && t < ntiles; ++t) {
+                const bool more = t + 1 < ntiles;
+                if (more) {
+                    if (!(ok = mbar_wait(KV_FULL((t + 1) % ST), ((t + 1) / ST) & 1, p.err, abort_flag))) break;
+                    tc_fence_after();
+                }
+                for (int x = 0; x < nslot && ok; ++x) {
+                    if (!(ok = pv(x, t))) break;
+                    if (more) qk(x, t + 1);
+                }
+                mma_commit(KV_EMPTY(t % ST));  // both heads are done with K_t and V_t
+            }
+            mma_commit(FIN);
+            mbar_wait(FIN, 0, p.err, abort_flag);
+        }
+    } else {
+        // -------------------------------------------------------- softmax
+        const int x = warp >> 2;  // head slot of this warpgroup
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + C::T_S + x * C::S_STR + lane_off;
+        const uint32_t tP = tmem + C::T_P + x * C::P_STR + lane_off;
+        const uint32_t tOx = tmem + C::T_O + x * D + lane_off;
+        const int prow = pa + r;
+        const bool active = x < nslot;
+        float m_run = -CUDART_INF_F, l = 0.f, lb = 0.f;  // lb: sum of the bf16-rounded P
+        bool ok = true;
+        for (int t = 0; active && t < ntiles; ++t) {
+            ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), t & 1, p.err, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const int kt = tile_of(t);
+            const bool full = tile_full(pa, pb, kt * BN, BN, p.Lk, w);
+            // One read of the row of S: all chunks are requested back to back and
+            // waited for once (each tensor-memory round trip costs hundreds of
+            // cycles).  Edge tiles build, per 32-key chunk, the bitmask of keys the
+            // row sees: the union of its sink, near and long key intervals.
+            constexpr int NC = BN / 32;  // 32-column chunks of the row
+            uint32_t sr[BN];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+            uint32_t vis[NC];
+            if (!full) {
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+                    const int j0 = kt * BN + c * 32;
+                    // key intervals [lo, hi] of the row, relative to j0
+                    const int sh = min(w.S - 1, prow) - j0;                    // sink [0, min(S-1, p)]
+                    const int nl = prow - w.N + 1 - j0, nh = prow - j0;        // near [p-N+1, p]
+                    const int ll = prow - w.e + 1 - j0, lh = prow - w.c - j0;  // long [p-e+1, p-c]
+                    auto bits = [](int lo, int hi) -> uint32_t {
+                        lo = max(lo, 0);
+                        hi = min(hi, 31);
+                        return lo > hi ? 0u : ((0xFFFFFFFFu >> (31 - (hi - lo))) << lo);
+                    };
+                    uint32_t m = bits(-j0, sh);
+                    if (w.N > 0) m |= bits(nl, nh);
+                    if (w.e > w.c) m |= bits(ll, lh);
+                    vis[c] = m;
+                }
+            }
+            tmem_wait_ld();
+            float mx4[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mx4[k] = -CUDART_INF_F;
+            if (full) {
+#pragma unroll
+                for (int e = 0; e < BN; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], __uint_as_float(sr[e]));
+            } else {
+#pragma unroll
+                for (int e = 0; e < BN; ++e) {
+                    if (!((vis[e >> 5] >> (e & 31)) & 1u)) sr[e] = __float_as_uint(-CUDART_INF_F);
+                    mx4[e & 3] = fmaxf(mx4[e & 3], __uint_as_float(sr[e]));
+                }
+            }
+            const float smax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            const float tmax = smax * p.scale_log2;  // scale > 0 keeps the order
+            // lazy rescale: keep the old reference max unless it is exceeded by
+            // 2^8.  S_x(t) being complete means PV_x(t-1) is too (the MMAs of one
+            // thread complete in order), so O_x can be rescaled right away.
+            const bool grow = tmax > m_run + 8.f;
+            const float alpha = grow ? fast_ex2(m_run - tmax) : 1.f;
+            const bool fix_o = grow && m_run != -CUDART_INF_F;
+            if (__any_sync(0xffffffffu, fix_o)) {
+                const float f = fix_o ? alpha : 1.f;
+#pragma unroll
+                for (int c = 0; c < D / 16; ++c) {
+                    uint32_t o[16];
+                    tmem_ld16(tOx + c * 16, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                    tmem_st16(tOx + c * 16, o);
+                }
+                tmem_wait_st();
+            }
+            if (grow) {
+                l *= alpha;
+                lb *= alpha;
+                m_run = tmax;
+            }
+            const float nms = m_run == -CUDART_INF_F ? 0.f : -m_run;
+            // P = 2^(s*scale - m) as bf16 into P_x, two keys per packed f32x2
+            // op; packed entry e (< BN/2) takes keys 2e and 2e+1 and is written
+            // over sr[e], already consumed
+            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(nms, nms);
+            float2 la = make_float2(0.f, 0.f), lba = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int e = 0; e < BN / 2; ++e) {
+                const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
+                                             sc2, nm2);
+                const float p0 = fast_ex2(xa.x), p1 = fast_ex2(xa.y);
+                const uint32_t pr = pack2(p0, p1);
+                la = __fadd2_rn(la, make_float2(p0, p1));
+                lba = __fadd2_rn(lba, make_float2(__uint_as_float(pr << 16), __uint_as_float(pr & 0xFFFF0000u)));
+                sr[e] = pr;
+            }
+#pragma unroll
+            for (int c = 0; c < NC; ++c) tmem_st16(tP + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c * 16]));
+            l += la.x + la.y;
+            lb += lba.x + lba.y;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(P_FULL(x));
+        }
+        if (active && ok && ntiles > 0) {
+            // PV_x(ntiles-2) is complete (S_x(ntiles-1) was), so O_DONE(x) has
+            // completed ntiles-1 or ntiles phases: the parity of the last one is
+            // unambiguous (a parity wait only tells apart adjacent phases)
+            ok = __all_sync(0xffffffffu, mbar_wait(O_DONE(x), (ntiles - 1) & 1, p.err, abort_flag));
+        }
+        tc_fence_after();
+        // epilogue: O / (sum of the bf16 P) in bf16, LSE (natural log) from the fp32 sum
+        if (active) {
+            const bool have = ok && ntiles > 0;
+            const float inv = (l > 0.f && lb > 0.f) ? 1.f / lb : 0.f;
+            const int hq = hq0 + x;
+            __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + b * p.os[0] +
+                                  (long long)(i0 + r) * p.os[1] + hq * p.os[2];
+#pragma unroll
+            for (int c = 0; c < D / 16; ++c) {
+                uint32_t o[16];
+                if (have) {
+                    tmem_ld16(tOx + c * 16, o);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] = 0u;
+                }
+                uint32_t pk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    pk[e] = pack2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+                if (r < nrows) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 16);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+            if (r < nrows)
+                p.lse[((long long)b * p.Hq + hq) * p.Lq + i0 + r] =
+                    l > 0.f ? m_run * 0.69314718055994531f + logf(l) : -CUDART_INF_F;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+// ----------------------------------------------------------------- host ----
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+}  // namespace
+
+// [B, L, H, d] bf16 tensor (strides in elements for b, l, h) as a 4-D map
+// with 64-element x `rows` boxes and 128-byte swizzle.
+bool make_bshd_map(CUtensorMap *m, const void *base, int d, long long L, long long H, long long B,
+                   const long long st[3], int rows)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)H, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)st[1] * 2, (cuuint64_t)st[2] * 2, (cuuint64_t)st[0] * 2};
+    for (int k = 0; k < 3; ++k)
+        if (strides[k] == 0) strides[k] = 16;  // a dimension of extent 1 with stride 0
+    cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D>
+static cudaError_t launch_fwd5_d(const AttnParams &p, cudaStream_t st)
+{
+    using C = FwdCfg<D>;
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!configured[dev & 63]) {
+        cudaError_t e = cudaFuncSetAttribute(fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return e;
+        configured[dev & 63] = true;
+    }
+    FwdArgs a;
+    memset(&a, 0, sizeof a);
+    a.p = p;
+    a.npair = (p.g + 1) / 2;
+    if (!make_bshd_map(&a.tq, p.q, D, p.Lq, p.Hq, p.B, p.qs, C::BM) ||
+        !make_bshd_map(&a.tk, p.k, D, p.Lk, p.Hkv, p.B, p.ks, C::BN) ||
+        !make_bshd_map(&a.tv, p.v, D, p.Lk, p.Hkv, p.B, p.vs, C::BN))
+        return cudaErrorInvalidValue;
+    dim3 grid(p.nqt, p.Hkv * a.npair, p.B);
+    fwd_sm100_kernel<D><<<grid, 320, C::SMEM, st>>>(a);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_sm100(const AttnParams &p, int D, cudaStream_t st)
+{
+    if (p.nqt == 0 || p.Hq == 0 || p.B == 0) return cudaSuccess;
+    return D == 128 ? launch_fwd5_d<128>(p, st) : launch_fwd5_d<64>(p, st);
+}
+
+}  // namespace cowa

@@ -2,6 +2,7 @@
 // kernel translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -51,9 +52,19 @@ cudaError_t launch_tile_classes(const int *sched, uint8_t *out, int kv_head, int
                                 int S, int N, int G, int W, int BM, int BN, int transposed,
                                 cudaStream_t st);
 
-// fwd_mma.cu
+// fwd_mma.cu (warp-level MMA forward; used when there are no keys to map)
 cudaError_t launch_fwd_mma(const AttnParams &p, int D, cudaStream_t st);
 constexpr int kFwdBM = 128, kFwdBN = 64;
+
+// fwd_sm100.cu (tcgen05 forward)
+cudaError_t launch_fwd_sm100(const AttnParams &p, int D, cudaStream_t st);
+constexpr int kFwd5BM = 128;
+// key-tile width of the tcgen05 forward: 96 for d = 64, 64 for d = 128 (a
+// softmax thread holds one row of a tile in registers)
+__host__ __device__ constexpr int fwd5_bn(int D) { return D == 128 ? 64 : 96; }
+// [B, L, H, d] bf16 tensor as a 4-D TMA map, 64-element x `rows` boxes, 128-byte swizzle
+bool make_bshd_map(CUtensorMap *m, const void *base, int d, long long L, long long H, long long B,
+                   const long long st[3], int rows);
 
 // bwd_mma.cu
 cudaError_t launch_bwd_mma(const AttnParams &p, int D, cudaStream_t st);

@@ -13,10 +13,7 @@ import torch
 
 pytestmark = pytest.mark.gpu
 
-BN = 64
-
-
-def expected_classes(oracle_mod, Lq, Lk, h, quad, BM):
+def expected_classes(oracle_mod, Lq, Lk, h, quad, BM, BN):
     counts = oracle_mod.tile_counts(Lq, Lk, h, quad, BM, BN)
     nqt, nkt = counts.shape
     rows = np.minimum(BM, Lq - np.arange(nqt) * BM)[:, None]
@@ -39,13 +36,20 @@ SMALL = [  # Lq, Lk, Hkv, quad
 ]
 
 
+# the tilings the kernels use: forward 128x96 (d=64) and 128x64 (d=128), dQ
+# 64x64, dK/dV key-tile major with 32 (d=128) or 64 (d=64) query rows per
+# step; 128x128 checks the general tile arithmetic
+TILINGS = [(128, 96, False), (128, 64, False), (64, 64, False), (32, 64, True), (64, 64, True),
+           (128, 128, False)]
+
+
 @pytest.mark.parametrize("Lq,Lk,Hkv,quad", SMALL)
-@pytest.mark.parametrize("BM,transposed", [(128, False), (64, False), (32, True), (64, True)])
-def test_schedule_small(oracle_mod, Lq, Lk, Hkv, quad, BM, transposed):
+@pytest.mark.parametrize("BM,BN,transposed", TILINGS)
+def test_schedule_small(oracle_mod, Lq, Lk, Hkv, quad, BM, BN, transposed):
     import structured_sparse_attention_block_b200 as cowa
     for h in range(Hkv):
         got = cowa.cowa_tile_classes(Lq, Lk, h, quad, BM, BN, transposed).cpu().numpy()
-        exp = expected_classes(oracle_mod, Lq, Lk, h, quad, BM)
+        exp = expected_classes(oracle_mod, Lq, Lk, h, quad, BM, BN)
         np.testing.assert_array_equal(got, exp, err_msg="head %d" % h)
 
 
@@ -56,7 +60,7 @@ def test_schedule_workloads(oracle_mod, name, heads):
     wl = WORKLOADS[name]
     heads = range(wl.Hkv) if heads is None else heads
     for h in heads:
-        for BM, tr in [(128, False), (64, True)]:
+        for BM, BN, tr in [(128, 96 if wl.d == 64 else 64, False), (64, 64, True)]:
             got = cowa.cowa_tile_classes(wl.Lq, wl.Lk, h, wl.quad, BM, BN, tr).cpu().numpy()
-            exp = expected_classes(oracle_mod, wl.Lq, wl.Lk, h, wl.quad, BM)
+            exp = expected_classes(oracle_mod, wl.Lq, wl.Lk, h, wl.quad, BM, BN)
             np.testing.assert_array_equal(got, exp, err_msg="%s head %d BM %d" % (name, h, BM))
