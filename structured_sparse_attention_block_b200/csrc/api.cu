@@ -220,9 +220,10 @@ size_t cowa_fwd_workspace_size(const cowa_shape_t *s, cowa_quad_t q)
 size_t cowa_bwd_workspace_size(const cowa_shape_t *s, cowa_quad_t q)
 {
     if (check_shape(s, q, false)) return 0;
-    return align256((size_t)(s->B * s->Hq * s->Lq) * sizeof(float)) +
-           sched_bytes(s->Hkv, cdiv(s->Lq, cowa::kBwdBM)) +
-           sched_bytes(s->Hkv, cdiv(s->Lk, cowa::kBwdBN)) + 256;
+    // per-row (-LSE*log2e, -delta) pairs padded to 64 rows (also holds the
+    // warp-level path's delta), then two schedules sized for the finer tiling
+    return align256((size_t)(s->B * s->Hq * cowa::bwd5_lq_pad(s->Lq)) * sizeof(float2)) +
+           sched_bytes(s->Hkv, cdiv(s->Lq, 64)) + sched_bytes(s->Hkv, cdiv(s->Lk, 64)) + 256;
 }
 
 size_t cowa_decode_workspace_size(const cowa_shape_t *s, cowa_quad_t q)
@@ -295,24 +296,44 @@ int cowa_bwd(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const
     p.q = q; p.k = k; p.v = v; p.o = (void *)o; p.lse_in = lse; p.dout = dout;
     p.dq = dq; p.dk = dk; p.dv = dv;
     p.B = (int)s->B; p.Lq = (int)s->Lq; p.Lk = (int)s->Lk;
-    const int QB = cowa::bwd_kv_qtile((int)s->d);
+    char *w = (char *)ws;
+    char *rows_ws = w;
+    w += align256((size_t)(s->B * s->Hq * cowa::bwd5_lq_pad(s->Lq)) * sizeof(float2));
+    int *sched_q = (int *)w;
+    w += sched_bytes(s->Hkv, cdiv(s->Lq, 64));
+    int *sched_t = (int *)w;
+    const int D = (int)s->d;
+    cudaError_t e;
+    if (s->Lq > 0 && s->Lk > 0) {
+        // tensor-core path: dK/dV over key tiles of 128, dQ over query tiles of 128
+        const int kv_bm = cowa::bwd5_kv_bm(D), dq_bn = cowa::bwd5_dq_bn(D);
+        const int nqt = (int)cdiv(s->Lq, cowa::kBwd5QTile), nkt = (int)cdiv(s->Lk, cowa::kBwd5KeyTile);
+        e = cowa::launch_schedule(sched_q, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W,
+                                  cowa::kBwd5QTile, dq_bn, 0, st);
+        if (e == cudaSuccess)
+            e = cowa::launch_schedule(sched_t, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W, kv_bm,
+                                      cowa::kBwd5KeyTile, 1, st);
+        if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+        e = cowa::launch_bwd_sm100(p, D, (float2 *)rows_ws, (int)cowa::bwd5_lq_pad(s->Lq), sched_q, nqt, sched_t,
+                                   nkt, st);
+        if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
+        if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+        return COWA_OK;
+    }
+    // no queries or no keys: the warp-level kernels write the zero gradients
+    const int QB = cowa::bwd_kv_qtile(D);
     p.nqt = (int)cdiv(s->Lq, cowa::kBwdBM);
     p.nkt = (int)cdiv(s->Lk, cowa::kBwdBN);
-    char *w = (char *)ws;
-    p.delta = (float *)w;
-    w += align256((size_t)(s->B * s->Hq * s->Lq) * sizeof(float));
-    int *sched_q = (int *)w;
-    w += sched_bytes(s->Hkv, p.nqt);
-    int *sched_t = (int *)w;
+    p.delta = (float *)rows_ws;
     p.sched = sched_q;
     p.sched_t = sched_t;
-    cudaError_t e = cowa::launch_schedule(sched_q, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W,
-                                          cowa::kBwdBM, cowa::kBwdBN, 0, st);
+    e = cowa::launch_schedule(sched_q, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W, cowa::kBwdBM,
+                              cowa::kBwdBN, 0, st);
     if (e == cudaSuccess)
         e = cowa::launch_schedule(sched_t, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W, QB,
                                   cowa::kBwdBN, 1, st);
     if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
-    e = cowa::launch_bwd_mma(p, (int)s->d, st);
+    e = cowa::launch_bwd_mma(p, D, st);
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return COWA_OK;
 }

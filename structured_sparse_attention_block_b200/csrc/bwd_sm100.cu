@@ -1,0 +1,708 @@
+// CoWA training backward on the 5th-generation tensor cores.
+//
+// Three kernels on the caller's stream; each output element has one writer,
+// so the result is deterministic.
+//
+// 1. bwd_prep_kernel: for every query row, (-LSE*log2(e), -delta) with
+//    delta = rowsum(dO * O), rows padded to a multiple of 64 (padding and rows
+//    that see no key get (-inf, 0), so their probabilities are 0).
+//
+// 2. dkdv_sm100_kernel, key-tile major: one CTA per (128 keys, KV head,
+//    batch).  The keys are the rows of every accumulator (tensor-memory lanes).
+//    Tasks are (query head of the group, query tile of BM rows) from the
+//    key-tile-major schedule.  Per task u, in buffer x = u % 2:
+//        S^T = K Q^T,  dP^T = V dO^T                   (MMA, into tensor memory)
+//        P^T = 2^(S^T*scale*log2e - LSE*log2e),  dS^T = P^T (dP^T - delta)
+//                                                      (warpgroup x, thread = key)
+//        dV += P^T dO,  dK += dS^T Q                   (MMA, P^T and dS^T from
+//                                                       tensor memory)
+//    Two warpgroups take alternate tasks so one computes while the MMAs of
+//    the other run.  dK is scaled by softmax_scale in the epilogue.
+//
+// 3. dq_sm100_kernel, query-tile major like the forward: per visible key tile
+//        S = Q K^T,  dP = dO V^T,  dS = P (dP - delta),  dQ += dS K.
+//    For d = 64 a CTA takes two query heads of a GQA group (same mask, same
+//    K/V tiles) with one warpgroup each.
+//
+// The elementwise warpgroups never read or write tensor-memory columns that
+// an MMA still uses: S/dP and P/dS live in separate regions, and a
+// tcgen05.commit tracks every earlier MMA of the issuing thread.  Every
+// mbarrier wait is bounded and reports a timeout through the error word.
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace cowa {
+
+using namespace sm100;
+
+// ------------------------------------------------------------- preprocess --
+template <int D>
+__global__ void bwd_prep_kernel(const AttnParams p, float2 *lsd, int lq_pad)
+{
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const long long total = (long long)p.B * p.Hq * lq_pad;
+    if (row >= total) return;
+    const int i = (int)(row % lq_pad);
+    const long long bh = row / lq_pad;  // b * Hq + hq
+    const int hq = (int)(bh % p.Hq), b = (int)(bh / p.Hq);
+    float s = 0.f, nl = -CUDART_INF_F;
+    if (i < p.Lq) {
+        const __nv_bfloat16 *o = reinterpret_cast<const __nv_bfloat16 *>(p.o) + b * p.os[0] +
+                                 (long long)i * p.os[1] + hq * p.os[2];
+        const __nv_bfloat16 *dout = reinterpret_cast<const __nv_bfloat16 *>(p.dout) + b * p.os[0] +
+                                    (long long)i * p.os[1] + hq * p.os[2];
+        constexpr int PER = D / 32;
+#pragma unroll
+        for (int x = 0; x < PER; x += 2) {
+            const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(o + lane * PER + x);
+            const __nv_bfloat162 c = *reinterpret_cast<const __nv_bfloat162 *>(dout + lane * PER + x);
+            s += __bfloat162float(a.x) * __bfloat162float(c.x) + __bfloat162float(a.y) * __bfloat162float(c.y);
+        }
+        const float lv = p.lse_in[bh * p.Lq + i];
+        nl = lv == -CUDART_INF_F ? -CUDART_INF_F : -lv * 1.4426950408889634f;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) lsd[row] = make_float2(nl, nl == -CUDART_INF_F ? 0.f : -s);
+}
+
+// bitmask of bit positions [lo, hi] within 0..31 (empty when lo > hi)
+__device__ __forceinline__ uint32_t span_bits(int lo, int hi)
+{
+    lo = max(lo, 0);
+    hi = min(hi, 31);
+    return lo > hi ? 0u : ((0xFFFFFFFFu >> (31 - (hi - lo))) << lo);
+}
+
+// ------------------------------------------------------------------ dK/dV --
+struct BwdArgs {
+    CUtensorMap tq, tk, tv, tdo;
+    AttnParams p;
+    const float2 *lsd;
+    int lq_pad;
+    int npair;
+};
+
+template <int D>
+struct KvCfg {
+    static constexpr int BN = kBwd5KeyTile;  // keys per CTA
+    static constexpr int BM = bwd5_kv_bm(D);  // queries per task
+    static constexpr int ST = 4;
+    static constexpr int KB = D / 64;
+    static constexpr int KV_BYTES = BN * D * 2;
+    static constexpr int QT_BYTES = BM * D * 2;
+    static constexpr int LSD_BYTES = BM * 8;
+    static constexpr int STAGE_BYTES = (2 * QT_BYTES + LSD_BYTES + 1023) / 1024 * 1024;
+    // tensor memory: dK, dV, then two buffers of S^T, dP^T, P^T (bf16), dS^T (bf16)
+    static constexpr int T_DK = 0, T_DV = D, T_BUF = 2 * D, BUF = 3 * BM;
+    static constexpr int NBAR = 7 + 2 * ST;
+    static constexpr int SMEM = 1024 + 2 * KV_BYTES + ST * STAGE_BYTES + 8 * NBAR + 16;
+    static constexpr uint32_t IDESC_S = idesc_bf16(128, BM, 0, 0);
+    static constexpr uint32_t IDESC_G = idesc_bf16(128, D, 0, 1);
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constant__ BwdArgs a)
+{
+    using C = KvCfg<D>;
+    constexpr int BN = C::BN, BM = C::BM, ST = C::ST, KB = C::KB;
+    const AttnParams &p = a.p;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char *sm = smem_raw + (base - raw);
+    const uint32_t sK = base, sV = base + C::KV_BYTES, sStage = base + 2 * C::KV_BYTES;
+    auto stage_q = [&](int s) { return sStage + s * C::STAGE_BYTES; };
+    auto stage_do = [&](int s) { return sStage + s * C::STAGE_BYTES + C::QT_BYTES; };
+    auto stage_lsd = [&](int s) {
+        return reinterpret_cast<const float2 *>(sm + 2 * C::KV_BYTES + s * C::STAGE_BYTES + 2 * C::QT_BYTES);
+    };
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 2 * C::KV_BYTES + ST * C::STAGE_BYTES);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const uint32_t bar0 = smem_addr(bars);
+    const uint32_t KV_LOADED = bar0;
+    auto Q_FULL = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto Q_EMPTY = [&](int s) { return bar0 + 8u * (1 + ST + s); };
+    auto S_FULL = [&](int x) { return bar0 + 8u * (1 + 2 * ST + x); };
+    auto P_FULL = [&](int x) { return bar0 + 8u * (3 + 2 * ST + x); };
+    const uint32_t DONE = bar0 + 8u * (5 + 2 * ST);
+    const uint32_t FIN = bar0 + 8u * (6 + 2 * ST);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int kt = blockIdx.x, hl = blockIdx.y, b = blockIdx.z;
+    const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
+    const int delta_pos = p.Lk - p.Lq;
+    const int c0 = kt * BN;
+
+    const int4 *e4 = reinterpret_cast<const int4 *>(p.sched_t + ((size_t)hl * p.nkt + kt) * kSchedInts);
+    const int4 e0 = e4[0], e1 = e4[1];
+    const int nr = e0.x;
+    const int lo0 = e0.y, lo1 = e0.w, lo2 = e1.y;
+    const int len0 = e0.z - e0.y, len1 = e1.x - e0.w, len2 = e1.z - e1.y;
+    const int nq = (nr > 0 ? len0 : 0) + (nr > 1 ? len1 : 0) + (nr > 2 ? len2 : 0);
+    const int ntask = nq * p.g;
+    auto task = [&](int u, int &hq, int &qt) {
+        hq = hl * p.g + u / nq;
+        int t = u % nq;
+        if (t < len0 || nr == 1) { qt = lo0 + t; return; }
+        t -= len0;
+        if (t < len1 || nr == 2) { qt = lo1 + t; return; }
+        qt = lo2 + t - len1;
+    };
+
+    if (tid == 0) {
+        mbar_init(KV_LOADED, 1);
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(Q_FULL(s), 1);
+            mbar_init(Q_EMPTY(s), 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(S_FULL(x), 1);
+            mbar_init(P_FULL(x), 128);
+        }
+        mbar_init(DONE, 1);
+        mbar_init(FIN, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_addr(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tmap(&a.tq);
+        prefetch_tmap(&a.tk);
+        prefetch_tmap(&a.tv);
+        prefetch_tmap(&a.tdo);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ TMA
+        if (lane == 0) {
+            mbar_expect_tx(KV_LOADED, 2 * C::KV_BYTES);
+            for (int kb = 0; kb < KB; ++kb) {
+                tma_load_4d(sK + kb * BN * 128, &a.tk, KV_LOADED, kb * 64, c0, hl, b);
+                tma_load_4d(sV + kb * BN * 128, &a.tv, KV_LOADED, kb * 64, c0, hl, b);
+            }
+            int issued = 0;
+            for (int u = 0; u < ntask; ++u) {
+                const int s = u % ST;
+                if (u >= ST && !mbar_wait(Q_EMPTY(s), ((u / ST) - 1) & 1, p.err, abort_flag)) break;
+                int hq, qt;
+                task(u, hq, qt);
+                mbar_expect_tx(Q_FULL(s), 2 * C::QT_BYTES + C::LSD_BYTES);
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_4d(stage_q(s) + kb * BM * 128, &a.tq, Q_FULL(s), kb * 64, qt * BM, hq, b);
+                    tma_load_4d(stage_do(s) + kb * BM * 128, &a.tdo, Q_FULL(s), kb * 64, qt * BM, hq, b);
+                }
+                bulk_load(stage_q(s) + 2 * C::QT_BYTES,
+                          a.lsd + ((long long)b * p.Hq + hq) * a.lq_pad + (long long)qt * BM, C::LSD_BYTES,
+                          Q_FULL(s));
+                issued = u + 1;
+            }
+            mbar_wait(KV_LOADED, 0, p.err, abort_flag);
+            for (int u = issued > ST ? issued - ST : 0; u < issued; ++u)
+                mbar_wait(Q_FULL(u % ST), (u / ST) & 1, p.err, abort_flag);
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ MMA
+        if (lane == 0) {
+            bool ok = mbar_wait(KV_LOADED, 0, p.err, abort_flag);
+            auto sdp = [&](int u) -> bool {  // S^T, dP^T of task u into buffer u % 2
+                const int s = u % ST, x = u & 1;
+                if (!mbar_wait(Q_FULL(s), (u / ST) & 1, p.err, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t tb = tmem + C::T_BUF + x * C::BUF;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ko = (kk >> 2) * BN * 128 + (kk & 3) * 32;
+                    const uint32_t qo = (kk >> 2) * BM * 128 + (kk & 3) * 32;
+                    mma_ss(tb, sdesc(sK + ko, 16, 1024), sdesc(stage_q(s) + qo, 16, 1024), C::IDESC_S, kk > 0);
+                    mma_ss(tb + BM, sdesc(sV + ko, 16, 1024), sdesc(stage_do(s) + qo, 16, 1024), C::IDESC_S,
+                           kk > 0);
+                }
+                mma_commit(S_FULL(x));
+                return true;
+            };
+            auto grad = [&](int u) -> bool {  // dV += P^T dO, dK += dS^T Q
+                const int s = u % ST, x = u & 1;
+                if (!mbar_wait(P_FULL(x), (u >> 1) & 1, p.err, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t tb = tmem + C::T_BUF + x * C::BUF;
+#pragma unroll
+                for (int k2 = 0; k2 < BM / 16; ++k2) {
+                    const uint32_t acc = (u > 0 || k2 > 0) ? 1u : 0u;
+                    mma_ts(tmem + C::T_DV, tb + 2 * BM + k2 * 8, sdesc(stage_do(s) + k2 * 2048, BM * 128, 1024),
+                           C::IDESC_G, acc);
+                    mma_ts(tmem + C::T_DK, tb + 2 * BM + BM / 2 + k2 * 8,
+                           sdesc(stage_q(s) + k2 * 2048, BM * 128, 1024), C::IDESC_G, acc);
+                }
+                mma_commit(Q_EMPTY(s));
+                return true;
+            };
+            if (ok && ntask > 0) ok = sdp(0);
+            if (ok && ntask > 1) ok = sdp(1);
+            for (int u = 0; ok && u < ntask; ++u) {
+                if (!(ok = grad(u))) break;
+                if (u + 2 < ntask) ok = sdp(u + 2);
+            }
+            mma_commit(DONE);
+            mma_commit(FIN);
+            mbar_wait(FIN, 0, p.err, abort_flag);
+        }
+    } else {
+        // ---------------------------------------------- P^T and dS^T per key
+        const int x = warp >> 2;
+        const int jl = (warp & 3) * 32 + lane;  // key row within the tile
+        const int jg = c0 + jl;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tb = tmem + C::T_BUF + x * C::BUF + lane_off;
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const long long pmax = (long long)p.Lk - 1;
+        // aligned positions p that see key jg: sink [jg, Lk-1], near
+        // [jg, jg+N-1], long [jg+c, jg+e-1]
+        const long long snk_hi = jg < w.S ? pmax : -1;
+        const long long nr_hi = w.N > 0 ? min((long long)jg + w.N - 1, pmax) : -1;
+        const long long lg_lo = (long long)jg + w.c, lg_hi = w.e > w.c ? min((long long)jg + w.e - 1, pmax) : -1;
+        bool ok = true;
+        for (int k = 0;; ++k) {
+            const int u = 2 * k + x;
+            if (u >= ntask) break;
+            ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), k & 1, p.err, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            int hq, qt;
+            task(u, hq, qt);
+            const int q0 = qt * BM;
+            const int nrows = min(BM, p.Lq - q0);
+            const int pa = q0 + delta_pos;
+            const bool full = tile_full(pa, pa + nrows - 1, c0, BN, p.Lk, w);
+            const float2 *lsd = stage_lsd(u % ST);
+#pragma unroll
+            for (int c = 0; c < BM / 32; ++c) {
+                uint32_t sr[32], dr[32];
+                tmem_ld32(tb + c * 32, sr);
+                tmem_ld32(tb + BM + c * 32, dr);
+                uint32_t vis = 0xFFFFFFFFu;
+                if (!full) {
+                    // query columns of this chunk: p = pa + c*32 + bit, rows < nrows
+                    const long long pc = (long long)pa + c * 32;
+                    const long long rmax = (long long)pa + nrows - 1;
+                    auto span = [&](long long lo, long long hi) -> uint32_t {
+                        hi = min(hi, rmax);
+                        if (hi < lo) return 0u;
+                        const long long a0 = lo - pc, a1 = hi - pc;
+                        if (a1 < 0 || a0 > 31) return 0u;
+                        return span_bits((int)max(a0, -1ll), (int)min(a1, 32ll));
+                    };
+                    vis = span(jg, snk_hi) | span(jg, nr_hi) | span(lg_lo, lg_hi);
+                }
+                tmem_wait_ld();
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float4 ld = *reinterpret_cast<const float4 *>(lsd + c * 32 + 2 * e);  // (-lse2, -delta) x2
+                    float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
+                                           sc2, make_float2(ld.x, ld.z));
+                    if (!((vis >> (2 * e)) & 1u)) xa.x = -CUDART_INF_F;
+                    if (!((vis >> (2 * e + 1)) & 1u)) xa.y = -CUDART_INF_F;
+                    const float2 pr = make_float2(fast_ex2(xa.x), fast_ex2(xa.y));
+                    const float2 t = __fadd2_rn(make_float2(__uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1])),
+                                                make_float2(ld.y, ld.w));
+                    const float2 ds = __fmul2_rn(pr, t);
+                    pk[e] = pack2(pr.x, pr.y);
+                    dk[e] = pack2(ds.x, ds.y);
+                }
+                tmem_st16(tb + 2 * BM + c * 16, pk);
+                tmem_st16(tb + 2 * BM + BM / 2 + c * 16, dk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(P_FULL(x));
+        }
+        // epilogue: warpgroup 0 writes dK (scaled), warpgroup 1 writes dV
+        ok = __all_sync(0xffffffffu, mbar_wait(DONE, 0, p.err, abort_flag) && ok);
+        tc_fence_after();
+        const bool have = ok && ntask > 0;
+        const float f = x == 0 ? p.scale : 1.f;
+        const uint32_t tg = tmem + (x == 0 ? C::T_DK : C::T_DV) + lane_off;
+        __nv_bfloat16 *grow_ = x == 0
+            ? reinterpret_cast<__nv_bfloat16 *>(p.dk) + b * p.ks[0] + (long long)jg * p.ks[1] + hl * p.ks[2]
+            : reinterpret_cast<__nv_bfloat16 *>(p.dv) + b * p.vs[0] + (long long)jg * p.vs[1] + hl * p.vs[2];
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+            uint32_t g[16];
+            if (have) {
+                tmem_ld16(tg + c * 16, g);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) g[e] = 0u;
+            }
+            uint32_t pk[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pk[e] = pack2(__uint_as_float(g[2 * e]) * f, __uint_as_float(g[2 * e + 1]) * f);
+            if (jg < p.Lk) {
+                uint4 *dst = reinterpret_cast<uint4 *>(grow_ + c * 16);
+                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+// --------------------------------------------------------------------- dQ --
+template <int D>
+struct DqCfg {
+    static constexpr int BM = kBwd5QTile;     // queries per CTA
+    static constexpr int BN = bwd5_dq_bn(D);  // keys per tile
+    static constexpr int NSLOT = D == 128 ? 1 : 2;
+    static constexpr int ST = D == 128 ? 2 : 4;
+    static constexpr int KB = D / 64;
+    static constexpr int QT_BYTES = BM * D * 2;  // one head's Q or dO tile
+    static constexpr int KV_BYTES = BN * D * 2;
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+    // tensor memory per slot: S, dP, dS (bf16), dQ
+    static constexpr int SLOT = D == 128 ? 512 : 256;
+    static constexpr int T_S = 0, T_DP = BN, T_DS = 2 * BN, T_DQ = D == 128 ? 384 : 192;
+    static constexpr int NBAR = 10 + 2 * ST;
+    static constexpr int SMEM = 1024 + 2 * NSLOT * QT_BYTES + ST * STAGE_BYTES + 8 * NBAR + 16;
+    static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
+    static constexpr uint32_t IDESC_Q = idesc_bf16(128, D, 0, 1);
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant__ BwdArgs a)
+{
+    using C = DqCfg<D>;
+    constexpr int BM = C::BM, BN = C::BN, ST = C::ST, KB = C::KB, NSLOT = C::NSLOT;
+    const AttnParams &p = a.p;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char *sm = smem_raw + (base - raw);
+    auto sQ = [&](int x) { return base + x * 2 * C::QT_BYTES; };
+    auto sDO = [&](int x) { return base + x * 2 * C::QT_BYTES + C::QT_BYTES; };
+    const uint32_t sStage = base + 2 * NSLOT * C::QT_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 2 * NSLOT * C::QT_BYTES + ST * C::STAGE_BYTES);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const uint32_t bar0 = smem_addr(bars);
+    const uint32_t BAR_Q = bar0;
+    auto KV_FULL = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto KV_EMPTY = [&](int s) { return bar0 + 8u * (1 + ST + s); };
+    auto S_FULL = [&](int x) { return bar0 + 8u * (1 + 2 * ST + x); };
+    auto DS_FULL = [&](int x) { return bar0 + 8u * (3 + 2 * ST + x); };
+    auto DONE = [&](int x) { return bar0 + 8u * (5 + 2 * ST + x); };
+    const uint32_t FIN = bar0 + 8u * (7 + 2 * ST);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qt = gridDim.x - 1 - blockIdx.x;
+    const int hl = blockIdx.y / a.npair, pair = blockIdx.y % a.npair;
+    const int hq0 = hl * p.g + NSLOT * pair;
+    const int nslot = min(NSLOT, p.g - NSLOT * pair);
+    const int b = blockIdx.z;
+    const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
+    const int delta_pos = p.Lk - p.Lq;
+    const int i0 = qt * BM;
+    const int nrows = min(BM, p.Lq - i0);
+    const int pa = i0 + delta_pos, pb = i0 + nrows - 1 + delta_pos;
+
+    const int4 *e4 = reinterpret_cast<const int4 *>(p.sched + ((size_t)hl * p.nqt + qt) * kSchedInts);
+    const int4 e0 = e4[0], e1 = e4[1];
+    const int nr = e0.x;
+    const int lo0 = e0.y, lo1 = e0.w, lo2 = e1.y;
+    const int len0 = e0.z - e0.y, len1 = e1.x - e0.w, len2 = e1.z - e1.y;
+    const int ntiles = (nr > 0 ? len0 : 0) + (nr > 1 ? len1 : 0) + (nr > 2 ? len2 : 0);
+    auto tile_of = [&](int t) {
+        if (t < len0 || nr == 1) return lo0 + t;
+        t -= len0;
+        if (t < len1 || nr == 2) return lo1 + t;
+        return lo2 + t - len1;
+    };
+
+    if (tid == 0) {
+        mbar_init(BAR_Q, 1);
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(KV_FULL(s), 1);
+            mbar_init(KV_EMPTY(s), 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(S_FULL(x), 1);
+            mbar_init(DS_FULL(x), 128);
+            mbar_init(DONE(x), 1);
+        }
+        mbar_init(FIN, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_addr(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tmap(&a.tq);
+        prefetch_tmap(&a.tk);
+        prefetch_tmap(&a.tv);
+        prefetch_tmap(&a.tdo);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ TMA
+        if (lane == 0) {
+            mbar_expect_tx(BAR_Q, nslot * 2 * C::QT_BYTES);
+            for (int x = 0; x < nslot; ++x)
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_4d(sQ(x) + kb * BM * 128, &a.tq, BAR_Q, kb * 64, i0, hq0 + x, b);
+                    tma_load_4d(sDO(x) + kb * BM * 128, &a.tdo, BAR_Q, kb * 64, i0, hq0 + x, b);
+                }
+            int issued = 0;
+            for (int t = 0; t < ntiles; ++t) {
+                const int s = t % ST;
+                if (t >= ST && !mbar_wait(KV_EMPTY(s), ((t / ST) - 1) & 1, p.err, abort_flag)) break;
+                const int kt = tile_of(t);
+                mbar_expect_tx(KV_FULL(s), C::STAGE_BYTES);
+                const uint32_t sk = sStage + s * C::STAGE_BYTES, sv = sk + C::KV_BYTES;
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_4d(sk + kb * BN * 128, &a.tk, KV_FULL(s), kb * 64, kt * BN, hl, b);
+                    tma_load_4d(sv + kb * BN * 128, &a.tv, KV_FULL(s), kb * 64, kt * BN, hl, b);
+                }
+                issued = t + 1;
+            }
+            mbar_wait(BAR_Q, 0, p.err, abort_flag);
+            for (int t = issued > ST ? issued - ST : 0; t < issued; ++t)
+                mbar_wait(KV_FULL(t % ST), (t / ST) & 1, p.err, abort_flag);
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ MMA
+        if (lane == 0) {
+            bool ok = mbar_wait(BAR_Q, 0, p.err, abort_flag);
+            auto sdp = [&](int x, int t) {  // S_x = Q_x K_t^T, dP_x = dO_x V_t^T
+                const uint32_t sk = sStage + (t % ST) * C::STAGE_BYTES, sv = sk + C::KV_BYTES;
+                const uint32_t ts = tmem + x * C::SLOT;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t qo = (kk >> 2) * BM * 128 + (kk & 3) * 32;
+                    const uint32_t ko = (kk >> 2) * BN * 128 + (kk & 3) * 32;
+                    mma_ss(ts + C::T_S, sdesc(sQ(x) + qo, 16, 1024), sdesc(sk + ko, 16, 1024), C::IDESC_S, kk > 0);
+                    mma_ss(ts + C::T_DP, sdesc(sDO(x) + qo, 16, 1024), sdesc(sv + ko, 16, 1024), C::IDESC_S,
+                           kk > 0);
+                }
+                mma_commit(S_FULL(x));
+            };
+            auto dq = [&](int x, int t) -> bool {  // dQ_x += dS_x K_t
+                if (!mbar_wait(DS_FULL(x), t & 1, p.err, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t sk = sStage + (t % ST) * C::STAGE_BYTES;
+                const uint32_t ts = tmem + x * C::SLOT;
+#pragma unroll
+                for (int k2 = 0; k2 < BN / 16; ++k2)
+                    mma_ts(ts + C::T_DQ, ts + C::T_DS + k2 * 8, sdesc(sk + k2 * 2048, BN * 128, 1024), C::IDESC_Q,
+                           (t > 0 || k2 > 0) ? 1u : 0u);
+                mma_commit(DONE(x));
+                return true;
+            };
+            if (ok && ntiles > 0) {
+                ok = mbar_wait(KV_FULL(0), 0, p.err, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    for (int x = 0; x < nslot; ++x) sdp(x, 0);
+                }
+            }
+            for (int t = 0; ok && t < ntiles; ++t) {
+                const bool more = t + 1 < ntiles;
+                if (more) {
+                    if (!(ok = mbar_wait(KV_FULL((t + 1) % ST), ((t + 1) / ST) & 1, p.err, abort_flag))) break;
+                    tc_fence_after();
+                }
+                for (int x = 0; x < nslot && ok; ++x) {
+                    if (!(ok = dq(x, t))) break;
+                    if (more) sdp(x, t + 1);
+                }
+                mma_commit(KV_EMPTY(t % ST));
+            }
+            mma_commit(FIN);
+            mbar_wait(FIN, 0, p.err, abort_flag);
+        }
+    } else {
+        // ------------------------------------------------- dS per query row
+        const int x = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t ts = tmem + x * C::SLOT + lane_off;
+        const int prow = pa + r;
+        const bool active = x < nslot;
+        const int hq = hq0 + x;
+        float nl = -CUDART_INF_F, nd = 0.f;
+        if (active && i0 + r < p.Lq) {
+            const float2 v = a.lsd[((long long)b * p.Hq + hq) * a.lq_pad + i0 + r];
+            nl = v.x;
+            nd = v.y;
+        }
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nl2 = make_float2(nl, nl),
+                     nd2 = make_float2(nd, nd);
+        bool ok = true;
+        for (int t = 0; active && t < ntiles; ++t) {
+            ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), t & 1, p.err, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const int kt = tile_of(t);
+            const bool full = tile_full(pa, pb, kt * BN, BN, p.Lk, w);
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t sr[32], dr[32];
+                tmem_ld32(ts + C::T_S + c * 32, sr);
+                tmem_ld32(ts + C::T_DP + c * 32, dr);
+                uint32_t vis = 0xFFFFFFFFu;
+                if (!full) {
+                    const int j0 = kt * BN + c * 32;
+                    vis = span_bits(-j0, min(w.S - 1, prow) - j0);
+                    if (w.N > 0) vis |= span_bits(prow - w.N + 1 - j0, prow - j0);
+                    if (w.e > w.c) vis |= span_bits(prow - w.e + 1 - j0, prow - w.c - j0);
+                }
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
+                                           sc2, nl2);
+                    if (!((vis >> (2 * e)) & 1u)) xa.x = -CUDART_INF_F;
+                    if (!((vis >> (2 * e + 1)) & 1u)) xa.y = -CUDART_INF_F;
+                    const float2 pr = make_float2(fast_ex2(xa.x), fast_ex2(xa.y));
+                    const float2 tt = __fadd2_rn(make_float2(__uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1])),
+                                                 nd2);
+                    const float2 ds = __fmul2_rn(pr, tt);
+                    pk[e] = pack2(ds.x, ds.y);
+                }
+                tmem_st16(ts + C::T_DS + c * 16, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(DS_FULL(x));
+        }
+        if (active && ok && ntiles > 0)
+            ok = __all_sync(0xffffffffu, mbar_wait(DONE(x), (ntiles - 1) & 1, p.err, abort_flag));
+        tc_fence_after();
+        if (active) {
+            const bool have = ok && ntiles > 0;
+            __nv_bfloat16 *drow = reinterpret_cast<__nv_bfloat16 *>(p.dq) + b * p.qs[0] +
+                                  (long long)(i0 + r) * p.qs[1] + hq * p.qs[2];
+#pragma unroll
+            for (int c = 0; c < D / 16; ++c) {
+                uint32_t g[16];
+                if (have) {
+                    tmem_ld16(ts + C::T_DQ + c * 16, g);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) g[e] = 0u;
+                }
+                uint32_t pk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    pk[e] = pack2(__uint_as_float(g[2 * e]) * p.scale, __uint_as_float(g[2 * e + 1]) * p.scale);
+                if (r < nrows) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(drow + c * 16);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+// ----------------------------------------------------------------- host ----
+template <int D>
+static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, const int *sched_dq, int nqt_dq,
+                                 const int *sched_kv, int nkt_kv, cudaStream_t st)
+{
+    using K = KvCfg<D>;
+    using Q = DqCfg<D>;
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!configured[dev & 63]) {
+        cudaError_t e = cudaFuncSetAttribute(dkdv_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(dq_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Q::SMEM);
+        if (e != cudaSuccess) return e;
+        configured[dev & 63] = true;
+    }
+    const long long rows = (long long)p.B * p.Hq * lq_pad;
+    if (rows > 0) {
+        bwd_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p, lsd, lq_pad);
+        note_launches(1);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    BwdArgs a;
+    memset(&a, 0, sizeof a);
+    a.p = p;
+    a.lsd = lsd;
+    a.lq_pad = lq_pad;
+    // dK/dV: query tiles of BM rows, key tiles of 128
+    if (!make_bshd_map(&a.tq, p.q, D, p.Lq, p.Hq, p.B, p.qs, K::BM) ||
+        !make_bshd_map(&a.tdo, p.dout, D, p.Lq, p.Hq, p.B, p.os, K::BM) ||
+        !make_bshd_map(&a.tk, p.k, D, p.Lk, p.Hkv, p.B, p.ks, K::BN) ||
+        !make_bshd_map(&a.tv, p.v, D, p.Lk, p.Hkv, p.B, p.vs, K::BN))
+        return cudaErrorInvalidValue;
+    a.p.sched_t = sched_kv;
+    a.p.nkt = nkt_kv;
+    if (nkt_kv > 0) {
+        dim3 g1(nkt_kv, p.Hkv, p.B);
+        dkdv_sm100_kernel<D><<<g1, 320, K::SMEM, st>>>(a);
+        note_launches(1);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    // dQ: query tiles of 128 rows, key tiles of BN
+    if (!make_bshd_map(&a.tq, p.q, D, p.Lq, p.Hq, p.B, p.qs, Q::BM) ||
+        !make_bshd_map(&a.tdo, p.dout, D, p.Lq, p.Hq, p.B, p.os, Q::BM) ||
+        !make_bshd_map(&a.tk, p.k, D, p.Lk, p.Hkv, p.B, p.ks, Q::BN) ||
+        !make_bshd_map(&a.tv, p.v, D, p.Lk, p.Hkv, p.B, p.vs, Q::BN))
+        return cudaErrorInvalidValue;
+    a.p.sched = sched_dq;
+    a.p.nqt = nqt_dq;
+    a.npair = (p.g + Q::NSLOT - 1) / Q::NSLOT;
+    if (nqt_dq > 0) {
+        dim3 g2(nqt_dq, p.Hkv * a.npair, p.B);
+        dq_sm100_kernel<D><<<g2, 320, Q::SMEM, st>>>(a);
+        note_launches(1);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+cudaError_t launch_bwd_sm100(const AttnParams &p, int D, float2 *lsd, int lq_pad, const int *sched_dq, int nqt_dq,
+                             const int *sched_kv, int nkt_kv, cudaStream_t st)
+{
+    if (p.B == 0 || p.Hq == 0) return cudaSuccess;
+    return D == 128 ? launch_bwd5_d<128>(p, lsd, lq_pad, sched_dq, nqt_dq, sched_kv, nkt_kv, st)
+                    : launch_bwd5_d<64>(p, lsd, lq_pad, sched_dq, nqt_dq, sched_kv, nkt_kv, st);
+}
+
+}  // namespace cowa

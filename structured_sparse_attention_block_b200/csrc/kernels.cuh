@@ -71,6 +71,15 @@ cudaError_t launch_bwd_mma(const AttnParams &p, int D, cudaStream_t st);
 constexpr int kBwdBM = 64, kBwdBN = 64;
 inline int bwd_kv_qtile(int D) { return D == 128 ? 32 : 64; }
 
+// bwd_sm100.cu (tcgen05 backward: preprocess, dK/dV pass, dQ pass)
+cudaError_t launch_bwd_sm100(const AttnParams &p, int D, float2 *lsd, int lq_pad, const int *sched_dq,
+                             int nqt_dq, const int *sched_kv, int nkt_kv, cudaStream_t st);
+constexpr int kBwd5KeyTile = 128;   // keys per dK/dV CTA (tensor-memory lanes)
+constexpr int kBwd5QTile = 128;     // queries per dQ CTA
+__host__ __device__ constexpr int bwd5_kv_bm(int D) { return D == 128 ? 32 : 64; }    // queries per dK/dV task
+__host__ __device__ constexpr int bwd5_dq_bn(int D) { return D == 128 ? 128 : 64; }   // keys per dQ tile
+inline long long bwd5_lq_pad(long long Lq) { return (Lq + 63) / 64 * 64; }
+
 // decode.cu
 cudaError_t launch_decode(const DecodeParams &p, int D, cudaStream_t st);
 constexpr int kDecBN = 64;

@@ -36,11 +36,12 @@ SMALL = [  # Lq, Lk, Hkv, quad
 ]
 
 
-# the tilings the kernels use: forward 128x96 (d=64) and 128x64 (d=128), dQ
-# 64x64, dK/dV key-tile major with 32 (d=128) or 64 (d=64) query rows per
-# step; 128x128 checks the general tile arithmetic
-TILINGS = [(128, 96, False), (128, 64, False), (64, 64, False), (32, 64, True), (64, 64, True),
-           (128, 128, False)]
+# the tilings the kernels use: forward 128x96 (d=64) and 128x64 (d=128);
+# backward dQ 128x64 (d=64) and 128x128 (d=128), dK/dV key-tile major over
+# 128 keys with 64 (d=64) or 32 (d=128) query rows per task; the warp-level
+# kernels' 64x64 and key-major 32/64 x 64
+TILINGS = [(128, 96, False), (128, 64, False), (128, 128, False), (64, 128, True), (32, 128, True),
+           (64, 64, False), (32, 64, True), (64, 64, True)]
 
 
 @pytest.mark.parametrize("Lq,Lk,Hkv,quad", SMALL)
@@ -60,7 +61,8 @@ def test_schedule_workloads(oracle_mod, name, heads):
     wl = WORKLOADS[name]
     heads = range(wl.Hkv) if heads is None else heads
     for h in heads:
-        for BM, BN, tr in [(128, 96 if wl.d == 64 else 64, False), (64, 64, True)]:
+        for BM, BN, tr in [(128, 96 if wl.d == 64 else 64, False), (128, 64 if wl.d == 64 else 128, False),
+                           (64 if wl.d == 64 else 32, 128, True)]:
             got = cowa.cowa_tile_classes(wl.Lq, wl.Lk, h, wl.quad, BM, BN, tr).cpu().numpy()
             exp = expected_classes(oracle_mod, wl.Lq, wl.Lk, h, wl.quad, BM, BN)
             np.testing.assert_array_equal(got, exp, err_msg="%s head %d BM %d" % (name, h, BM))
