@@ -134,27 +134,32 @@ __host__ __device__ inline Ranges key_tile_ranges(int c0, int c1, int Lq, int Lk
 // j >= S the rows that see it form j + D with D = [0,N) u [c,e); a row
 // range fits one connected part [a,b] of D iff j lies in [pb-b, pa-a].  Sink
 // columns j < S need j <= pa.  The tile is full iff its columns are covered
-// by the union of those column intervals.
+// by the union of those (at most three) column intervals.  Scalars only, so
+// the per-tile test stays in registers.
 __host__ __device__ inline bool tile_full(int pa, int pb, int c0, int BN, int Lk, const Win &w)
 {
     const int c1 = c0 + BN - 1;
     if (c1 >= Lk || pa < 0) return false;
-    int lo[3], hi[3], n = 0;
-    if (w.S > 0) { lo[n] = 0; hi[n] = w.S - 1 < pa ? w.S - 1 : pa; ++n; }
     const bool has_near = w.N > 0, has_long = w.e > w.c;
-    if (has_near && has_long && w.c <= w.N) {  // near and long windows touch
-        lo[n] = pb - (w.e - 1); hi[n] = pa; ++n;
-    } else {
-        if (has_near) { lo[n] = pb - (w.N - 1); hi[n] = pa; ++n; }
-        if (has_long) { lo[n] = pb - (w.e - 1); hi[n] = pa - w.c; ++n; }
-    }
-    for (int a = (w.S > 0 ? 1 : 0); a < n; ++a)
-        if (lo[a] < w.S) lo[a] = w.S;
+    const bool touch = has_near && has_long && w.c <= w.N;  // near and long windows adjoin
+    // sink [0, min(S-1, pa)]
+    const int lo0 = 0, hi0 = w.S > 0 ? (w.S - 1 < pa ? w.S - 1 : pa) : -1;
+    // near, or near and long together when they adjoin: [pb-(end-1), pa], j >= S
+    int lo1 = pb - ((touch ? w.e : w.N) - 1);
+    lo1 = lo1 < w.S ? w.S : lo1;
+    const int hi1 = has_near ? pa : -1;
+    // long on its own: [pb-(e-1), pa-c], j >= S
+    int lo2 = pb - (w.e - 1);
+    lo2 = lo2 < w.S ? w.S : lo2;
+    const int hi2 = (has_long && !touch) ? pa - w.c : -1;
     // greedy cover of [c0, c1]
     int x = c0;
-    for (int pass = 0; pass < 3; ++pass)
-        for (int a = 0; a < n; ++a)
-            if (lo[a] <= hi[a] && lo[a] <= x && x <= hi[a]) x = hi[a] + 1;
+#pragma unroll
+    for (int pass = 0; pass < 3; ++pass) {
+        if (lo0 <= x && x <= hi0) x = hi0 + 1;
+        if (lo1 <= x && x <= hi1) x = hi1 + 1;
+        if (lo2 <= x && x <= hi2) x = hi2 + 1;
+    }
     return x > c1;
 }
 

@@ -12,22 +12,27 @@
 //              with P_x(t) read from its own tensor-memory region (a later MMA
 //              writing S_x is not ordered after an earlier MMA's read of P from
 //              the same columns, so P never shares columns with S).  Order:
-//              S_0(0) S_1(0), then per tile  PV_0(t) S_0(t+1) PV_1(t) S_1(t+1),
-//              so each softmax warpgroup only waits on its own MMAs and the two
-//              warpgroups overlap;
+//              S_0(0) S_1(0), then per tile PV_0(t) S_0(t+1) PV_1(t) S_1(t+1)
+//              (with S double-buffered, SDB, S_x(t+2) follows PV_x(t)), so
+//              each softmax warpgroup only waits on its own MMAs;
 //   warps 0-3  softmax of slot 0, warps 4-7 softmax of slot 1: thread r of a
 //              warpgroup owns query row r.  Pass 1 reads the row of S in
 //              32-column chunks and takes the max (edge tiles only apply the
 //              element mask); pass 2 re-reads S, writes P = 2^(s*scale - m) as
-//              bf16 to P_x, and sums P twice: in fp32 for the LSE and as the
-//              rounded bf16 values for the normalisation of O, so O is divided
-//              by exactly the weights the PV product used.  The O row is
+//              bf16 to P_x and sums P in fp32 for the LSE.  The normalisation
+//              of O uses the sum of the bf16 P the PV product used, which a
+//              16-column MMA of P against a block of ones accumulates in
+//              tensor memory (L_x), so O is divided by exactly the weights it
+//              accumulated.  The O row is
 //              rescaled in tensor memory only when the max grows by more than
 //              2^8 (until then the stale max is a valid reference point).
 // Key tiles are 96 wide for d = 64 and 64 wide for d = 128: a softmax thread
-// reads its whole row of S_x with one tensor-memory round trip and keeps it in
-// registers.  Tensor-memory columns: S_x at x*128 (d = 64) or x*64 (d = 128),
-// P_x at 256 + 64x or 128 + 32x, O_x at 384 + 64x or 256 + 128x.  A tcgen05.commit tracks every earlier MMA of the issuing
+// reads its whole row of S_x with one tensor-memory round trip and keeps it
+// in registers.  Tensor-memory columns for d = 64: S_x at 128x, the bf16 row
+// sums L_x at 128x + 96, P_x at 256 + 64x, O_x at 384 + 64x; for d = 128:
+// S_x at 64x, P_x at 128 + 32x, L_x at 192 + 16x, O_x at 256 + 128x.  (A
+// double-buffered S with 64-key tiles, SDB, measured slower for d = 64: the
+// per-tile work shrinks and more tiles need the element mask.)  A tcgen05.commit tracks every earlier MMA of the issuing
 // thread, so S_x(t+1) complete implies PV_x(t) complete: P_x and O_x are free
 // to rewrite once the softmax holds S_x(t+1).
 // Every mbarrier wait is bounded; a wait that runs out records a timeout in
@@ -52,18 +57,26 @@ struct FwdArgs {
 template <int D>
 struct FwdCfg {
     static constexpr int BM = 128, BN = fwd5_bn(D);
-    static constexpr int STAGES = 4;
-    // tensor-memory column offsets and per-slot strides (32-column aligned)
-    static constexpr int S_STR = D == 128 ? 64 : 128, P_STR = S_STR / 2;
-    static constexpr int T_S = 0, T_P = 2 * S_STR, T_O = D == 128 ? 256 : 384;
+    static constexpr int STAGES = 4;  // tiles t, t+1, t+2 are resident at once
+    static constexpr bool SDB = false;  // S double-buffered per slot (needs BN = 64 for d = 64)
+    // tensor-memory column of S_x (buffer sb), P_x, L_x, O_x
+    static constexpr __host__ __device__ int t_s(int x, int sb)
+    {
+        return SDB ? 256 * x + 64 * sb : (D == 128 ? 64 * x : 128 * x);
+    }
+    static constexpr __host__ __device__ int t_p(int x) { return SDB ? 256 * x + 128 : (D == 128 ? 128 + 32 * x : 256 + 64 * x); }
+    static constexpr __host__ __device__ int t_l(int x) { return SDB ? 256 * x + 160 : (D == 128 ? 192 + 16 * x : 128 * x + 96); }
+    static constexpr __host__ __device__ int t_o(int x) { return SDB ? 256 * x + 192 : (D == 128 ? 256 + 128 * x : 384 + 64 * x); }
+    static constexpr int ONES_BYTES = 2048;  // 16 key rows x 128 bytes of bf16 1.0
     static constexpr int KB = D / 64;                 // 128-byte blocks along d
     static constexpr int Q_BYTES = BM * D * 2;        // one head's query tile
     static constexpr int KV_BYTES = BN * D * 2;       // one of K or V
     static constexpr int STAGE_BYTES = 2 * KV_BYTES;
     static constexpr int NBAR = 10 + 2 * STAGES;
-    static constexpr int SMEM = 1024 + 2 * Q_BYTES + STAGES * STAGE_BYTES + 8 * NBAR + 16;
+    static constexpr int SMEM = 1024 + 2 * Q_BYTES + STAGES * STAGE_BYTES + ONES_BYTES + 8 * NBAR + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
     static constexpr uint32_t IDESC_O = idesc_bf16(128, D, 0, 1);
+    static constexpr uint32_t IDESC_L = idesc_bf16(128, 16, 0, 1);
 };
 
 template <int D>
@@ -78,7 +91,8 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
     unsigned char *sm = smem_raw + (base - raw);
     const uint32_t sQ = base;  // slot x at sQ + x * Q_BYTES
     const uint32_t sStage = base + 2 * C::Q_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 2 * C::Q_BYTES + ST * C::STAGE_BYTES);
+    const uint32_t sOnes = sStage + ST * C::STAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 2 * C::Q_BYTES + ST * C::STAGE_BYTES + C::ONES_BYTES);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const uint32_t bar0 = smem_addr(bars);
@@ -139,6 +153,12 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         prefetch_tmap(&a.tk);
         prefetch_tmap(&a.tv);
     }
+    {
+        // bf16 1.0 everywhere in the ones block (any swizzle reads ones)
+        uint32_t *ones = reinterpret_cast<uint32_t *>(sm + 2 * C::Q_BYTES + ST * C::STAGE_BYTES);
+        for (int k = tid; k < C::ONES_BYTES / 4; k += blockDim.x) ones[k] = 0x3F803F80u;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -179,39 +199,42 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t ad = sdesc(sQ + x * C::Q_BYTES + (kk >> 2) * BM * 128 + (kk & 3) * 32, 16, 1024);
                     const uint64_t bd = sdesc(sk + (kk >> 2) * BN * 128 + (kk & 3) * 32, 16, 1024);
-                    mma_ss(tmem + C::T_S + x * C::S_STR, ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::t_s(x, t & 1), ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(S_FULL(x));
             };
-            auto pv = [&](int x, int t) -> bool {  // O_x += P_x(t) V_t
+            auto pv = [&](int x, int t) -> bool {  // O_x += P_x(t) V_t, L_x += P_x(t) 1
                 if (!mbar_wait(P_FULL(x), t & 1, p.err, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t sv = sStage + (t % ST) * C::STAGE_BYTES + C::KV_BYTES;
+                const uint64_t od = sdesc(sOnes, 128, 1024);
 #pragma unroll
                 for (int k2 = 0; k2 < BN / 16; ++k2) {
                     const uint64_t bd = sdesc(sv + k2 * 2048, BN * 128, 1024);
-                    mma_ts(tmem + C::T_O + x * D, tmem + C::T_P + x * C::P_STR + k2 * 8, bd, C::IDESC_O,
-                           (t > 0 || k2 > 0) ? 1u : 0u);
+                    const uint32_t pa_ = tmem + C::t_p(x) + k2 * 8;
+                    const uint32_t acc = (t > 0 || k2 > 0) ? 1u : 0u;
+                    mma_ts(tmem + C::t_o(x), pa_, bd, C::IDESC_O, acc);
+                    mma_ts(tmem + C::t_l(x), pa_, od, C::IDESC_L, acc);
                 }
                 mma_commit(O_DONE(x));
                 return true;
             };
-            if (ok && ntiles > 0) {
-                ok = mbar_wait(KV_FULL(0), 0, p.err, abort_flag);
-                if (ok) {
-                    tc_fence_after();
-                    for (int x = 0; x < nslot; ++x) qk(x, 0);
-                }
+            constexpr int AHEAD = C::SDB ? 2 : 1;  // S tiles issued ahead of the softmax
+            for (int t = 0; ok && t < AHEAD && t < ntiles; ++t) {
+                if (!(ok = mbar_wait(KV_FULL(t % ST), (t / ST) & 1, p.err, abort_flag))) break;
+                tc_fence_after();
+                for (int x = 0; x < nslot; ++x) qk(x, t);
             }
             for (int t = 0; ok && t < ntiles; ++t) {
-                const bool more = t + 1 < ntiles;
+                const int tn = t + AHEAD;  // the tile whose S follows PV_x(t)
+                const bool more = tn < ntiles;
                 if (more) {
-                    if (!(ok = mbar_wait(KV_FULL((t + 1) % ST), ((t + 1) / ST) & 1, p.err, abort_flag))) break;
+                    if (!(ok = mbar_wait(KV_FULL(tn % ST), (tn / ST) & 1, p.err, abort_flag))) break;
                     tc_fence_after();
                 }
                 for (int x = 0; x < nslot && ok; ++x) {
                     if (!(ok = pv(x, t))) break;
-                    if (more) qk(x, t + 1);
+                    if (more) qk(x, tn);
                 }
                 mma_commit(KV_EMPTY(t % ST));  // both heads are done with K_t and V_t
             }
@@ -223,17 +246,18 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         const int x = warp >> 2;  // head slot of this warpgroup
         const int r = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + C::T_S + x * C::S_STR + lane_off;
-        const uint32_t tP = tmem + C::T_P + x * C::P_STR + lane_off;
-        const uint32_t tOx = tmem + C::T_O + x * D + lane_off;
+        const uint32_t tP = tmem + C::t_p(x) + lane_off;
+        const uint32_t tOx = tmem + C::t_o(x) + lane_off;
+        const uint32_t tLx = tmem + C::t_l(x) + lane_off;
         const int prow = pa + r;
         const bool active = x < nslot;
-        float m_run = -CUDART_INF_F, l = 0.f, lb = 0.f;  // lb: sum of the bf16-rounded P
+        float m_run = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         for (int t = 0; active && t < ntiles; ++t) {
             ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), t & 1, p.err, abort_flag));
             if (!ok) break;
             tc_fence_after();
+            const uint32_t tS = tmem + C::t_s(x, t & 1) + lane_off;
             const int kt = tile_of(t);
             const bool full = tile_full(pa, pb, kt * BN, BN, p.Lk, w);
             // One read of the row of S: all chunks are requested back to back and
@@ -265,43 +289,50 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                 }
             }
             tmem_wait_ld();
+            if (!full) {
+#pragma unroll
+                for (int e = 0; e < BN; ++e)
+                    if (!((vis[e >> 5] >> (e & 31)) & 1u)) sr[e] = __float_as_uint(-CUDART_INF_F);
+            }
             float mx4[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) mx4[k] = -CUDART_INF_F;
-            if (full) {
 #pragma unroll
-                for (int e = 0; e < BN; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], __uint_as_float(sr[e]));
-            } else {
-#pragma unroll
-                for (int e = 0; e < BN; ++e) {
-                    if (!((vis[e >> 5] >> (e & 31)) & 1u)) sr[e] = __float_as_uint(-CUDART_INF_F);
-                    mx4[e & 3] = fmaxf(mx4[e & 3], __uint_as_float(sr[e]));
-                }
+            for (int e = 0; e < BN; e += 8) {
+                mx4[0] = max3(mx4[0], __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+                mx4[1] = max3(mx4[1], __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
+                mx4[2] = max3(mx4[2], __uint_as_float(sr[e + 4]), __uint_as_float(sr[e + 5]));
+                mx4[3] = max3(mx4[3], __uint_as_float(sr[e + 6]), __uint_as_float(sr[e + 7]));
             }
-            const float smax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            const float smax = fmaxf(max3(mx4[0], mx4[1], mx4[2]), mx4[3]);
             const float tmax = smax * p.scale_log2;  // scale > 0 keeps the order
-            // lazy rescale: keep the old reference max unless it is exceeded by
-            // 2^8.  S_x(t) being complete means PV_x(t-1) is too (the MMAs of one
-            // thread complete in order), so O_x can be rescaled right away.
+            // P_x and O_x are rewritten below: PV_x(t-1) must be complete (it
+            // almost always is by now; O_DONE(x) has completed t-1 or t phases)
+            if (t > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(O_DONE(x), (t - 1) & 1, p.err, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+            }
+            // lazy rescale: keep the old reference max unless it is exceeded by 2^8
             const bool grow = tmax > m_run + 8.f;
             const float alpha = grow ? fast_ex2(m_run - tmax) : 1.f;
             const bool fix_o = grow && m_run != -CUDART_INF_F;
             if (__any_sync(0xffffffffu, fix_o)) {
                 const float f = fix_o ? alpha : 1.f;
 #pragma unroll
-                for (int c = 0; c < D / 16; ++c) {
+                for (int c = 0; c <= D / 16; ++c) {  // O, then the bf16 sums
                     uint32_t o[16];
-                    tmem_ld16(tOx + c * 16, o);
+                    const uint32_t ta = c < D / 16 ? tOx + c * 16 : tLx;
+                    tmem_ld16(ta, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                    tmem_st16(tOx + c * 16, o);
+                    tmem_st16(ta, o);
                 }
                 tmem_wait_st();
             }
             if (grow) {
                 l *= alpha;
-                lb *= alpha;
                 m_run = tmax;
             }
             const float nms = m_run == -CUDART_INF_F ? 0.f : -m_run;
@@ -309,27 +340,27 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             // op; packed entry e (< BN/2) takes keys 2e and 2e+1 and is written
             // over sr[e], already consumed
             const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(nms, nms);
-            float2 la = make_float2(0.f, 0.f), lba = make_float2(0.f, 0.f);
+            float2 la = make_float2(0.f, 0.f), lc = make_float2(0.f, 0.f);
 #pragma unroll
             for (int e = 0; e < BN / 2; ++e) {
                 const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
                                              sc2, nm2);
                 const float p0 = fast_ex2(xa.x), p1 = fast_ex2(xa.y);
-                const uint32_t pr = pack2(p0, p1);
-                la = __fadd2_rn(la, make_float2(p0, p1));
-                lba = __fadd2_rn(lba, make_float2(__uint_as_float(pr << 16), __uint_as_float(pr & 0xFFFF0000u)));
-                sr[e] = pr;
+                if (e & 1)
+                    lc = __fadd2_rn(lc, make_float2(p0, p1));
+                else
+                    la = __fadd2_rn(la, make_float2(p0, p1));
+                sr[e] = pack2(p0, p1);
             }
 #pragma unroll
             for (int c = 0; c < NC; ++c) tmem_st16(tP + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c * 16]));
-            l += la.x + la.y;
-            lb += lba.x + lba.y;
+            l += (la.x + la.y) + (lc.x + lc.y);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(P_FULL(x));
         }
         if (active && ok && ntiles > 0) {
-            // PV_x(ntiles-2) is complete (S_x(ntiles-1) was), so O_DONE(x) has
+            // PV_x(ntiles-2) was waited for at the last tile, so O_DONE(x) has
             // completed ntiles-1 or ntiles phases: the parity of the last one is
             // unambiguous (a parity wait only tells apart adjacent phases)
             ok = __all_sync(0xffffffffu, mbar_wait(O_DONE(x), (ntiles - 1) & 1, p.err, abort_flag));
@@ -338,6 +369,13 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         // epilogue: O / (sum of the bf16 P) in bf16, LSE (natural log) from the fp32 sum
         if (active) {
             const bool have = ok && ntiles > 0;
+            float lb = 0.f;  // sum of the bf16 P that O accumulated
+            if (have) {
+                uint32_t lv[16];
+                tmem_ld16(tLx, lv);
+                tmem_wait_ld();
+                lb = __uint_as_float(lv[0]);
+            }
             const float inv = (l > 0.f && lb > 0.f) ? 1.f / lb : 0.f;
             const int hq = hq0 + x;
             __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + b * p.os[0] +

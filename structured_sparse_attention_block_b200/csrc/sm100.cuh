@@ -249,6 +249,14 @@ __device__ __forceinline__ float fast_ex2(float x)
     return y;
 }
 
+// max of three values in one instruction (sm_100)
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t pack2(float lo, float hi)
 {
     uint32_t r;
