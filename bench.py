@@ -170,26 +170,69 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# Source files each kernel is built from: its traffic record is valid only
+# while their hash matches the one stored beside the counters.
+KERNEL_SOURCES = {
+    "fwd_sm100": ["fwd_sm100.cu"],
+    "dkdv_sm100": ["bwd_sm100.cu"],
+    "dq_sm100": ["bwd_sm100.cu"],
+    "bwd_prep": ["bwd_sm100.cu"],
+    "decode_split": ["decode.cu"],
+    "decode_combine": ["decode.cu"],
+}
+SHARED_SOURCES = ["common.cuh", "kernels.cuh", "sm100.cuh"]
+
+
+def kernel_source_sha(kernel):
+    """First 16 hex digits of sha256 over the kernel's source files."""
+    import hashlib
+    csrc = os.path.join(ROOT, "structured_sparse_attention_block_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(KERNEL_SOURCES.get(kernel, []) + SHARED_SOURCES):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
 def load_traffic(kernel, workload):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources (matched by a hash of csrc/)."""
+    """DRAM bytes (read + write) per launch from the committed ncu counters,
+    or None when none were taken on the kernel's current sources."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             entries = json.load(f)
     except (OSError, ValueError):
         return None
-    import hashlib
-    csrc = os.path.join(ROOT, "structured_sparse_attention_block_b200", "csrc")
-    h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
-    digest = h.hexdigest()[:16]
+    if kernel not in KERNEL_SOURCES:
+        return None
+    digest = kernel_source_sha(kernel)
     for e in entries:
-        if e.get("kernel") == kernel and e.get("workload") == workload and e.get("csrc_sha") == digest:
+        if e.get("kernel") == kernel and e.get("workload") == workload and e.get("src_sha") == digest:
             return e.get("bytes_per_launch")
     return None
+
+
+def kernel_work(wl, pairs, dec_keys):
+    """Algorithmic work of one launch of each library kernel on a workload:
+    (bound, amount, unit of amount, how it is counted).  Tensor-bound kernels
+    count 2*d flops per visible (query head, key) pair and GEMM; HBM-bound
+    ones the bytes they must move once."""
+    d, B, Lq, Hq, Hkv = wl.d, wl.B, wl.Lq, wl.Hq, wl.Hkv
+    g = Hq // Hkv
+    rows = B * Hq * Lq
+    lq_pad = -(-Lq // 64) * 64
+    return {
+        "fwd_sm100": ("tensor", pairs * 4 * d, "flop",
+                      "4*d flops per visible pair (S = QK^T, O += PV), %d pairs" % pairs),
+        "dkdv_sm100": ("tensor", pairs * 8 * d, "flop",
+                       "8*d flops per visible pair (S^T, dP^T, dV += P^T dO, dK += dS^T Q), %d pairs" % pairs),
+        "dq_sm100": ("tensor", pairs * 6 * d, "flop",
+                     "6*d flops per visible pair (S, dP, dQ += dS K), %d pairs" % pairs),
+        "bwd_prep": ("hbm", rows * (2 * d * 2 + 4) + B * Hq * lq_pad * 8, "byte",
+                     "read O and dO (bf16) and LSE, write 8 bytes per padded row"),
+        "decode_split": ("hbm", dec_keys * 2 * d * 2, "byte",
+                         "visible K and V bytes, %d visible (KV head, key) pairs" % dec_keys),
+    }
 
 
 # ------------------------------------------------------------- GPU arm ----
@@ -234,23 +277,50 @@ def run_cowa(args, rank, world, local_rank):
         if ev is not None:
             ev[3].record(stream)
 
-    for _ in range(args.warmup):
+    # warm-up; all but the first step are traced kernel by kernel, which
+    # names the kernel with the largest share of the step
+    for i in range(args.warmup):
+        if i == 1:
+            cowa.cowa_trace_start(32 * args.warmup + 64)
         flush.zero_()
         step()
     torch.cuda.synchronize()
+    cowa.cowa_trace_stop()
+    warm_trace, dropped = cowa.cowa_trace_entries()
+    cowa.cowa_trace_start(0)
     cowa.cowa_get_device_error(dev)
+    if dropped or not warm_trace:
+        raise SystemExit("kernel trace of the warm-up incomplete")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    pairs = visible_pairs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, quad)
+    dec_keys = decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, quad)
+    work = kernel_work(wl, pairs, dec_keys)
+    warm = {}
+    for name, ms in warm_trace:
+        n, tot = warm.get(name, (0, 0.0))
+        warm[name] = (n + 1, tot + ms)
+    top = max((n for n in warm if n in work), key=lambda n: warm[n][1])
+    if world > 1:  # every rank times the same kernel
+        top = sorted(work)[int(max_over_ranks([float(sorted(work).index(top))], world, dev)[0])]
+
     launches0 = cowa.cowa_launch_count()
+    # the dominant kernel's launches in the timed steps get their own event pair
+    cowa.cowa_trace_start(4 * args.steps + 16, only=top)
     with ClockSampler(local_rank) as clocks:
         for i in range(args.steps):
             flush.zero_()
             step(evs[i])
         torch.cuda.synchronize()
+    cowa.cowa_trace_stop()
     launches = cowa.cowa_launch_count() - launches0
+    trace, dropped = cowa.cowa_trace_entries()
+    cowa.cowa_trace_start(0)
+    if dropped or not trace:
+        raise SystemExit("kernel trace of %s incomplete" % top)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -262,8 +332,6 @@ def run_cowa(args, rank, world, local_rank):
     t_step = sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps
     t_step, t_fwd, t_bwd, t_dec = max_over_ranks([t_step, t_fwd, t_bwd, t_dec], world, dev)
 
-    pairs = visible_pairs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, quad)
-    dec_keys = decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, quad)
     g = wl.Hq // wl.Hkv
     flops_step = pairs * 14 * wl.d + dec_keys * g * 4 * wl.d
     dec_bytes = dec_keys * 2 * wl.d * 2
@@ -278,13 +346,38 @@ def run_cowa(args, rank, world, local_rank):
     bwd_tflops = pairs * 10 * wl.d / (t_bwd * 1e-3) / 1e12
     fwd_tflops = pairs * 4 * wl.d / (t_fwd * 1e-3) / 1e12
     dec_gbs = dec_bytes / (t_dec * 1e-3) / 1e9
+
+    # per-kernel shares from the traced warm-up steps; the roofline kernel's
+    # time from its traced launches inside the timed steps
+    names = sorted(warm)
+    avg = max_over_ranks([warm[n][1] / warm[n][0] for n in names], world, dev)
+    total = sum(warm[n][1] for n in names)
+    kernels = {}
+    for n, a in zip(names, avg):
+        kernels[n] = {"launches": warm[n][0], "avg_ms": round(a, 5),
+                      "share": round(warm[n][1] / total, 4)}
+        if n in work:
+            bound, amount, unit, _ = work[n]
+            if bound == "tensor":
+                kernels[n]["tflops"] = round(amount / (a * 1e-3) / 1e12, 2)
+            else:
+                kernels[n]["gbs"] = round(amount / (a * 1e-3) / 1e9, 1)
+    bound, amount, unit, how = work[top]
+    a_ms = max_over_ranks([sum(ms for _, ms in trace) / len(trace)], world, dev)[0]
+    if bound == "tensor":
+        achieved, peak, runit = amount / (a_ms * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        psrc = "%s bf16_tflops (burst: the kernel runs %.2f ms inside a %.2f ms step)" % (
+            peak_src, a_ms, t_step)
+    else:
+        achieved, peak, runit = amount / (a_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        psrc = "%s hbm_gbs" % peak_src
     roofline = {
-        "kernel": "cowa_bwd (dK/dV + dQ passes)",
-        "bound": "tensor", "achieved": round(bwd_tflops, 2), "peak": peaks["bf16_tflops"],
-        "unit": "TFLOP/s", "frac": round(bwd_tflops / peaks["bf16_tflops"], 4),
-        "peak_source": "%s bf16_tflops (burst)" % peak_src,
-        "traffic": load_traffic("bwd", wl.name),
-        "algorithmic": "10*d flops per visible pair, %d pairs" % pairs,
+        "kernel": top, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
+        "unit": runit, "frac": round(achieved / peak, 4), "peak_source": psrc,
+        "traffic": load_traffic(top, wl.name),
+        "algorithmic": "%s per launch: %s" % (unit, how),
+        "avg_launch_ms": round(a_ms, 5), "launches_timed": len(trace),
+        "timing": "CUDA events around each launch of the kernel in the timed steps, on its stream",
     }
     result = {
         "metric": "effective TFLOP/s on visible pairs (fwd/bwd) & decode GB/s, % of B200 roofline",
@@ -304,6 +397,8 @@ def run_cowa(args, rank, world, local_rank):
             "decode_ms": round(t_dec, 4), "decode_gbs": round(dec_gbs, 1),
             "decode_frac": round(dec_gbs / peaks["hbm_gbs"], 4),
             "visible_pairs": pairs, "decode_visible_keys": dec_keys,
+            "kernels": kernels,
+            "kernels_from": "CUDA events around every library launch of the traced warm-up steps",
         },
         "roofline": roofline,
         "clocks": clocks.summary(),

@@ -99,6 +99,30 @@ COWA_API int cowa_abi_version(void);
 COWA_API uint64_t cowa_launch_count(void);
 
 /*
+ * Kernel trace, a measurement aid with no counterpart in the paper.
+ * cowa_trace_start(capacity, only) creates `capacity` CUDA event pairs on
+ * the current device and turns tracing on (capacity 0 turns it off and frees
+ * them); any earlier trace is discarded.  While on, each kernel the library
+ * launches on that device -- only the kernel named `only`, unless `only` is
+ * NULL or "" -- records one pair on its own stream, bracketing that launch
+ * alone; launches past the capacity, or on another device, are counted by
+ * cowa_trace_dropped() and not recorded.  cowa_trace_stop() stops
+ * recording and keeps the records.  cowa_trace_entry(i, &name, &ms) waits for
+ * record i (0 <= i < cowa_trace_size()) and gives the kernel's name (a
+ * static string: "fwd_sm100", "dkdv_sm100", "dq_sm100", "bwd_prep",
+ * "decode_split", "decode_combine", "schedule", ...) and its duration in
+ * milliseconds.  Start/stop are not meant to race with launches from other
+ * host threads; entries stay valid until the next cowa_trace_start.
+ * Errors: COWA_ERR_INVALID_ARG (capacity outside 0..2^20, `only` of 64
+ * characters or more, index out of range, NULL output), COWA_ERR_CUDA (event creation or timing failed).
+ */
+COWA_API int cowa_trace_start(int64_t capacity, const char *only);
+COWA_API int cowa_trace_stop(void);
+COWA_API int64_t cowa_trace_size(void);
+COWA_API int64_t cowa_trace_dropped(void);
+COWA_API int cowa_trace_entry(int64_t i, const char **name, float *ms);
+
+/*
  * Default quadruple: G = 0 and W = ceil((Lk - N) / Hkv), clamped at 0, so
  * the Hkv long windows exactly cover distances N .. Lk-1.  Hkv here is the
  * GLOBAL number of KV heads.

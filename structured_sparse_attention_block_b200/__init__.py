@@ -28,7 +28,7 @@ import torch
 __all__ = ["CowaError", "cowa_fwd", "cowa_bwd", "cowa_decode", "cowa_default_quad",
            "cowa_tile_classes", "cowa_fwd_workspace_size", "cowa_bwd_workspace_size",
            "cowa_decode_workspace_size", "cowa_get_device_error", "cowa_launch_count",
-           "cowa_decode_noalloc",
+           "cowa_decode_noalloc", "cowa_trace_start", "cowa_trace_stop", "cowa_trace_entries",
            "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -101,6 +101,14 @@ def lib():
         L.cowa_tile_classes.argtypes = [i64, i64, i64, Quad, i32, i32, ctypes.c_int, vp, vp, sz, vp]
         L.cowa_get_device_error.restype = ctypes.c_int
         L.cowa_get_device_error.argtypes = [vp]
+        L.cowa_trace_start.restype = ctypes.c_int
+        L.cowa_trace_start.argtypes = [i64, ctypes.c_char_p]
+        L.cowa_trace_stop.restype = ctypes.c_int
+        L.cowa_trace_size.restype = i64
+        L.cowa_trace_dropped.restype = i64
+        L.cowa_trace_entry.restype = ctypes.c_int
+        L.cowa_trace_entry.argtypes = [i64, ctypes.POINTER(ctypes.c_char_p),
+                                       ctypes.POINTER(ctypes.c_float)]
         _lib = L
     return _lib
 
@@ -306,6 +314,29 @@ def cowa_tile_classes(Lq, Lk, kv_head, quad, BM, BN=64, transposed=False, device
 def cowa_launch_count() -> int:
     """Kernels the library has launched in this process (all devices)."""
     return int(lib().cowa_launch_count())
+
+
+def cowa_trace_start(capacity: int, only: str = None) -> None:
+    """Record a CUDA event pair around each of the next ``capacity`` library
+    launches on the current device -- of the kernel named ``only``, if given
+    (0 turns tracing off)."""
+    _check(lib().cowa_trace_start(int(capacity), only.encode() if only else None))
+
+
+def cowa_trace_stop() -> None:
+    _check(lib().cowa_trace_stop())
+
+
+def cowa_trace_entries():
+    """(kernel name, milliseconds) of every traced launch, in launch order,
+    and the number of launches that were not recorded."""
+    L = lib()
+    out = []
+    name, ms = ctypes.c_char_p(), ctypes.c_float()
+    for i in range(int(L.cowa_trace_size())):
+        _check(L.cowa_trace_entry(i, ctypes.byref(name), ctypes.byref(ms)))
+        out.append((name.value.decode(), float(ms.value)))
+    return out, int(L.cowa_trace_dropped())
 
 
 def cowa_get_device_error(device=None):

@@ -10,6 +10,8 @@
 #include "kernels.cuh"
 
 #include <atomic>
+#include <mutex>
+#include <vector>
 
 namespace cowa {
 __device__ int g_cowa_device_error = 0;
@@ -19,7 +21,65 @@ __device__ int g_cowa_device_error = 0;
 int set_error_detail(int status, const char *detail);
 
 static std::atomic<unsigned long long> g_launches{0};
-void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+// Kernel trace: while on, every launch records an event pair on its stream.
+// The events are created up front by cowa_trace_start so that recording
+// costs two cudaEventRecord calls per launch and no allocation.
+struct TraceRec {
+    const char *name;
+    cudaEvent_t a, b;
+};
+static std::mutex g_trace_mu;
+static std::atomic<int> g_trace_on{0};
+static int g_trace_dev = -1;
+static std::vector<TraceRec> g_trace;  // capacity entries, events created
+static char g_trace_only[64] = "";     // trace only this kernel ("" = all)
+static size_t g_trace_used = 0;
+static size_t g_trace_dropped = 0;
+static thread_local long long tl_open = -1;  // record opened by launch_begin
+
+void launch_begin(const char *name, cudaStream_t st)
+{
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    tl_open = -1;
+    if (!g_trace_on.load(std::memory_order_acquire)) return;
+    if (g_trace_only[0] && strcmp(name, g_trace_only) != 0) return;
+    int dev = -1;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    if (!g_trace_on.load(std::memory_order_relaxed) || dev != g_trace_dev ||
+        g_trace_used == g_trace.size()) {
+        ++g_trace_dropped;
+        return;
+    }
+    TraceRec &r = g_trace[g_trace_used];
+    r.name = name;
+    if (cudaEventRecord(r.a, st) != cudaSuccess) {
+        ++g_trace_dropped;
+        return;
+    }
+    tl_open = (long long)g_trace_used++;
+}
+
+void launch_end(cudaStream_t st)
+{
+    if (tl_open < 0) return;
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    if ((size_t)tl_open < g_trace_used && cudaEventRecord(g_trace[tl_open].b, st) != cudaSuccess)
+        g_trace[tl_open].name = nullptr;  // unusable record
+    tl_open = -1;
+}
+
+void trace_clear_locked()
+{
+    for (TraceRec &r : g_trace) {
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    g_trace.clear();
+    g_trace_used = g_trace_dropped = 0;
+    g_trace_dev = -1;
+}
 }
 
 namespace {
@@ -79,6 +139,8 @@ int *device_error_word()
 
 constexpr long long kMaxLen = 1ll << 30;
 
+long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int check_quad(cowa_quad_t q)
@@ -113,6 +175,11 @@ int check_shape(const cowa_shape_t *s, cowa_quad_t q, bool decode)
         return fail(COWA_ERR_INVALID_ARG, "negative size in shape");
     if (s->Lq >= kMaxLen || s->Lk >= kMaxLen || s->B > 65535 || s->Hq > 65535 || s->Hkv > 65535)
         return fail(COWA_ERR_UNSUPPORTED, "sequence length must be < 2^30, B/heads <= 65535");
+    // the tiled kernels use 1-D grids of (tile, head, batch) blocks; no
+    // problem that fits in device memory comes near this bound
+    if (!decode && (s->B * s->Hq * cdiv(s->Lq, 32) > 0x7fffffffll ||
+                    s->B * s->Hkv * cdiv(s->Lk, 32) > 0x7fffffffll))
+        return fail(COWA_ERR_UNSUPPORTED, "B * heads * length / 32 exceeds 2^31 - 1");
     if (s->Hq > 0 && (s->Hkv == 0 || s->Hq % s->Hkv))
         return fail(COWA_ERR_INVALID_ARG, "Hq=%lld is not a multiple of Hkv=%lld", (long long)s->Hq,
                     (long long)s->Hkv);
@@ -156,7 +223,6 @@ void fill_common(P &p, const cowa_shape_t *s, cowa_quad_t q, float scale)
 
 size_t sched_bytes(long long heads, long long tiles) { return align256((size_t)(heads * tiles) * 8 * sizeof(int)); }
 
-long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
 int decode_splits(const cowa_shape_t *s, cowa_quad_t q, int sms)
 {
@@ -198,6 +264,75 @@ const char *cowa_last_error_detail(void) { return tl_detail; }
 int cowa_abi_version(void) { return COWA_ABI_VERSION; }
 
 uint64_t cowa_launch_count(void) { return cowa::g_launches.load(std::memory_order_relaxed); }
+
+int cowa_trace_start(int64_t capacity, const char *only)
+{
+    if (capacity < 0 || capacity > (1 << 20))
+        return fail(COWA_ERR_INVALID_ARG, "trace capacity %lld outside 0 .. 2^20", (long long)capacity);
+    if (only && strlen(only) >= sizeof cowa::g_trace_only)
+        return fail(COWA_ERR_INVALID_ARG, "trace filter longer than %d characters",
+                    (int)sizeof cowa::g_trace_only - 1);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    cowa::g_trace_on.store(0, std::memory_order_release);
+    std::lock_guard<std::mutex> lk(cowa::g_trace_mu);
+    cowa::trace_clear_locked();
+    cowa::g_trace.reserve((size_t)capacity);
+    for (int64_t i = 0; i < capacity; ++i) {
+        cowa::TraceRec r{nullptr, nullptr, nullptr};
+        if ((e = cudaEventCreate(&r.a)) != cudaSuccess) break;
+        if ((e = cudaEventCreate(&r.b)) != cudaSuccess) {
+            cudaEventDestroy(r.a);
+            break;
+        }
+        cowa::g_trace.push_back(r);
+    }
+    if (e != cudaSuccess) {
+        cowa::trace_clear_locked();
+        return cuda_fail(e, "cudaEventCreate");
+    }
+    cowa::g_trace_dev = dev;
+    snprintf(cowa::g_trace_only, sizeof cowa::g_trace_only, "%s", only ? only : "");
+    cowa::g_trace_on.store(capacity > 0 ? 1 : 0, std::memory_order_release);
+    return COWA_OK;
+}
+
+int cowa_trace_stop(void)
+{
+    cowa::g_trace_on.store(0, std::memory_order_release);
+    return COWA_OK;
+}
+
+int64_t cowa_trace_size(void)
+{
+    std::lock_guard<std::mutex> lk(cowa::g_trace_mu);
+    return (int64_t)cowa::g_trace_used;
+}
+
+int64_t cowa_trace_dropped(void)
+{
+    std::lock_guard<std::mutex> lk(cowa::g_trace_mu);
+    return (int64_t)cowa::g_trace_dropped;
+}
+
+int cowa_trace_entry(int64_t i, const char **name, float *ms)
+{
+    std::lock_guard<std::mutex> lk(cowa::g_trace_mu);
+    if (i < 0 || (size_t)i >= cowa::g_trace_used || !name || !ms)
+        return fail(COWA_ERR_INVALID_ARG, "trace entry %lld of %lld (or NULL output)", (long long)i,
+                    (long long)cowa::g_trace_used);
+    const cowa::TraceRec &r = cowa::g_trace[(size_t)i];
+    if (!r.name) return fail(COWA_ERR_CUDA, "trace entry %lld has no end event", (long long)i);
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+    float t = 0.f;
+    e = cudaEventElapsedTime(&t, r.a, r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+    *name = r.name;
+    *ms = t;
+    return COWA_OK;
+}
 
 cowa_quad_t cowa_default_quad(int64_t Lk, int64_t Hkv, int32_t S, int32_t N)
 {

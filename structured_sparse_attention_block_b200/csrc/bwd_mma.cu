@@ -411,23 +411,26 @@ static cudaError_t launch_bwd_d(const AttnParams &p, cudaStream_t st)
     }
     const long long rows = (long long)p.B * p.Hq * p.Lq;
     if (rows > 0) {
+        launch_begin("delta_mma", st);
         delta_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
-        note_launches(1);
+        launch_end(st);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.nkt > 0) {
         dim3 g1(p.nkt, p.Hkv, p.B);
+        launch_begin("dkdv_mma", st);
         dkdv_mma_kernel<D, QB><<<g1, 128, smem_kv, st>>>(p);
-        note_launches(1);
+        launch_end(st);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     const int nqt = (p.Lq + kBwdBM - 1) / kBwdBM;
     if (nqt > 0) {
         dim3 g2(nqt, p.Hq, p.B);
+        launch_begin("dq_mma", st);
         dq_mma_kernel<D><<<g2, 128, smem_q, st>>>(p);
-        note_launches(1);
+        launch_end(st);
         e = cudaGetLastError();
     }
     return e;

@@ -17,12 +17,20 @@
 //        dV += P^T dO,  dK += dS^T Q                   (MMA, P^T and dS^T from
 //                                                       tensor memory)
 //    Two warpgroups take alternate tasks so one computes while the MMAs of
-//    the other run.  dK is scaled by softmax_scale in the epilogue.
+//    the other run.  Warpgroup x releases S^T/dP^T of task u as soon as it
+//    has read them (S_FREE) and the MMA thread issues S^T/dP^T of task u+2
+//    into the same buffer before the gradient MMAs of task u, so the next
+//    task's scores are ready when the warpgroup finishes; P^T/dS^T of task
+//    u+2 are written only after those gradient MMAs complete (G_DONE).
+//    dK is scaled by softmax_scale in the epilogue.
 //
 // 3. dq_sm100_kernel, query-tile major like the forward: per visible key tile
 //        S = Q K^T,  dP = dO V^T,  dS = P (dP - delta),  dQ += dS K.
 //    For d = 64 a CTA takes two query heads of a GQA group (same mask, same
-//    K/V tiles) with one warpgroup each.
+//    K/V tiles) with one warpgroup each.  As in the dK/dV pass, S and dP of
+//    tile t+1 are issued once the warpgroup has read those of tile t
+//    (S_FREE), ahead of dQ += dS(t) K_t; dS(t+1) is written after that dQ
+//    MMA completes (DONE).
 //
 // The elementwise warpgroups never read or write tensor-memory columns that
 // an MMA still uses: S/dP and P/dS live in separate regions, and a
@@ -99,7 +107,7 @@ struct KvCfg {
     static constexpr int STAGE_BYTES = (2 * QT_BYTES + LSD_BYTES + 1023) / 1024 * 1024;
     // tensor memory: dK, dV, then two buffers of S^T, dP^T, P^T (bf16), dS^T (bf16)
     static constexpr int T_DK = 0, T_DV = D, T_BUF = 2 * D, BUF = 3 * BM;
-    static constexpr int NBAR = 7 + 2 * ST;
+    static constexpr int NBAR = 11 + 2 * ST;
     static constexpr int SMEM = 1024 + 2 * KV_BYTES + ST * STAGE_BYTES + 8 * NBAR + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BM, 0, 0);
     static constexpr uint32_t IDESC_G = idesc_bf16(128, D, 0, 1);
@@ -132,9 +140,12 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
     auto P_FULL = [&](int x) { return bar0 + 8u * (3 + 2 * ST + x); };
     const uint32_t DONE = bar0 + 8u * (5 + 2 * ST);
     const uint32_t FIN = bar0 + 8u * (6 + 2 * ST);
+    auto S_FREE = [&](int x) { return bar0 + 8u * (7 + 2 * ST + x); };
+    auto G_DONE = [&](int x) { return bar0 + 8u * (9 + 2 * ST + x); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int kt = blockIdx.x, hl = blockIdx.y, b = blockIdx.z;
+    const TilePos pos = tile_pos(p.Hkv, p.B);
+    const int kt = pos.step, hl = pos.slot, b = pos.b;  // sink keys first
     const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
     const int delta_pos = p.Lk - p.Lq;
     const int c0 = kt * BN;
@@ -164,6 +175,8 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
         for (int x = 0; x < 2; ++x) {
             mbar_init(S_FULL(x), 1);
             mbar_init(P_FULL(x), 128);
+            mbar_init(S_FREE(x), 4);  // one arrival per warp
+            mbar_init(G_DONE(x), 1);
         }
         mbar_init(DONE, 1);
         mbar_init(FIN, 1);
@@ -247,13 +260,19 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
                            sdesc(stage_q(s) + k2 * 2048, BM * 128, 1024), C::IDESC_G, acc);
                 }
                 mma_commit(Q_EMPTY(s));
+                mma_commit(G_DONE(x));
                 return true;
             };
             if (ok && ntask > 0) ok = sdp(0);
             if (ok && ntask > 1) ok = sdp(1);
             for (int u = 0; ok && u < ntask; ++u) {
-                if (!(ok = grad(u))) break;
-                if (u + 2 < ntask) ok = sdp(u + 2);
+                if (u + 2 < ntask) {
+                    // warpgroup u % 2 holds S^T and dP^T of task u in registers
+                    if (!(ok = mbar_wait(S_FREE(u & 1), (u >> 1) & 1, p.err, abort_flag))) break;
+                    tc_fence_after();
+                    if (!(ok = sdp(u + 2))) break;
+                }
+                ok = grad(u);
             }
             mma_commit(DONE);
             mma_commit(FIN);
@@ -307,6 +326,12 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
                     vis = span(jg, snk_hi) | span(jg, nr_hi) | span(lg_lo, lg_hi);
                 }
                 tmem_wait_ld();
+                if (c == BM / 32 - 1) {
+                    // all of S^T and dP^T read: S^T/dP^T of task u+2 may land
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(S_FREE(x));
+                }
                 uint32_t pk[16], dk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -322,9 +347,17 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
                     pk[e] = pack2(pr.x, pr.y);
                     dk[e] = pack2(ds.x, ds.y);
                 }
+                if (c == 0 && k > 0) {
+                    // the gradient MMAs of task u-2 read P^T/dS^T of this buffer
+                    // (G_DONE(x) has completed k-1 or k phases)
+                    ok = __all_sync(0xffffffffu, mbar_wait(G_DONE(x), (k - 1) & 1, p.err, abort_flag));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
                 tmem_st16(tb + 2 * BM + c * 16, pk);
                 tmem_st16(tb + 2 * BM + BM / 2 + c * 16, dk);
             }
+            if (!ok) break;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(P_FULL(x));
@@ -379,7 +412,7 @@ struct DqCfg {
     // tensor memory per slot: S, dP, dS (bf16), dQ
     static constexpr int SLOT = D == 128 ? 512 : 256;
     static constexpr int T_S = 0, T_DP = BN, T_DS = 2 * BN, T_DQ = D == 128 ? 384 : 192;
-    static constexpr int NBAR = 10 + 2 * ST;
+    static constexpr int NBAR = 12 + 2 * ST;
     static constexpr int SMEM = 1024 + 2 * NSLOT * QT_BYTES + ST * STAGE_BYTES + 8 * NBAR + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
     static constexpr uint32_t IDESC_Q = idesc_bf16(128, D, 0, 1);
@@ -409,13 +442,15 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
     auto DS_FULL = [&](int x) { return bar0 + 8u * (3 + 2 * ST + x); };
     auto DONE = [&](int x) { return bar0 + 8u * (5 + 2 * ST + x); };
     const uint32_t FIN = bar0 + 8u * (7 + 2 * ST);
+    auto S_FREE = [&](int x) { return bar0 + 8u * (8 + 2 * ST + x); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int qt = gridDim.x - 1 - blockIdx.x;
-    const int hl = blockIdx.y / a.npair, pair = blockIdx.y % a.npair;
+    const TilePos pos = tile_pos(p.Hkv * a.npair, p.B);
+    const int qt = p.nqt - 1 - pos.step;  // long rows first
+    const int hl = pos.slot / a.npair, pair = pos.slot % a.npair;
     const int hq0 = hl * p.g + NSLOT * pair;
     const int nslot = min(NSLOT, p.g - NSLOT * pair);
-    const int b = blockIdx.z;
+    const int b = pos.b;
     const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
     const int delta_pos = p.Lk - p.Lq;
     const int i0 = qt * BM;
@@ -445,6 +480,7 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
             mbar_init(S_FULL(x), 1);
             mbar_init(DS_FULL(x), 128);
             mbar_init(DONE(x), 1);
+            mbar_init(S_FREE(x), 4);  // one arrival per warp
         }
         mbar_init(FIN, 1);
         *abort_flag = 0;
@@ -528,15 +564,16 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
                 }
             }
             for (int t = 0; ok && t < ntiles; ++t) {
-                const bool more = t + 1 < ntiles;
-                if (more) {
+                if (t + 1 < ntiles) {
                     if (!(ok = mbar_wait(KV_FULL((t + 1) % ST), ((t + 1) / ST) & 1, p.err, abort_flag))) break;
-                    tc_fence_after();
+                    for (int x = 0; x < nslot && ok; ++x) {
+                        // warpgroup x holds S_x(t) and dP_x(t) in registers
+                        if (!(ok = mbar_wait(S_FREE(x), t & 1, p.err, abort_flag))) break;
+                        tc_fence_after();
+                        sdp(x, t + 1);
+                    }
                 }
-                for (int x = 0; x < nslot && ok; ++x) {
-                    if (!(ok = dq(x, t))) break;
-                    if (more) sdp(x, t + 1);
-                }
+                for (int x = 0; x < nslot && ok; ++x) ok = dq(x, t);
                 mma_commit(KV_EMPTY(t % ST));
             }
             mma_commit(FIN);
@@ -579,6 +616,12 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
                     if (w.e > w.c) vis |= span_bits(prow - w.e + 1 - j0, prow - w.c - j0);
                 }
                 tmem_wait_ld();
+                if (c == BN / 32 - 1) {
+                    // all of S and dP read: those of tile t+1 may land
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(S_FREE(x));
+                }
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -592,8 +635,16 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
                     const float2 ds = __fmul2_rn(pr, tt);
                     pk[e] = pack2(ds.x, ds.y);
                 }
+                if (c == 0 && t > 0) {
+                    // dQ += dS(t-1) K reads the dS columns (DONE(x) has
+                    // completed t-1 or t phases)
+                    ok = __all_sync(0xffffffffu, mbar_wait(DONE(x), (t - 1) & 1, p.err, abort_flag));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
                 tmem_st16(ts + C::T_DS + c * 16, pk);
             }
+            if (!ok) break;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(DS_FULL(x));
@@ -653,8 +704,9 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, c
     }
     const long long rows = (long long)p.B * p.Hq * lq_pad;
     if (rows > 0) {
+        launch_begin("bwd_prep", st);
         bwd_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p, lsd, lq_pad);
-        note_launches(1);
+        launch_end(st);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -673,9 +725,11 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, c
     a.p.sched_t = sched_kv;
     a.p.nkt = nkt_kv;
     if (nkt_kv > 0) {
-        dim3 g1(nkt_kv, p.Hkv, p.B);
+        const unsigned g1 = tile_grid_blocks(nkt_kv, p.Hkv, p.B);
+        if (!g1) return cudaErrorInvalidConfiguration;
+        launch_begin("dkdv_sm100", st);
         dkdv_sm100_kernel<D><<<g1, 320, K::SMEM, st>>>(a);
-        note_launches(1);
+        launch_end(st);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -689,9 +743,11 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, c
     a.p.nqt = nqt_dq;
     a.npair = (p.g + Q::NSLOT - 1) / Q::NSLOT;
     if (nqt_dq > 0) {
-        dim3 g2(nqt_dq, p.Hkv * a.npair, p.B);
+        const unsigned g2 = tile_grid_blocks(nqt_dq, (long long)p.Hkv * a.npair, p.B);
+        if (!g2) return cudaErrorInvalidConfiguration;
+        launch_begin("dq_sm100", st);
         dq_sm100_kernel<D><<<g2, 320, Q::SMEM, st>>>(a);
-        note_launches(1);
+        launch_end(st);
         e = cudaGetLastError();
     }
     return e;

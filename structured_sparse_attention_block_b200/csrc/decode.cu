@@ -279,12 +279,14 @@ static cudaError_t launch_decode_d(const DecodeParams &p, cudaStream_t st)
         configured[dev & 63] = true;
     }
     dim3 grid(p.splits, p.Hkv, p.B);
+    launch_begin("decode_split", st);
     decode_split_kernel<D><<<grid, 128, smem, st>>>(p);
-    note_launches(1);
+    launch_end(st);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    launch_begin("decode_combine", st);
     decode_combine_kernel<D><<<p.B * p.Hq, 128, 0, st>>>(p);
-    note_launches(1);
+    launch_end(st);
     return cudaGetLastError();
 }
 

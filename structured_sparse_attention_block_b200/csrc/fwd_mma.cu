@@ -211,8 +211,9 @@ static cudaError_t launch_fwd_d(const AttnParams &p, cudaStream_t st)
         configured[dev & 63] = true;
     }
     dim3 grid(p.nqt, p.Hq, p.B);
+    launch_begin("fwd_mma", st);
     fwd_mma_kernel<D><<<grid, 256, smem, st>>>(p);
-    note_launches(1);
+    launch_end(st);
     return cudaGetLastError();
 }
 

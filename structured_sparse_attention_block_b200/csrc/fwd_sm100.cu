@@ -11,10 +11,11 @@
 //              x in {0, 1}: S_x(t) = Q_x K_t^T into S_x, and O_x += P_x(t) V_t
 //              with P_x(t) read from its own tensor-memory region (a later MMA
 //              writing S_x is not ordered after an earlier MMA's read of P from
-//              the same columns, so P never shares columns with S).  Order:
-//              S_0(0) S_1(0), then per tile PV_0(t) S_0(t+1) PV_1(t) S_1(t+1)
-//              (with S double-buffered, SDB, S_x(t+2) follows PV_x(t)), so
-//              each softmax warpgroup only waits on its own MMAs;
+//              the same columns, so P never shares columns with S).  S_x(t+1)
+//              is issued as soon as softmax x has pulled S_x(t) into registers
+//              (S_FREE), so the next score tile is computed while the softmax
+//              of the current one runs; PV_x(t) follows when P_x(t) is written
+//              (P_FULL).  Order per tile: S_0(t+1) S_1(t+1) PV_0(t) PV_1(t);
 //   warps 0-3  softmax of slot 0, warps 4-7 softmax of slot 1: thread r of a
 //              warpgroup owns query row r.  Pass 1 reads the row of S in
 //              32-column chunks and takes the max (edge tiles only apply the
@@ -30,11 +31,9 @@
 // reads its whole row of S_x with one tensor-memory round trip and keeps it
 // in registers.  Tensor-memory columns for d = 64: S_x at 128x, the bf16 row
 // sums L_x at 128x + 96, P_x at 256 + 64x, O_x at 384 + 64x; for d = 128:
-// S_x at 64x, P_x at 128 + 32x, L_x at 192 + 16x, O_x at 256 + 128x.  (A
-// double-buffered S with 64-key tiles, SDB, measured slower for d = 64: the
-// per-tile work shrinks and more tiles need the element mask.)  A tcgen05.commit tracks every earlier MMA of the issuing
-// thread, so S_x(t+1) complete implies PV_x(t) complete: P_x and O_x are free
-// to rewrite once the softmax holds S_x(t+1).
+// S_x at 64x, P_x at 128 + 32x, L_x at 192 + 16x, O_x at 256 + 128x.
+// Softmax x rewrites P_x and rescales O_x for tile t only after O_DONE_x says
+// PV_x(t-1) is complete.
 // Every mbarrier wait is bounded; a wait that runs out records a timeout in
 // the device error word and the CTA winds down.
 #include <cudaTypedefs.h>
@@ -58,21 +57,17 @@ template <int D>
 struct FwdCfg {
     static constexpr int BM = 128, BN = fwd5_bn(D);
     static constexpr int STAGES = 4;  // tiles t, t+1, t+2 are resident at once
-    static constexpr bool SDB = false;  // S double-buffered per slot (needs BN = 64 for d = 64)
-    // tensor-memory column of S_x (buffer sb), P_x, L_x, O_x
-    static constexpr __host__ __device__ int t_s(int x, int sb)
-    {
-        return SDB ? 256 * x + 64 * sb : (D == 128 ? 64 * x : 128 * x);
-    }
-    static constexpr __host__ __device__ int t_p(int x) { return SDB ? 256 * x + 128 : (D == 128 ? 128 + 32 * x : 256 + 64 * x); }
-    static constexpr __host__ __device__ int t_l(int x) { return SDB ? 256 * x + 160 : (D == 128 ? 192 + 16 * x : 128 * x + 96); }
-    static constexpr __host__ __device__ int t_o(int x) { return SDB ? 256 * x + 192 : (D == 128 ? 256 + 128 * x : 384 + 64 * x); }
+    // tensor-memory column of S_x, P_x, L_x, O_x
+    static constexpr __host__ __device__ int t_s(int x) { return D == 128 ? 64 * x : 128 * x; }
+    static constexpr __host__ __device__ int t_p(int x) { return D == 128 ? 128 + 32 * x : 256 + 64 * x; }
+    static constexpr __host__ __device__ int t_l(int x) { return D == 128 ? 192 + 16 * x : 128 * x + 96; }
+    static constexpr __host__ __device__ int t_o(int x) { return D == 128 ? 256 + 128 * x : 384 + 64 * x; }
     static constexpr int ONES_BYTES = 2048;  // 16 key rows x 128 bytes of bf16 1.0
     static constexpr int KB = D / 64;                 // 128-byte blocks along d
     static constexpr int Q_BYTES = BM * D * 2;        // one head's query tile
     static constexpr int KV_BYTES = BN * D * 2;       // one of K or V
     static constexpr int STAGE_BYTES = 2 * KV_BYTES;
-    static constexpr int NBAR = 10 + 2 * STAGES;
+    static constexpr int NBAR = 12 + 2 * STAGES;
     static constexpr int SMEM = 1024 + 2 * Q_BYTES + STAGES * STAGE_BYTES + ONES_BYTES + 8 * NBAR + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
     static constexpr uint32_t IDESC_O = idesc_bf16(128, D, 0, 1);
@@ -102,14 +97,16 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
     auto S_FULL = [&](int x) { return bar0 + 8u * (1 + 2 * ST + x); };
     auto P_FULL = [&](int x) { return bar0 + 8u * (3 + 2 * ST + x); };
     auto O_DONE = [&](int x) { return bar0 + 8u * (5 + 2 * ST + x); };
-    const uint32_t FIN = bar0 + 8u * (7 + 2 * ST);
+    auto S_FREE = [&](int x) { return bar0 + 8u * (7 + 2 * ST + x); };
+    const uint32_t FIN = bar0 + 8u * (9 + 2 * ST);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int qt = gridDim.x - 1 - blockIdx.x;  // long rows first
-    const int hl = blockIdx.y / a.npair, pair = blockIdx.y % a.npair;
+    const TilePos pos = tile_pos(p.Hkv * a.npair, p.B);
+    const int qt = p.nqt - 1 - pos.step;  // long rows first
+    const int hl = pos.slot / a.npair, pair = pos.slot % a.npair;
     const int hq0 = hl * p.g + 2 * pair;
     const int nslot = (2 * pair + 1 < p.g) ? 2 : 1;  // an odd group leaves the last head alone
-    const int b = blockIdx.z;
+    const int b = pos.b;
     const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
     const int delta = p.Lk - p.Lq;
     const int i0 = qt * BM;
@@ -139,6 +136,7 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             mbar_init(S_FULL(x), 1);
             mbar_init(P_FULL(x), 128);
             mbar_init(O_DONE(x), 1);
+            mbar_init(S_FREE(x), 4);  // one arrival per softmax warp
         }
         mbar_init(FIN, 1);
         *abort_flag = 0;
@@ -199,7 +197,7 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t ad = sdesc(sQ + x * C::Q_BYTES + (kk >> 2) * BM * 128 + (kk & 3) * 32, 16, 1024);
                     const uint64_t bd = sdesc(sk + (kk >> 2) * BN * 128 + (kk & 3) * 32, 16, 1024);
-                    mma_ss(tmem + C::t_s(x, t & 1), ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::t_s(x), ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(S_FULL(x));
             };
@@ -219,23 +217,22 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                 mma_commit(O_DONE(x));
                 return true;
             };
-            constexpr int AHEAD = C::SDB ? 2 : 1;  // S tiles issued ahead of the softmax
-            for (int t = 0; ok && t < AHEAD && t < ntiles; ++t) {
-                if (!(ok = mbar_wait(KV_FULL(t % ST), (t / ST) & 1, p.err, abort_flag))) break;
+            if (ntiles > 0 && (ok = ok && mbar_wait(KV_FULL(0), 0, p.err, abort_flag))) {
                 tc_fence_after();
-                for (int x = 0; x < nslot; ++x) qk(x, t);
+                for (int x = 0; x < nslot; ++x) qk(x, 0);
             }
             for (int t = 0; ok && t < ntiles; ++t) {
-                const int tn = t + AHEAD;  // the tile whose S follows PV_x(t)
-                const bool more = tn < ntiles;
-                if (more) {
+                const int tn = t + 1;
+                if (tn < ntiles) {
                     if (!(ok = mbar_wait(KV_FULL(tn % ST), (tn / ST) & 1, p.err, abort_flag))) break;
-                    tc_fence_after();
+                    for (int x = 0; x < nslot && ok; ++x) {
+                        // softmax x holds S_x(t) in registers: S_x may be rewritten
+                        if (!(ok = mbar_wait(S_FREE(x), t & 1, p.err, abort_flag))) break;
+                        tc_fence_after();
+                        qk(x, tn);
+                    }
                 }
-                for (int x = 0; x < nslot && ok; ++x) {
-                    if (!(ok = pv(x, t))) break;
-                    if (more) qk(x, tn);
-                }
+                for (int x = 0; x < nslot && ok; ++x) ok = pv(x, t);
                 mma_commit(KV_EMPTY(t % ST));  // both heads are done with K_t and V_t
             }
             mma_commit(FIN);
@@ -257,7 +254,7 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), t & 1, p.err, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t tS = tmem + C::t_s(x, t & 1) + lane_off;
+            const uint32_t tS = tmem + C::t_s(x) + lane_off;
             const int kt = tile_of(t);
             const bool full = tile_full(pa, pb, kt * BN, BN, p.Lk, w);
             // One read of the row of S: all chunks are requested back to back and
@@ -289,6 +286,10 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                 }
             }
             tmem_wait_ld();
+            // the row is in registers: S_x(t+1) may overwrite S_x
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(S_FREE(x));
             if (!full) {
 #pragma unroll
                 for (int e = 0; e < BN; ++e)
@@ -306,8 +307,9 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             }
             const float smax = fmaxf(max3(mx4[0], mx4[1], mx4[2]), mx4[3]);
             const float tmax = smax * p.scale_log2;  // scale > 0 keeps the order
-            // P_x and O_x are rewritten below: PV_x(t-1) must be complete (it
-            // almost always is by now; O_DONE(x) has completed t-1 or t phases)
+            // P_x and O_x are rewritten below: PV_x(t-1) must be complete
+            // (O_DONE(x) has completed t-1 or t phases: PV_x(t) waits for the
+            // P_FULL arrival below)
             if (t > 0) {
                 ok = __all_sync(0xffffffffu, mbar_wait(O_DONE(x), (t - 1) & 1, p.err, abort_flag));
                 if (!ok) break;
@@ -469,9 +471,11 @@ static cudaError_t launch_fwd5_d(const AttnParams &p, cudaStream_t st)
         !make_bshd_map(&a.tk, p.k, D, p.Lk, p.Hkv, p.B, p.ks, C::BN) ||
         !make_bshd_map(&a.tv, p.v, D, p.Lk, p.Hkv, p.B, p.vs, C::BN))
         return cudaErrorInvalidValue;
-    dim3 grid(p.nqt, p.Hkv * a.npair, p.B);
-    fwd_sm100_kernel<D><<<grid, 320, C::SMEM, st>>>(a);
-    note_launches(1);
+    const unsigned blocks = tile_grid_blocks(p.nqt, (long long)p.Hkv * a.npair, p.B);
+    if (!blocks) return cudaErrorInvalidConfiguration;
+    launch_begin("fwd_sm100", st);
+    fwd_sm100_kernel<D><<<blocks, 320, C::SMEM, st>>>(a);
+    launch_end(st);
     return cudaGetLastError();
 }
 

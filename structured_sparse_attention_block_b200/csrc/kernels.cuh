@@ -41,8 +41,11 @@ struct DecodeParams {
     int *err;
 };
 
-// api.cu: process-wide count of kernels this library has launched
-void note_launches(int n);
+// api.cu: every kernel launch of the library is bracketed by these two calls:
+// they count launches and, while tracing is on, record a CUDA event pair on
+// the launching stream under the kernel's name.
+void launch_begin(const char *name, cudaStream_t st);
+void launch_end(cudaStream_t st);
 
 // schedule.cu
 cudaError_t launch_schedule(int *sched, int Hkv, int kv_head_offset, int Lq,
@@ -79,6 +82,33 @@ constexpr int kBwd5QTile = 128;     // queries per dQ CTA
 __host__ __device__ constexpr int bwd5_kv_bm(int D) { return D == 128 ? 32 : 64; }    // queries per dK/dV task
 __host__ __device__ constexpr int bwd5_dq_bn(int D) { return D == 128 ? 128 : 64; }   // keys per dQ tile
 inline long long bwd5_lq_pad(long long Lq) { return (Lq + 63) / 64 * 64; }
+
+// Launch order of the tiled tcgen05 kernels: a 1-D grid whose block index
+// runs over (head slot, batch) fastest and over the tile step slowest.  The
+// launcher maps step 0 to the heaviest tile of every head (the last query
+// tile for the query-major passes, the first key tile, which holds the sink
+// keys, for the key-major pass), so the long CTAs start in the first waves
+// and the short ones fill the tail.
+struct TilePos {
+    int step, slot, b;
+};
+__device__ __forceinline__ TilePos tile_pos(int nslot, int B)
+{
+    const unsigned per = (unsigned)nslot * (unsigned)B;
+    const unsigned lin = blockIdx.x;
+    TilePos t;
+    t.step = (int)(lin / per);
+    const unsigned r = lin - (unsigned)t.step * per;
+    t.b = (int)(r / (unsigned)nslot);
+    t.slot = (int)(r - (unsigned)t.b * (unsigned)nslot);
+    return t;
+}
+// Blocks of such a grid, or 0 when it would exceed the 2^31 - 1 limit.
+inline unsigned tile_grid_blocks(long long ntile, long long nslot, long long B)
+{
+    const long long n = ntile * nslot * B;
+    return n > 0x7fffffffll ? 0u : (unsigned)n;
+}
 
 // decode.cu
 cudaError_t launch_decode(const DecodeParams &p, int D, cudaStream_t st);

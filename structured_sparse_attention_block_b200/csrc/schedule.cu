@@ -43,9 +43,10 @@ cudaError_t launch_schedule(int *sched, int Hkv, int kv_head_offset, int Lq, int
     const int ntile = transposed ? (Lk + BN - 1) / BN : (Lq + BM - 1) / BM;
     if (ntile == 0 || Hkv == 0) return cudaSuccess;
     dim3 grid((ntile + 127) / 128, Hkv);
+    launch_begin("schedule", st);
     schedule_kernel<<<grid, 128, 0, st>>>(sched, kv_head_offset, Lq, Lk, S, N, G, W, BM, BN,
                                           transposed, ntile);
-    note_launches(1);
+    launch_end(st);
     return cudaGetLastError();
 }
 
@@ -79,9 +80,10 @@ cudaError_t launch_tile_classes(const int *sched, uint8_t *out, int kv_head, int
     const int nqt = (Lq + BM - 1) / BM, nkt = (Lk + BN - 1) / BN;
     const long long n = (long long)nqt * nkt;
     if (n == 0) return cudaSuccess;
+    launch_begin("tile_classes", st);
     tile_class_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
         sched, out, kv_head, Lq, Lk, S, N, G, W, BM, BN, transposed, nqt, nkt);
-    note_launches(1);
+    launch_end(st);
     return cudaGetLastError();
 }
 

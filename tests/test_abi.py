@@ -99,3 +99,14 @@ def test_oracle_is_not_reachable_from_the_product():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle|#include\s+\S*oracle|cowa_ref_",
                                      text, flags=re.M), f
+
+
+def test_trace_argument_errors(cowa):
+    lib = cowa.lib()
+    assert lib.cowa_trace_start(-1, None) == 1
+    assert lib.cowa_trace_start(1 << 21, None) == 1
+    assert lib.cowa_trace_start(4, b"x" * 64) == 1
+    assert lib.cowa_trace_stop() == 0
+    assert lib.cowa_trace_size() == 0
+    name, ms = ctypes.c_char_p(), ctypes.c_float()
+    assert lib.cowa_trace_entry(0, ctypes.byref(name), ctypes.byref(ms)) == 1
