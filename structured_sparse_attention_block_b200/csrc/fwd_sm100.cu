@@ -21,17 +21,16 @@
 //              32-column chunks and takes the max (edge tiles only apply the
 //              element mask); pass 2 re-reads S, writes P = 2^(s*scale - m) as
 //              bf16 to P_x and sums P in fp32 for the LSE.  The normalisation
-//              of O uses the sum of the bf16 P the PV product used, which a
-//              16-column MMA of P against a block of ones accumulates in
-//              tensor memory (L_x), so O is divided by exactly the weights it
-//              accumulated.  The O row is
+//              of O uses the sum of the bf16-rounded P the PV product used
+//              (unpacked from the packed pairs and summed alongside), so O is
+//              divided by exactly the weights it accumulated.  The O row is
 //              rescaled in tensor memory only when the max grows by more than
 //              2^8 (until then the stale max is a valid reference point).
 // Key tiles are 96 wide for d = 64 and 64 wide for d = 128: a softmax thread
 // reads its whole row of S_x with one tensor-memory round trip and keeps it
-// in registers.  Tensor-memory columns for d = 64: S_x at 128x, the bf16 row
-// sums L_x at 128x + 96, P_x at 256 + 64x, O_x at 384 + 64x; for d = 128:
-// S_x at 64x, P_x at 128 + 32x, L_x at 192 + 16x, O_x at 256 + 128x.
+// in registers.  Tensor-memory columns for d = 64: S_x at 128x, P_x at
+// 256 + 64x, O_x at 384 + 64x; for d = 128: S_x at 64x, P_x at 128 + 32x,
+// O_x at 256 + 128x.
 // Softmax x rewrites P_x and rescales O_x for tile t only after O_DONE_x says
 // PV_x(t-1) is complete.
 // Every mbarrier wait is bounded; a wait that runs out records a timeout in
@@ -57,21 +56,18 @@ template <int D>
 struct FwdCfg {
     static constexpr int BM = 128, BN = fwd5_bn(D);
     static constexpr int STAGES = 4;  // tiles t, t+1, t+2 are resident at once
-    // tensor-memory column of S_x, P_x, L_x, O_x
+    // tensor-memory column of S_x, P_x, O_x
     static constexpr __host__ __device__ int t_s(int x) { return D == 128 ? 64 * x : 128 * x; }
     static constexpr __host__ __device__ int t_p(int x) { return D == 128 ? 128 + 32 * x : 256 + 64 * x; }
-    static constexpr __host__ __device__ int t_l(int x) { return D == 128 ? 192 + 16 * x : 128 * x + 96; }
     static constexpr __host__ __device__ int t_o(int x) { return D == 128 ? 256 + 128 * x : 384 + 64 * x; }
-    static constexpr int ONES_BYTES = 2048;  // 16 key rows x 128 bytes of bf16 1.0
     static constexpr int KB = D / 64;                 // 128-byte blocks along d
     static constexpr int Q_BYTES = BM * D * 2;        // one head's query tile
     static constexpr int KV_BYTES = BN * D * 2;       // one of K or V
     static constexpr int STAGE_BYTES = 2 * KV_BYTES;
     static constexpr int NBAR = 12 + 2 * STAGES;
-    static constexpr int SMEM = 1024 + 2 * Q_BYTES + STAGES * STAGE_BYTES + ONES_BYTES + 8 * NBAR + 16;
+    static constexpr int SMEM = 1024 + 2 * Q_BYTES + STAGES * STAGE_BYTES + 8 * NBAR + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
     static constexpr uint32_t IDESC_O = idesc_bf16(128, D, 0, 1);
-    static constexpr uint32_t IDESC_L = idesc_bf16(128, 16, 0, 1);
 };
 
 template <int D>
@@ -86,8 +82,7 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
     unsigned char *sm = smem_raw + (base - raw);
     const uint32_t sQ = base;  // slot x at sQ + x * Q_BYTES
     const uint32_t sStage = base + 2 * C::Q_BYTES;
-    const uint32_t sOnes = sStage + ST * C::STAGE_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 2 * C::Q_BYTES + ST * C::STAGE_BYTES + C::ONES_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 2 * C::Q_BYTES + ST * C::STAGE_BYTES);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const uint32_t bar0 = smem_addr(bars);
@@ -151,12 +146,6 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         prefetch_tmap(&a.tk);
         prefetch_tmap(&a.tv);
     }
-    {
-        // bf16 1.0 everywhere in the ones block (any swizzle reads ones)
-        uint32_t *ones = reinterpret_cast<uint32_t *>(sm + 2 * C::Q_BYTES + ST * C::STAGE_BYTES);
-        for (int k = tid; k < C::ONES_BYTES / 4; k += blockDim.x) ones[k] = 0x3F803F80u;
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -201,18 +190,14 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                 }
                 mma_commit(S_FULL(x));
             };
-            auto pv = [&](int x, int t) -> bool {  // O_x += P_x(t) V_t, L_x += P_x(t) 1
+            auto pv = [&](int x, int t) -> bool {  // O_x += P_x(t) V_t
                 if (!mbar_wait(P_FULL(x), t & 1, p.err, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t sv = sStage + (t % ST) * C::STAGE_BYTES + C::KV_BYTES;
-                const uint64_t od = sdesc(sOnes, 128, 1024);
 #pragma unroll
                 for (int k2 = 0; k2 < BN / 16; ++k2) {
                     const uint64_t bd = sdesc(sv + k2 * 2048, BN * 128, 1024);
-                    const uint32_t pa_ = tmem + C::t_p(x) + k2 * 8;
-                    const uint32_t acc = (t > 0 || k2 > 0) ? 1u : 0u;
-                    mma_ts(tmem + C::t_o(x), pa_, bd, C::IDESC_O, acc);
-                    mma_ts(tmem + C::t_l(x), pa_, od, C::IDESC_L, acc);
+                    mma_ts(tmem + C::t_o(x), tmem + C::t_p(x) + k2 * 8, bd, C::IDESC_O, (t > 0 || k2 > 0) ? 1u : 0u);
                 }
                 mma_commit(O_DONE(x));
                 return true;
@@ -245,10 +230,9 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tP = tmem + C::t_p(x) + lane_off;
         const uint32_t tOx = tmem + C::t_o(x) + lane_off;
-        const uint32_t tLx = tmem + C::t_l(x) + lane_off;
         const int prow = pa + r;
         const bool active = x < nslot;
-        float m_run = -CUDART_INF_F, l = 0.f;
+        float m_run = -CUDART_INF_F, l = 0.f, lb = 0.f;  // fp32 and bf16-rounded sums of P
         bool ok = true;
         for (int t = 0; active && t < ntiles; ++t) {
             ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), t & 1, p.err, abort_flag));
@@ -322,9 +306,9 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             if (__any_sync(0xffffffffu, fix_o)) {
                 const float f = fix_o ? alpha : 1.f;
 #pragma unroll
-                for (int c = 0; c <= D / 16; ++c) {  // O, then the bf16 sums
+                for (int c = 0; c < D / 16; ++c) {
                     uint32_t o[16];
-                    const uint32_t ta = c < D / 16 ? tOx + c * 16 : tLx;
+                    const uint32_t ta = tOx + c * 16;
                     tmem_ld16(ta, o);
                     tmem_wait_ld();
 #pragma unroll
@@ -335,6 +319,7 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             }
             if (grow) {
                 l *= alpha;
+                lb *= alpha;
                 m_run = tmax;
             }
             const float nms = m_run == -CUDART_INF_F ? 0.f : -m_run;
@@ -343,20 +328,28 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             // over sr[e], already consumed
             const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(nms, nms);
             float2 la = make_float2(0.f, 0.f), lc = make_float2(0.f, 0.f);
+            float2 ba = make_float2(0.f, 0.f), bc = make_float2(0.f, 0.f);
 #pragma unroll
             for (int e = 0; e < BN / 2; ++e) {
                 const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
                                              sc2, nm2);
                 const float p0 = fast_ex2(xa.x), p1 = fast_ex2(xa.y);
-                if (e & 1)
+                const uint32_t pk = pack2(p0, p1);
+                // the two bf16 values as fp32 (low half: key 2e, high: key 2e+1)
+                const float2 pr = make_float2(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u));
+                if (e & 1) {
                     lc = __fadd2_rn(lc, make_float2(p0, p1));
-                else
+                    bc = __fadd2_rn(bc, pr);
+                } else {
                     la = __fadd2_rn(la, make_float2(p0, p1));
-                sr[e] = pack2(p0, p1);
+                    ba = __fadd2_rn(ba, pr);
+                }
+                sr[e] = pk;
             }
 #pragma unroll
             for (int c = 0; c < NC; ++c) tmem_st16(tP + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c * 16]));
             l += (la.x + la.y) + (lc.x + lc.y);
+            lb += (ba.x + ba.y) + (bc.x + bc.y);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(P_FULL(x));
@@ -371,13 +364,6 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         // epilogue: O / (sum of the bf16 P) in bf16, LSE (natural log) from the fp32 sum
         if (active) {
             const bool have = ok && ntiles > 0;
-            float lb = 0.f;  // sum of the bf16 P that O accumulated
-            if (have) {
-                uint32_t lv[16];
-                tmem_ld16(tLx, lv);
-                tmem_wait_ld();
-                lb = __uint_as_float(lv[0]);
-            }
             const float inv = (l > 0.f && lb > 0.f) ? 1.f / lb : 0.f;
             const int hq = hq0 + x;
             __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + b * p.os[0] +
