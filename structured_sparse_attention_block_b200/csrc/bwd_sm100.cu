@@ -228,56 +228,68 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA
-        if (lane == 0) {
-            bool ok = mbar_wait(KV_LOADED, 0, p.err, abort_flag);
-            auto sdp = [&](int u) -> bool {  // S^T, dP^T of task u into buffer u % 2
-                const int s = u % ST, x = u & 1;
-                if (!mbar_wait(Q_FULL(s), (u / ST) & 1, p.err, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t tb = tmem + C::T_BUF + x * C::BUF;
+        // the whole warp runs the loop; one elected lane issues
+        const uint32_t FULL = 0xffffffffu;
+        bool ok = __all_sync(FULL, mbar_wait(KV_LOADED, 0, p.err, abort_flag));
+        const uint64_t dk0 = sdesc(sK, 16, 1024), dv0 = sdesc(sV, 16, 1024);
+        const uint64_t dq0 = sdesc(stage_q(0), 16, 1024), ddo0 = sdesc(stage_do(0), 16, 1024);
+        const uint64_t dqm0 = sdesc(stage_q(0), BM * 128, 1024), ddom0 = sdesc(stage_do(0), BM * 128, 1024);
+        auto sdp = [&](int u) -> bool {  // S^T, dP^T of task u into buffer u % 2
+            const int s = u % ST, x = u & 1;
+            if (!__all_sync(FULL, mbar_wait(Q_FULL(s), (u / ST) & 1, p.err, abort_flag))) return false;
+            tc_fence_after();
+            const uint32_t tb = tmem + C::T_BUF + x * C::BUF;
+            const uint32_t so = (uint32_t)s * C::STAGE_BYTES;
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ko = (kk >> 2) * BN * 128 + (kk & 3) * 32;
-                    const uint32_t qo = (kk >> 2) * BM * 128 + (kk & 3) * 32;
-                    mma_ss(tb, sdesc(sK + ko, 16, 1024), sdesc(stage_q(s) + qo, 16, 1024), C::IDESC_S, kk > 0);
-                    mma_ss(tb + BM, sdesc(sV + ko, 16, 1024), sdesc(stage_do(s) + qo, 16, 1024), C::IDESC_S,
-                           kk > 0);
+                    const uint32_t qo = so + (kk >> 2) * BM * 128 + (kk & 3) * 32;
+                    mma_ss(tb, sdesc_add(dk0, ko), sdesc_add(dq0, qo), C::IDESC_S, kk > 0);
+                    mma_ss(tb + BM, sdesc_add(dv0, ko), sdesc_add(ddo0, qo), C::IDESC_S, kk > 0);
                 }
                 mma_commit(S_FULL(x));
-                return true;
-            };
-            auto grad = [&](int u) -> bool {  // dV += P^T dO, dK += dS^T Q
-                const int s = u % ST, x = u & 1;
-                if (!mbar_wait(P_FULL(x), (u >> 1) & 1, p.err, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t tb = tmem + C::T_BUF + x * C::BUF;
+            }
+            __syncwarp();
+            return true;
+        };
+        auto grad = [&](int u) -> bool {  // dV += P^T dO, dK += dS^T Q
+            const int s = u % ST, x = u & 1;
+            if (!__all_sync(FULL, mbar_wait(P_FULL(x), (u >> 1) & 1, p.err, abort_flag))) return false;
+            tc_fence_after();
+            const uint32_t tb = tmem + C::T_BUF + x * C::BUF;
+            const uint32_t so = (uint32_t)s * C::STAGE_BYTES;
+            if (elect_one()) {
 #pragma unroll
                 for (int k2 = 0; k2 < BM / 16; ++k2) {
                     const uint32_t acc = (u > 0 || k2 > 0) ? 1u : 0u;
-                    mma_ts(tmem + C::T_DV, tb + 2 * BM + k2 * 8, sdesc(stage_do(s) + k2 * 2048, BM * 128, 1024),
-                           C::IDESC_G, acc);
-                    mma_ts(tmem + C::T_DK, tb + 2 * BM + BM / 2 + k2 * 8,
-                           sdesc(stage_q(s) + k2 * 2048, BM * 128, 1024), C::IDESC_G, acc);
+                    mma_ts(tmem + C::T_DV, tb + 2 * BM + k2 * 8, sdesc_add(ddom0, so + k2 * 2048), C::IDESC_G, acc);
+                    mma_ts(tmem + C::T_DK, tb + 2 * BM + BM / 2 + k2 * 8, sdesc_add(dqm0, so + k2 * 2048), C::IDESC_G,
+                           acc);
                 }
                 mma_commit(Q_EMPTY(s));
                 mma_commit(G_DONE(x));
-                return true;
-            };
-            if (ok && ntask > 0) ok = sdp(0);
-            if (ok && ntask > 1) ok = sdp(1);
-            for (int u = 0; ok && u < ntask; ++u) {
-                if (u + 2 < ntask) {
-                    // warpgroup u % 2 holds S^T and dP^T of task u in registers
-                    if (!(ok = mbar_wait(S_FREE(u & 1), (u >> 1) & 1, p.err, abort_flag))) break;
-                    tc_fence_after();
-                    if (!(ok = sdp(u + 2))) break;
-                }
-                ok = grad(u);
             }
+            __syncwarp();
+            return true;
+        };
+        if (ok && ntask > 0) ok = sdp(0);
+        if (ok && ntask > 1) ok = sdp(1);
+        for (int u = 0; ok && u < ntask; ++u) {
+            if (u + 2 < ntask) {
+                // warpgroup u % 2 holds S^T and dP^T of task u in registers
+                if (!(ok = __all_sync(FULL, mbar_wait(S_FREE(u & 1), (u >> 1) & 1, p.err, abort_flag)))) break;
+                tc_fence_after();
+                if (!(ok = sdp(u + 2))) break;
+            }
+            ok = grad(u);
+        }
+        if (elect_one()) {
             mma_commit(DONE);
             mma_commit(FIN);
-            mbar_wait(FIN, 0, p.err, abort_flag);
         }
+        __syncwarp();
+        mbar_wait(FIN, 0, p.err, abort_flag);
     } else {
         // ---------------------------------------------- P^T and dS^T per key
         const int x = warp >> 2;
@@ -529,56 +541,67 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA
-        if (lane == 0) {
-            bool ok = mbar_wait(BAR_Q, 0, p.err, abort_flag);
-            auto sdp = [&](int x, int t) {  // S_x = Q_x K_t^T, dP_x = dO_x V_t^T
-                const uint32_t sk = sStage + (t % ST) * C::STAGE_BYTES, sv = sk + C::KV_BYTES;
-                const uint32_t ts = tmem + x * C::SLOT;
+        // the whole warp runs the loop; one elected lane issues
+        const uint32_t FULL = 0xffffffffu;
+        bool ok = __all_sync(FULL, mbar_wait(BAR_Q, 0, p.err, abort_flag));
+        const uint64_t dq0 = sdesc(sQ(0), 16, 1024), ddo0 = sdesc(sDO(0), 16, 1024);
+        const uint64_t dk0 = sdesc(sStage, 16, 1024), dv0 = sdesc(sStage + C::KV_BYTES, 16, 1024);
+        const uint64_t dkm0 = sdesc(sStage, BN * 128, 1024);
+        auto sdp = [&](int x, int t) {  // S_x = Q_x K_t^T, dP_x = dO_x V_t^T
+            const uint32_t so = (uint32_t)(t % ST) * C::STAGE_BYTES;
+            const uint32_t ts = tmem + x * C::SLOT;
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t qo = (kk >> 2) * BM * 128 + (kk & 3) * 32;
-                    const uint32_t ko = (kk >> 2) * BN * 128 + (kk & 3) * 32;
-                    mma_ss(ts + C::T_S, sdesc(sQ(x) + qo, 16, 1024), sdesc(sk + ko, 16, 1024), C::IDESC_S, kk > 0);
-                    mma_ss(ts + C::T_DP, sdesc(sDO(x) + qo, 16, 1024), sdesc(sv + ko, 16, 1024), C::IDESC_S,
-                           kk > 0);
+                    const uint32_t qo = x * 2 * C::QT_BYTES + (kk >> 2) * BM * 128 + (kk & 3) * 32;
+                    const uint32_t ko = so + (kk >> 2) * BN * 128 + (kk & 3) * 32;
+                    mma_ss(ts + C::T_S, sdesc_add(dq0, qo), sdesc_add(dk0, ko), C::IDESC_S, kk > 0);
+                    mma_ss(ts + C::T_DP, sdesc_add(ddo0, qo), sdesc_add(dv0, ko), C::IDESC_S, kk > 0);
                 }
                 mma_commit(S_FULL(x));
-            };
-            auto dq = [&](int x, int t) -> bool {  // dQ_x += dS_x K_t
-                if (!mbar_wait(DS_FULL(x), t & 1, p.err, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t sk = sStage + (t % ST) * C::STAGE_BYTES;
-                const uint32_t ts = tmem + x * C::SLOT;
+            }
+            __syncwarp();
+        };
+        auto dq = [&](int x, int t) -> bool {  // dQ_x += dS_x K_t
+            if (!__all_sync(FULL, mbar_wait(DS_FULL(x), t & 1, p.err, abort_flag))) return false;
+            tc_fence_after();
+            const uint32_t so = (uint32_t)(t % ST) * C::STAGE_BYTES;
+            const uint32_t ts = tmem + x * C::SLOT;
+            if (elect_one()) {
 #pragma unroll
                 for (int k2 = 0; k2 < BN / 16; ++k2)
-                    mma_ts(ts + C::T_DQ, ts + C::T_DS + k2 * 8, sdesc(sk + k2 * 2048, BN * 128, 1024), C::IDESC_Q,
+                    mma_ts(ts + C::T_DQ, ts + C::T_DS + k2 * 8, sdesc_add(dkm0, so + k2 * 2048), C::IDESC_Q,
                            (t > 0 || k2 > 0) ? 1u : 0u);
                 mma_commit(DONE(x));
-                return true;
-            };
-            if (ok && ntiles > 0) {
-                ok = mbar_wait(KV_FULL(0), 0, p.err, abort_flag);
-                if (ok) {
-                    tc_fence_after();
-                    for (int x = 0; x < nslot; ++x) sdp(x, 0);
-                }
             }
-            for (int t = 0; ok && t < ntiles; ++t) {
-                if (t + 1 < ntiles) {
-                    if (!(ok = mbar_wait(KV_FULL((t + 1) % ST), ((t + 1) / ST) & 1, p.err, abort_flag))) break;
-                    for (int x = 0; x < nslot && ok; ++x) {
-                        // warpgroup x holds S_x(t) and dP_x(t) in registers
-                        if (!(ok = mbar_wait(S_FREE(x), t & 1, p.err, abort_flag))) break;
-                        tc_fence_after();
-                        sdp(x, t + 1);
-                    }
-                }
-                for (int x = 0; x < nslot && ok; ++x) ok = dq(x, t);
-                mma_commit(KV_EMPTY(t % ST));
+            __syncwarp();
+            return true;
+        };
+        if (ok && ntiles > 0) {
+            ok = __all_sync(FULL, mbar_wait(KV_FULL(0), 0, p.err, abort_flag));
+            if (ok) {
+                tc_fence_after();
+                for (int x = 0; x < nslot; ++x) sdp(x, 0);
             }
-            mma_commit(FIN);
-            mbar_wait(FIN, 0, p.err, abort_flag);
         }
+        for (int t = 0; ok && t < ntiles; ++t) {
+            if (t + 1 < ntiles) {
+                if (!(ok = __all_sync(FULL, mbar_wait(KV_FULL((t + 1) % ST), ((t + 1) / ST) & 1, p.err, abort_flag))))
+                    break;
+                for (int x = 0; x < nslot && ok; ++x) {
+                    // warpgroup x holds S_x(t) and dP_x(t) in registers
+                    if (!(ok = __all_sync(FULL, mbar_wait(S_FREE(x), t & 1, p.err, abort_flag)))) break;
+                    tc_fence_after();
+                    sdp(x, t + 1);
+                }
+            }
+            for (int x = 0; x < nslot && ok; ++x) ok = dq(x, t);
+            if (elect_one()) mma_commit(KV_EMPTY(t % ST));
+            __syncwarp();
+        }
+        if (elect_one()) mma_commit(FIN);
+        __syncwarp();
+        mbar_wait(FIN, 0, p.err, abort_flag);
     } else {
         // ------------------------------------------------- dS per query row
         const int x = warp >> 2;

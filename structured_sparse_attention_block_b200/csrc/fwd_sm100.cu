@@ -178,51 +178,64 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA
-        if (lane == 0) {
-            bool ok = mbar_wait(BAR_Q, 0, p.err, abort_flag);
-            auto qk = [&](int x, int t) {  // S_x(t) = Q_x K_t^T
-                const uint32_t sk = sStage + (t % ST) * C::STAGE_BYTES;
+        // the whole warp runs the loop; one elected lane issues
+        const uint32_t FULL = 0xffffffffu;
+        bool ok = __all_sync(FULL, mbar_wait(BAR_Q, 0, p.err, abort_flag));
+        // descriptor bases: Q of slot 0, K and V of stage 0 (the others are
+        // fixed byte offsets from these)
+        const uint64_t dq0 = sdesc(sQ, 16, 1024);
+        const uint64_t dk0 = sdesc(sStage, 16, 1024);
+        const uint64_t dv0 = sdesc(sStage + C::KV_BYTES, BN * 128, 1024);
+        auto qk = [&](int x, int t) {  // S_x(t) = Q_x K_t^T
+            const uint32_t so = (uint32_t)(t % ST) * C::STAGE_BYTES;
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t ad = sdesc(sQ + x * C::Q_BYTES + (kk >> 2) * BM * 128 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = sdesc(sk + (kk >> 2) * BN * 128 + (kk & 3) * 32, 16, 1024);
+                    const uint32_t off = (kk & 3) * 32;
+                    const uint64_t ad = sdesc_add(dq0, x * C::Q_BYTES + (kk >> 2) * BM * 128 + off);
+                    const uint64_t bd = sdesc_add(dk0, so + (kk >> 2) * BN * 128 + off);
                     mma_ss(tmem + C::t_s(x), ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(S_FULL(x));
-            };
-            auto pv = [&](int x, int t) -> bool {  // O_x += P_x(t) V_t
-                if (!mbar_wait(P_FULL(x), t & 1, p.err, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t sv = sStage + (t % ST) * C::STAGE_BYTES + C::KV_BYTES;
+            }
+            __syncwarp();
+        };
+        auto pv = [&](int x, int t) -> bool {  // O_x += P_x(t) V_t
+            if (!__all_sync(FULL, mbar_wait(P_FULL(x), t & 1, p.err, abort_flag))) return false;
+            tc_fence_after();
+            const uint32_t so = (uint32_t)(t % ST) * C::STAGE_BYTES;
+            if (elect_one()) {
 #pragma unroll
-                for (int k2 = 0; k2 < BN / 16; ++k2) {
-                    const uint64_t bd = sdesc(sv + k2 * 2048, BN * 128, 1024);
-                    mma_ts(tmem + C::t_o(x), tmem + C::t_p(x) + k2 * 8, bd, C::IDESC_O, (t > 0 || k2 > 0) ? 1u : 0u);
-                }
+                for (int k2 = 0; k2 < BN / 16; ++k2)
+                    mma_ts(tmem + C::t_o(x), tmem + C::t_p(x) + k2 * 8, sdesc_add(dv0, so + k2 * 2048), C::IDESC_O,
+                           (t > 0 || k2 > 0) ? 1u : 0u);
                 mma_commit(O_DONE(x));
-                return true;
-            };
-            if (ntiles > 0 && (ok = ok && mbar_wait(KV_FULL(0), 0, p.err, abort_flag))) {
-                tc_fence_after();
-                for (int x = 0; x < nslot; ++x) qk(x, 0);
             }
-            for (int t = 0; ok && t < ntiles; ++t) {
-                const int tn = t + 1;
-                if (tn < ntiles) {
-                    if (!(ok = mbar_wait(KV_FULL(tn % ST), (tn / ST) & 1, p.err, abort_flag))) break;
-                    for (int x = 0; x < nslot && ok; ++x) {
-                        // softmax x holds S_x(t) in registers: S_x may be rewritten
-                        if (!(ok = mbar_wait(S_FREE(x), t & 1, p.err, abort_flag))) break;
-                        tc_fence_after();
-                        qk(x, tn);
-                    }
-                }
-                for (int x = 0; x < nslot && ok; ++x) ok = pv(x, t);
-                mma_commit(KV_EMPTY(t % ST));  // both heads are done with K_t and V_t
-            }
-            mma_commit(FIN);
-            mbar_wait(FIN, 0, p.err, abort_flag);
+            __syncwarp();
+            return true;
+        };
+        if (ntiles > 0 && (ok = ok && __all_sync(FULL, mbar_wait(KV_FULL(0), 0, p.err, abort_flag)))) {
+            tc_fence_after();
+            for (int x = 0; x < nslot; ++x) qk(x, 0);
         }
+        for (int t = 0; ok && t < ntiles; ++t) {
+            const int tn = t + 1;
+            if (tn < ntiles) {
+                if (!(ok = __all_sync(FULL, mbar_wait(KV_FULL(tn % ST), (tn / ST) & 1, p.err, abort_flag)))) break;
+                for (int x = 0; x < nslot && ok; ++x) {
+                    // softmax x holds S_x(t) in registers: S_x may be rewritten
+                    if (!(ok = __all_sync(FULL, mbar_wait(S_FREE(x), t & 1, p.err, abort_flag)))) break;
+                    tc_fence_after();
+                    qk(x, tn);
+                }
+            }
+            for (int x = 0; x < nslot && ok; ++x) ok = pv(x, t);
+            if (elect_one()) mma_commit(KV_EMPTY(t % ST));  // both heads are done with K_t and V_t
+            __syncwarp();
+        }
+        if (elect_one()) mma_commit(FIN);
+        __syncwarp();
+        mbar_wait(FIN, 0, p.err, abort_flag);
     } else {
         // -------------------------------------------------------- softmax
         const int x = warp >> 2;  // head slot of this warpgroup

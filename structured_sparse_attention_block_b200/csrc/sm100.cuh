@@ -72,6 +72,21 @@ __device__ __forceinline__ bool mbar_test_sleep(uint32_t bar, uint32_t parity, u
     return ok != 0;
 }
 
+// One lane of the (converged) warp: the issuing lane of a tcgen05
+// instruction.  The MMA role runs on the whole warp, reconverging after each
+// issue; commits from a warp whose other lanes have left the loop measured
+// several times slower.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // Waits for the phase of `parity` to complete.  Returns false (after
 // recording the timeout) if it does not within kWaitLimitNs, or at once if
 // the CTA is aborting.
@@ -205,6 +220,15 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 accumulate:
 // bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format,
 // 15 A major (0 = K), 16 B major (0 = K, 1 = MN), 17-22 N >> 3, 24-28 M >> 4.
+// `d` with its start-address field advanced by `bytes` (a multiple of 16).
+// The field holds shared-memory address / 16 in 14 bits, which no address
+// of a 227 KB allocation overflows, so only the low word changes.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes)
+{
+    const uint32_t lo = (uint32_t)d + (bytes >> 4), hi = (uint32_t)(d >> 32);
+    return ((uint64_t)hi << 32) | lo;
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn)
 {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
