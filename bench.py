@@ -405,6 +405,9 @@ def run_cowa(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": int(launches),
     }
+    if args.full_mask:
+        result["full_mask_control"] = run_full_mask(args, cowa, wl, q, k, v, do, qd, seqlens, dev, stream,
+                                                    flush, world, (t_fwd, t_bwd, t_dec))
     if args.decode_workload:
         result["decode_workload"] = run_decode_workload(args, cowa, dev, stream, flush, world, peaks, peak_src)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -450,6 +453,62 @@ def run_e2e(args, cowa, wl, q, k, v, do, qd, seqlens, quad, dev, stream, flush, 
     return {"ms": ms, "ms_per_step": round(ms, 4),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "path": "pinned host -> device copies, cowa_fwd/bwd/decode, device -> pinned host"}
+
+
+def run_full_mask(args, cowa, wl, q, k, v, do, qd, seqlens, dev, stream, flush, world, t_cowa):
+    """The same step with the full-causal quadruple (0, Lk, 0, 0): every key
+    at distance 0 .. p is visible to every head.  The ratio of the two times
+    is the speedup over a full causal mask, bounded by the ratio of visible
+    work (full-causal pairs / CoWA pairs)."""
+    import torch.distributed as dist
+    quad = (0, wl.Lk, 0, 0)
+    o = torch.empty_like(q)
+    lse = torch.empty((wl.B, wl.Hq, wl.Lq), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    od = torch.empty_like(qd)
+    lsed = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device=dev)
+    ws_f = torch.empty(cowa.cowa_fwd_workspace_size(q, k, quad), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(cowa.cowa_bwd_workspace_size(q, k, quad), dtype=torch.uint8, device=dev)
+    ws_d = torch.empty(cowa.cowa_decode_workspace_size(qd, k, quad), dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        cowa.cowa_fwd(q, k, v, quad, out=o, lse=lse, workspace=ws_f)
+        if ev is not None:
+            ev[1].record(stream)
+        cowa.cowa_bwd(q, k, v, o, lse, do, quad, dq=dq, dk=dk, dv=dv, workspace=ws_b)
+        if ev is not None:
+            ev[2].record(stream)
+        cowa.cowa_decode(qd, k, v, seqlens, quad, out=od, lse=lsed, workspace=ws_d)
+        if ev is not None:
+            ev[3].record(stream)
+
+    steps = max(3, min(args.steps, 10))
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    if world > 1:
+        dist.barrier()
+    for i in range(steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    cowa.cowa_get_device_error(dev)
+    t = [sum(e[a].elapsed_time(e[a + 1]) for e in evs) / steps for a in range(3)]
+    t = max_over_ranks(t, world, dev)
+    full_pairs = visible_pairs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, quad)
+    cowa_pairs = visible_pairs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, wl.quad)
+    full_keys = decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, quad)
+    cowa_keys = decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, wl.quad)
+    return {"quad": list(quad), "steps": steps,
+            "fwd_ms": round(t[0], 4), "bwd_ms": round(t[1], 4), "decode_ms": round(t[2], 4),
+            "speedup_fwd": round(t[0] / t_cowa[0], 3), "speedup_bwd": round(t[1] / t_cowa[1], 3),
+            "speedup_decode": round(t[2] / t_cowa[2], 3),
+            "visible_work_ratio_fwd_bwd": round(full_pairs / cowa_pairs, 3),
+            "visible_work_ratio_decode": round(full_keys / cowa_keys, 3)}
 
 
 def run_decode_workload(args, cowa, dev, stream, flush, world, peaks, peak_src):
@@ -558,6 +617,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=512, help="query rows per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-workload", dest="decode_workload", action="store_false")
+    ap.add_argument("--no-full-mask", dest="full_mask", action="store_false",
+                    help="skip the full-causal-mask control run of the same step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -304,41 +304,19 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             }
             const float smax = fmaxf(max3(mx4[0], mx4[1], mx4[2]), mx4[3]);
             const float tmax = smax * p.scale_log2;  // scale > 0 keeps the order
-            // P_x and O_x are rewritten below: PV_x(t-1) must be complete
-            // (O_DONE(x) has completed t-1 or t phases: PV_x(t) waits for the
-            // P_FULL arrival below)
-            if (t > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(O_DONE(x), (t - 1) & 1, p.err, abort_flag));
-                if (!ok) break;
-                tc_fence_after();
-            }
             // lazy rescale: keep the old reference max unless it is exceeded by 2^8
             const bool grow = tmax > m_run + 8.f;
             const float alpha = grow ? fast_ex2(m_run - tmax) : 1.f;
             const bool fix_o = grow && m_run != -CUDART_INF_F;
-            if (__any_sync(0xffffffffu, fix_o)) {
-                const float f = fix_o ? alpha : 1.f;
-#pragma unroll
-                for (int c = 0; c < D / 16; ++c) {
-                    uint32_t o[16];
-                    const uint32_t ta = tOx + c * 16;
-                    tmem_ld16(ta, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                    tmem_st16(ta, o);
-                }
-                tmem_wait_st();
-            }
             if (grow) {
                 l *= alpha;
                 lb *= alpha;
                 m_run = tmax;
             }
             const float nms = m_run == -CUDART_INF_F ? 0.f : -m_run;
-            // P = 2^(s*scale - m) as bf16 into P_x, two keys per packed f32x2
-            // op; packed entry e (< BN/2) takes keys 2e and 2e+1 and is written
-            // over sr[e], already consumed
+            // P = 2^(s*scale - m) as bf16, two keys per packed f32x2 op; packed
+            // entry e (< BN/2) takes keys 2e and 2e+1 and is written over
+            // sr[e], already consumed
             const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(nms, nms);
             float2 la = make_float2(0.f, 0.f), lc = make_float2(0.f, 0.f);
             float2 ba = make_float2(0.f, 0.f), bc = make_float2(0.f, 0.f);
@@ -346,7 +324,15 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             for (int e = 0; e < BN / 2; ++e) {
                 const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
                                              sc2, nm2);
-                const float p0 = fast_ex2(xa.x), p1 = fast_ex2(xa.y);
+                float p0, p1;
+                if (e % 3 == 2) {  // one pair in three on the FMA pipe, the rest on the MUFU
+                    const float2 pp = exp2_poly2(xa);
+                    p0 = pp.x;
+                    p1 = pp.y;
+                } else {
+                    p0 = fast_ex2(xa.x);
+                    p1 = fast_ex2(xa.y);
+                }
                 const uint32_t pk = pack2(p0, p1);
                 // the two bf16 values as fp32 (low half: key 2e, high: key 2e+1)
                 const float2 pr = make_float2(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u));
@@ -359,10 +345,32 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                 }
                 sr[e] = pk;
             }
-#pragma unroll
-            for (int c = 0; c < NC; ++c) tmem_st16(tP + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c * 16]));
             l += (la.x + la.y) + (lc.x + lc.y);
             lb += (ba.x + ba.y) + (bc.x + bc.y);
+            // P_x and O_x are rewritten from here on: PV_x(t-1) must be complete
+            // (O_DONE(x) has completed t-1 or t phases: PV_x(t) waits for the
+            // P_FULL arrival below)
+            if (t > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(O_DONE(x), (t - 1) & 1, p.err, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+            }
+#pragma unroll
+            for (int c = 0; c < NC; ++c) tmem_st16(tP + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c * 16]));
+            if (__any_sync(0xffffffffu, fix_o)) {
+                // O holds tiles < t weighted against the old max: scale its row
+                const float f = fix_o ? alpha : 1.f;
+#pragma unroll
+                for (int c = 0; c < D / 16; ++c) {
+                    uint32_t o[16];
+                    const uint32_t ta = tOx + c * 16;
+                    tmem_ld16(ta, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                    tmem_st16(ta, o);
+                }
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(P_FULL(x));

@@ -281,6 +281,32 @@ __device__ __forceinline__ float max3(float a, float b, float c)
     return r;
 }
 
+// 2^x for a pair, on the FMA pipe instead of the MUFU: x = j + f with
+// j = rint(x) (the 1.5 * 2^23 shift puts j in the low mantissa bits) and f in
+// [-0.5, 0.5]; 2^f from a cubic fitted for minimum maximum relative error on
+// that interval (7.5e-5; exp2_fit.py), 2^j built as an exponent field.
+// x is clamped at -127, where the exponent field is 0, so -inf (a masked
+// key) and anything below -127 give exactly 0.
+constexpr float kExp2C0 = 9.999280572e-01f;
+constexpr float kExp2C1 = 6.932601929e-01f;
+constexpr float kExp2C2 = 2.426114976e-01f;
+constexpr float kExp2C3 = 5.517605320e-02f;
+__device__ __forceinline__ float2 exp2_poly2(float2 x)
+{
+    x.x = fmaxf(x.x, -127.f);
+    x.y = fmaxf(x.y, -127.f);
+    const float2 sh = make_float2(12582912.f, 12582912.f);
+    const float2 t = __fadd2_rn(x, sh);
+    const float2 j = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+    const float2 f = __fadd2_rn(x, make_float2(-j.x, -j.y));
+    float2 p = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+    p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
+    p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
+    const float2 sc = make_float2(__uint_as_float((__float_as_uint(t.x) << 23) + (127u << 23)),
+                                  __uint_as_float((__float_as_uint(t.y) << 23) + (127u << 23)));
+    return __fmul2_rn(p, sc);
+}
+
 __device__ __forceinline__ uint32_t pack2(float lo, float hi)
 {
     uint32_t r;
