@@ -21,16 +21,17 @@
 //              32-column chunks and takes the max (edge tiles only apply the
 //              element mask); pass 2 re-reads S, writes P = 2^(s*scale - m) as
 //              bf16 to P_x and sums P in fp32 for the LSE.  The normalisation
-//              of O uses the sum of the bf16-rounded P the PV product used
-//              (unpacked from the packed pairs and summed alongside), so O is
-//              divided by exactly the weights it accumulated.  The O row is
+//              of O uses the sum of the bf16 P the PV product used: each
+//              stage holds a block of ones after V, so the PV MMA, 16 columns
+//              wider than d, accumulates that sum next to O, and O is divided
+//              by exactly the weights it accumulated.  The O row is
 //              rescaled in tensor memory only when the max grows by more than
 //              2^8 (until then the stale max is a valid reference point).
 // Key tiles are 96 wide for d = 64 and 64 wide for d = 128: a softmax thread
 // reads its whole row of S_x with one tensor-memory round trip and keeps it
-// in registers.  Tensor-memory columns for d = 64: S_x at 128x, P_x at
-// 256 + 64x, O_x at 384 + 64x; for d = 128: S_x at 64x, P_x at 128 + 32x,
-// O_x at 256 + 128x.
+// in registers.  Tensor-memory columns (O_x is d + 16 wide: O, then the bf16
+// row sums) for d = 64: S_x at 96x, P_x at 192 + 64x, O_x at 320 + 96x; for
+// d = 128: S_x at 64x, P_x at 128 + 32x, O_x at 192 + 160x.
 // Softmax x rewrites P_x and rescales O_x for tile t only after O_DONE_x says
 // PV_x(t-1) is complete.
 // Every mbarrier wait is bounded; a wait that runs out records a timeout in
@@ -57,17 +58,22 @@ struct FwdCfg {
     static constexpr int BM = 128, BN = fwd5_bn(D);
     static constexpr int STAGES = 4;  // tiles t, t+1, t+2 are resident at once
     // tensor-memory column of S_x, P_x, O_x
-    static constexpr __host__ __device__ int t_s(int x) { return D == 128 ? 64 * x : 128 * x; }
-    static constexpr __host__ __device__ int t_p(int x) { return D == 128 ? 128 + 32 * x : 256 + 64 * x; }
-    static constexpr __host__ __device__ int t_o(int x) { return D == 128 ? 256 + 128 * x : 384 + 64 * x; }
+    static constexpr __host__ __device__ int t_s(int x) { return D == 128 ? 64 * x : 96 * x; }
+    static constexpr __host__ __device__ int t_p(int x) { return D == 128 ? 128 + 32 * x : 192 + 64 * x; }
+    static constexpr __host__ __device__ int t_o(int x) { return D == 128 ? 192 + 160 * x : 320 + 96 * x; }
+    static constexpr int OW = D + 16;                 // O columns, then the bf16 row sums
+    // exponentials on the FMA pipe: one pair in three for d = 64, where the
+    // softmax paces the kernel; none for d = 128, where it measured slower
+    static constexpr int POLY_EVERY = D == 64 ? 3 : 0;
     static constexpr int KB = D / 64;                 // 128-byte blocks along d
     static constexpr int Q_BYTES = BM * D * 2;        // one head's query tile
     static constexpr int KV_BYTES = BN * D * 2;       // one of K or V
-    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+    static constexpr int ONES_BYTES = BN * 128;       // bf16 1.0, one 128-byte row per key
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES + ONES_BYTES;
     static constexpr int NBAR = 12 + 2 * STAGES;
     static constexpr int SMEM = 1024 + 2 * Q_BYTES + STAGES * STAGE_BYTES + 8 * NBAR + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
-    static constexpr uint32_t IDESC_O = idesc_bf16(128, D, 0, 1);
+    static constexpr uint32_t IDESC_O = idesc_bf16(128, OW, 0, 1);
 };
 
 template <int D>
@@ -141,6 +147,13 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         tmem_alloc(smem_addr(tmem_slot), 512);
         tmem_relinquish();
     }
+    // the ones block of every stage (TMA never writes it); the PV MMA reads it
+    // as B columns d .. d+15, any swizzle of an all-ones row reads ones
+    for (int s = 0; s < ST; ++s) {
+        uint32_t *ones = reinterpret_cast<uint32_t *>(sm + 2 * C::Q_BYTES + s * C::STAGE_BYTES + 2 * C::KV_BYTES);
+        for (int k = tid; k < C::ONES_BYTES / 4; k += blockDim.x) ones[k] = 0x3F803F80u;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (warp == 8 && lane == 0) {
         prefetch_tmap(&a.tq);
         prefetch_tmap(&a.tk);
@@ -163,7 +176,7 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                 const int s = t % ST;
                 if (t >= ST && !mbar_wait(KV_EMPTY(s), ((t / ST) - 1) & 1, p.err, abort_flag)) break;
                 const int kt = tile_of(t);
-                mbar_expect_tx(KV_FULL(s), C::STAGE_BYTES);
+                mbar_expect_tx(KV_FULL(s), 2 * C::KV_BYTES);
                 const uint32_t sk = sStage + s * C::STAGE_BYTES, sv = sk + C::KV_BYTES;
                 for (int kb = 0; kb < KB; ++kb) {
                     tma_load_4d(sk + kb * BN * 128, &a.tk, KV_FULL(s), kb * 64, kt * BN, hl, b);
@@ -245,7 +258,7 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         const uint32_t tOx = tmem + C::t_o(x) + lane_off;
         const int prow = pa + r;
         const bool active = x < nslot;
-        float m_run = -CUDART_INF_F, l = 0.f, lb = 0.f;  // fp32 and bf16-rounded sums of P
+        float m_run = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         for (int t = 0; active && t < ntiles; ++t) {
             ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), t & 1, p.err, abort_flag));
@@ -310,7 +323,6 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             const bool fix_o = grow && m_run != -CUDART_INF_F;
             if (grow) {
                 l *= alpha;
-                lb *= alpha;
                 m_run = tmax;
             }
             const float nms = m_run == -CUDART_INF_F ? 0.f : -m_run;
@@ -319,13 +331,12 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             // sr[e], already consumed
             const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(nms, nms);
             float2 la = make_float2(0.f, 0.f), lc = make_float2(0.f, 0.f);
-            float2 ba = make_float2(0.f, 0.f), bc = make_float2(0.f, 0.f);
 #pragma unroll
             for (int e = 0; e < BN / 2; ++e) {
                 const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
                                              sc2, nm2);
                 float p0, p1;
-                if (e % 3 == 2) {  // one pair in three on the FMA pipe, the rest on the MUFU
+                if (C::POLY_EVERY && e % C::POLY_EVERY == C::POLY_EVERY - 1) {  // FMA pipe, the rest on the MUFU
                     const float2 pp = exp2_poly2(xa);
                     p0 = pp.x;
                     p1 = pp.y;
@@ -333,20 +344,13 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                     p0 = fast_ex2(xa.x);
                     p1 = fast_ex2(xa.y);
                 }
-                const uint32_t pk = pack2(p0, p1);
-                // the two bf16 values as fp32 (low half: key 2e, high: key 2e+1)
-                const float2 pr = make_float2(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u));
-                if (e & 1) {
+                if (e & 1)
                     lc = __fadd2_rn(lc, make_float2(p0, p1));
-                    bc = __fadd2_rn(bc, pr);
-                } else {
+                else
                     la = __fadd2_rn(la, make_float2(p0, p1));
-                    ba = __fadd2_rn(ba, pr);
-                }
-                sr[e] = pk;
+                sr[e] = pack2(p0, p1);
             }
             l += (la.x + la.y) + (lc.x + lc.y);
-            lb += (ba.x + ba.y) + (bc.x + bc.y);
             // P_x and O_x are rewritten from here on: PV_x(t-1) must be complete
             // (O_DONE(x) has completed t-1 or t phases: PV_x(t) waits for the
             // P_FULL arrival below)
@@ -361,7 +365,7 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                 // O holds tiles < t weighted against the old max: scale its row
                 const float f = fix_o ? alpha : 1.f;
 #pragma unroll
-                for (int c = 0; c < D / 16; ++c) {
+                for (int c = 0; c < C::OW / 16; ++c) {  // O and its bf16 row sums
                     uint32_t o[16];
                     const uint32_t ta = tOx + c * 16;
                     tmem_ld16(ta, o);
@@ -385,6 +389,13 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         // epilogue: O / (sum of the bf16 P) in bf16, LSE (natural log) from the fp32 sum
         if (active) {
             const bool have = ok && ntiles > 0;
+            float lb = 0.f;  // sum of the bf16 P that O accumulated
+            if (have) {
+                uint32_t lv[16];
+                tmem_ld16(tOx + D, lv);
+                tmem_wait_ld();
+                lb = __uint_as_float(lv[0]);
+            }
             const float inv = (l > 0.f && lb > 0.f) ? 1.f / lb : 0.f;
             const int hq = hq0 + x;
             __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + b * p.os[0] +
