@@ -298,45 +298,54 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tb = tmem + C::T_BUF + x * C::BUF + lane_off;
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-        const long long pmax = (long long)p.Lk - 1;
         // aligned positions p that see key jg: sink [jg, Lk-1], near
-        // [jg, jg+N-1], long [jg+c, jg+e-1]
-        const long long snk_hi = jg < w.S ? pmax : -1;
-        const long long nr_hi = w.N > 0 ? min((long long)jg + w.N - 1, pmax) : -1;
-        const long long lg_lo = (long long)jg + w.c, lg_hi = w.e > w.c ? min((long long)jg + w.e - 1, pmax) : -1;
+        // [jg, jg+N-1], long [jg+c, jg+e-1], as 32-bit bounds (an empty
+        // interval has hi < lo; every position is below 2^30)
+        const long long pmax = (long long)p.Lk - 1;
+        const int snk_hi = jg < w.S ? (int)pmax : -1;
+        const int nr_hi = w.N > 0 ? (int)min((long long)jg + w.N - 1, pmax) : -1;
+        const int lg_lo = (int)min((long long)jg + w.c, pmax + 1);
+        const int lg_hi = w.e > w.c ? (int)min((long long)jg + w.e - 1, pmax) : -1;
+        // this warpgroup's tasks u = x, x+2, ...: query head gi of the group
+        // and position t in the key tile's query-tile list, advanced without
+        // division
+        int gi = nq > 0 ? x / nq : 0, tq = nq > 0 ? x % nq : 0;
         bool ok = true;
         for (int k = 0;; ++k) {
             const int u = 2 * k + x;
             if (u >= ntask) break;
-            ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), k & 1, p.err, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            int hq, qt;
-            task(u, hq, qt);
+            // task set-up, independent of the scores: done while they land
+            const int qt = tq < len0 || nr == 1 ? lo0 + tq
+                           : (tq - len0 < len1 || nr == 2 ? lo1 + tq - len0 : lo2 + tq - len0 - len1);
+            tq += 2;
+            while (tq >= nq) {
+                tq -= nq;
+                ++gi;
+            }
             const int q0 = qt * BM;
             const int nrows = min(BM, p.Lq - q0);
             const int pa = q0 + delta_pos;
             const bool full = tile_full(pa, pa + nrows - 1, c0, BN, p.Lk, w);
+            uint32_t vis[BM / 32];
+#pragma unroll
+            for (int c = 0; c < BM / 32; ++c) {
+                // query columns of chunk c: p = pa + c*32 + bit, rows < nrows
+                const int pc = pa + c * 32, rmax = pa + nrows - 1;
+                auto span = [&](int lo, int hi) -> uint32_t {
+                    hi = min(hi, rmax);
+                    return hi < lo ? 0u : span_bits(lo - pc, hi - pc);
+                };
+                vis[c] = full ? 0xFFFFFFFFu : (span(jg, snk_hi) | span(jg, nr_hi) | span(lg_lo, lg_hi));
+            }
             const float2 *lsd = stage_lsd(u % ST);
+            ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), k & 1, p.err, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
 #pragma unroll
             for (int c = 0; c < BM / 32; ++c) {
                 uint32_t sr[32], dr[32];
                 tmem_ld32(tb + c * 32, sr);
                 tmem_ld32(tb + BM + c * 32, dr);
-                uint32_t vis = 0xFFFFFFFFu;
-                if (!full) {
-                    // query columns of this chunk: p = pa + c*32 + bit, rows < nrows
-                    const long long pc = (long long)pa + c * 32;
-                    const long long rmax = (long long)pa + nrows - 1;
-                    auto span = [&](long long lo, long long hi) -> uint32_t {
-                        hi = min(hi, rmax);
-                        if (hi < lo) return 0u;
-                        const long long a0 = lo - pc, a1 = hi - pc;
-                        if (a1 < 0 || a0 > 31) return 0u;
-                        return span_bits((int)max(a0, -1ll), (int)min(a1, 32ll));
-                    };
-                    vis = span(jg, snk_hi) | span(jg, nr_hi) | span(lg_lo, lg_hi);
-                }
                 tmem_wait_ld();
                 if (c == BM / 32 - 1) {
                     // all of S^T and dP^T read: S^T/dP^T of task u+2 may land
@@ -344,14 +353,17 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
                     __syncwarp();
                     if (lane == 0) mbar_arrive(S_FREE(x));
                 }
+                if (!full) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (!((vis[c] >> e) & 1u)) sr[e] = __float_as_uint(-CUDART_INF_F);
+                }
                 uint32_t pk[16], dk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const float4 ld = *reinterpret_cast<const float4 *>(lsd + c * 32 + 2 * e);  // (-lse2, -delta) x2
-                    float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
-                                           sc2, make_float2(ld.x, ld.z));
-                    if (!((vis >> (2 * e)) & 1u)) xa.x = -CUDART_INF_F;
-                    if (!((vis >> (2 * e + 1)) & 1u)) xa.y = -CUDART_INF_F;
+                    const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
+                                                 sc2, make_float2(ld.x, ld.z));
                     const float2 pr = make_float2(fast_ex2(xa.x), fast_ex2(xa.y));
                     const float2 t = __fadd2_rn(make_float2(__uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1])),
                                                 make_float2(ld.y, ld.w));
@@ -621,23 +633,26 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
                      nd2 = make_float2(nd, nd);
         bool ok = true;
         for (int t = 0; active && t < ntiles; ++t) {
+            // tile set-up, independent of the scores: done while they land
+            const int kt = tile_of(t);
+            const bool full = tile_full(pa, pb, kt * BN, BN, p.Lk, w);
+            uint32_t vis[BN / 32];
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) {
+                const int j0 = kt * BN + c * 32;
+                uint32_t m = span_bits(-j0, min(w.S - 1, prow) - j0);
+                if (w.N > 0) m |= span_bits(prow - w.N + 1 - j0, prow - j0);
+                if (w.e > w.c) m |= span_bits(prow - w.e + 1 - j0, prow - w.c - j0);
+                vis[c] = full ? 0xFFFFFFFFu : m;
+            }
             ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), t & 1, p.err, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const int kt = tile_of(t);
-            const bool full = tile_full(pa, pb, kt * BN, BN, p.Lk, w);
 #pragma unroll
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t sr[32], dr[32];
                 tmem_ld32(ts + C::T_S + c * 32, sr);
                 tmem_ld32(ts + C::T_DP + c * 32, dr);
-                uint32_t vis = 0xFFFFFFFFu;
-                if (!full) {
-                    const int j0 = kt * BN + c * 32;
-                    vis = span_bits(-j0, min(w.S - 1, prow) - j0);
-                    if (w.N > 0) vis |= span_bits(prow - w.N + 1 - j0, prow - j0);
-                    if (w.e > w.c) vis |= span_bits(prow - w.e + 1 - j0, prow - w.c - j0);
-                }
                 tmem_wait_ld();
                 if (c == BN / 32 - 1) {
                     // all of S and dP read: those of tile t+1 may land
@@ -645,13 +660,16 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
                     __syncwarp();
                     if (lane == 0) mbar_arrive(S_FREE(x));
                 }
+                if (!full) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (!((vis[c] >> e) & 1u)) sr[e] = __float_as_uint(-CUDART_INF_F);
+                }
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
-                                           sc2, nl2);
-                    if (!((vis >> (2 * e)) & 1u)) xa.x = -CUDART_INF_F;
-                    if (!((vis >> (2 * e + 1)) & 1u)) xa.y = -CUDART_INF_F;
+                    const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
+                                                 sc2, nl2);
                     const float2 pr = make_float2(fast_ex2(xa.x), fast_ex2(xa.y));
                     const float2 tt = __fadd2_rn(make_float2(__uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1])),
                                                  nd2);

@@ -261,20 +261,12 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         float m_run = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         for (int t = 0; active && t < ntiles; ++t) {
-            ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), t & 1, p.err, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t tS = tmem + C::t_s(x) + lane_off;
+            // tile set-up, independent of the scores: done while they land.
+            // Edge tiles build, per 32-key chunk, the bitmask of keys the row
+            // sees: the union of its sink, near and long key intervals.
             const int kt = tile_of(t);
             const bool full = tile_full(pa, pb, kt * BN, BN, p.Lk, w);
-            // One read of the row of S: all chunks are requested back to back and
-            // waited for once (each tensor-memory round trip costs hundreds of
-            // cycles).  Edge tiles build, per 32-key chunk, the bitmask of keys the
-            // row sees: the union of its sink, near and long key intervals.
             constexpr int NC = BN / 32;  // 32-column chunks of the row
-            uint32_t sr[BN];
-#pragma unroll
-            for (int c = 0; c < NC; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
             uint32_t vis[NC];
             if (!full) {
 #pragma unroll
@@ -295,6 +287,15 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                     vis[c] = m;
                 }
             }
+            ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), t & 1, p.err, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t tS = tmem + C::t_s(x) + lane_off;
+            // one read of the row of S: all chunks are requested back to back
+            // and waited for once
+            uint32_t sr[BN];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
             tmem_wait_ld();
             // the row is in registers: S_x(t+1) may overwrite S_x
             tc_fence_before();
