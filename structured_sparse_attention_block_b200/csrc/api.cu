@@ -224,6 +224,11 @@ void fill_common(P &p, const cowa_shape_t *s, cowa_quad_t q, float scale)
 size_t sched_bytes(long long heads, long long tiles) { return align256((size_t)(heads * tiles) * 8 * sizeof(int)); }
 
 
+// Splits of each (batch, KV head) key range.  The split kernel is memory
+// bound and its CTAs all do about the same work, so the time is set by the
+// number of full waves of resident CTAs: pick the smallest split count whose
+// waves-per-unit-of-work is within 3 % of the best, over 1 .. 64 splits and
+// at most one split per key tile.
 int decode_splits(const cowa_shape_t *s, cowa_quad_t q, int sms)
 {
     const long long pairs = s->B * s->Hkv;
@@ -231,11 +236,16 @@ int decode_splits(const cowa_shape_t *s, cowa_quad_t q, int sms)
     long long keys = (long long)q.S + q.N + q.W;
     if (keys > s->Lk) keys = s->Lk;
     const long long tiles = cdiv(keys, cowa::kDecBN) + 3;
-    long long sp = cdiv(4ll * sms, pairs);
-    if (sp > tiles) sp = tiles;
-    if (sp > 64) sp = 64;
-    if (sp < 1) sp = 1;
-    return (int)sp;
+    const long long resident = (long long)sms * cowa::decode_ctas_per_sm((int)s->d);
+    const long long max_sp = tiles < 64 ? tiles : 64;
+    double best = 1e30;
+    for (long long sp = 1; sp <= max_sp; ++sp) {
+        const double v = (double)cdiv(pairs * sp, resident) / (double)sp;
+        if (v < best) best = v;
+    }
+    for (long long sp = 1; sp <= max_sp; ++sp)
+        if ((double)cdiv(pairs * sp, resident) / (double)sp <= best * 1.03) return (int)sp;
+    return (int)max_sp;
 }
 
 }  // namespace

@@ -267,7 +267,7 @@ __global__ void decode_combine_kernel(const DecodeParams p)
 template <int D>
 static cudaError_t launch_decode_d(const DecodeParams &p, cudaStream_t st)
 {
-    constexpr int smem = (6 * kDecBN * D + 16 * D) * 2;
+    constexpr int smem = decode_smem_bytes(D);
     static_assert((128 + 64 * D) * 4 <= 6 * kDecBN * D * 2, "merge scratch must fit the K/V stages");
     static bool configured[64] = {};
     int dev = 0;

@@ -113,5 +113,9 @@ inline unsigned tile_grid_blocks(long long ntile, long long nslot, long long B)
 // decode.cu
 cudaError_t launch_decode(const DecodeParams &p, int D, cudaStream_t st);
 constexpr int kDecBN = 64;
+// shared memory of one split CTA: three K/V stages of kDecBN keys and the
+// 16-row query block; CTAs of it that fit on one SM (228 KB, 128 threads)
+constexpr int decode_smem_bytes(int D) { return (6 * kDecBN * D + 16 * D) * 2; }
+constexpr int decode_ctas_per_sm(int D) { return (228 * 1024) / (decode_smem_bytes(D) + 1024); }
 
 }  // namespace cowa
