@@ -208,6 +208,19 @@ def decode(q, k_cache, v_cache, seqlens, quad, scale=None, kv_head_offset=0,
     return o, lse
 
 
+def window_keys(p_lo, horizon, w, quad) -> np.ndarray:
+    """Sorted keys that some query position in [p_lo, p_lo + horizon) sees
+    through window index w: the key set a decode cache for those positions
+    must hold for that KV head (Digest, execution notes: decoding reads only
+    the windows, which is where its KV-cache saving comes from).  Brute force
+    over the dense mask, so it restates no interval arithmetic."""
+    if horizon <= 0:
+        return np.zeros(0, dtype=np.int64)
+    Lk = int(p_lo) + int(horizon)
+    m = mask(int(horizon), Lk, int(w), quad)  # row i is position p_lo + i
+    return np.nonzero(m.any(axis=0))[0].astype(np.int64)
+
+
 def bf16_bits(x) -> np.ndarray:
     """Round fp32/fp64 values to bf16 (round to nearest even); return bit patterns.
 
@@ -227,4 +240,4 @@ def bits_to_f64(bits) -> np.ndarray:
 
 
 __all__ = ["threads", "default_quad", "visible", "mask", "tile_counts", "fwd", "fwd_rows", "bwd",
-           "bwd_dq_rows", "bwd_dkv_cols", "decode", "bf16_bits", "bits_to_f64"]
+           "bwd_dq_rows", "bwd_dkv_cols", "decode", "window_keys", "bf16_bits", "bits_to_f64"]

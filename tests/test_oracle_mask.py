@@ -149,3 +149,32 @@ def test_tile_counts_match_the_dense_mask(oracle_mod):
                 for kt in range(counts.shape[1]):
                     blk = m[qt * BM:(qt + 1) * BM, kt * BN:(kt + 1) * BN]
                     assert counts[qt, kt] == blk.sum()
+
+
+def _window_keys_loop(p_lo, horizon, w, quad):
+    # the visibility rule written out once more as a plain double loop
+    S, N, G, W = quad
+    keys = set()
+    for p in range(p_lo, p_lo + horizon):
+        for j in range(0, p + 1):
+            d = p - j
+            if j < S or d < N or (N + G + w * W <= d < N + G + (w + 1) * W):
+                keys.add(j)
+    return sorted(keys)
+
+
+@pytest.mark.parametrize("p_lo,horizon,w,quad", [
+    (200, 1, 0, (4, 16, 0, 24)), (200, 9, 3, (4, 16, 0, 24)), (37, 5, 1, (0, 8, 2, 5)),
+    (500, 17, 7, (16, 32, 0, 60)), (3, 4, 0, (0, 0, 0, 0)), (90, 30, 2, (8, 8, 8, 8))])
+def test_window_keys_match_the_rule(oracle_mod, p_lo, horizon, w, quad):
+    got = oracle_mod.window_keys(p_lo, horizon, w, quad)
+    assert list(got) == _window_keys_loop(p_lo, horizon, w, quad)
+
+
+def test_window_keys_size_bound(oracle_mod):
+    # a head's windowed key set never exceeds sink + near + long + 2 * horizon
+    S, N, G, W = quad = (16, 64, 0, 96)
+    for w in range(4):
+        for p_lo, hz in ((1000, 1), (1000, 50), (300, 7)):
+            n = len(oracle_mod.window_keys(p_lo, hz, w, quad))
+            assert n <= S + N + W + 2 * hz
