@@ -99,6 +99,48 @@ COWA_API int cowa_abi_version(void);
 COWA_API uint64_t cowa_launch_count(void);
 
 /*
+ * Windowed decode cache (paper: decoding reads only each head's windows;
+ * Digest, execution notes, and the decode memory saving of the abstract).
+ * For a horizon of R query positions [origin[b], origin[b] + R) of sequence
+ * b, KV head h only ever sees the keys of sink [0, S), near
+ * [origin-N+1, origin+R-1] and its long slice [origin-e+1, origin+R-1-c]
+ * (c = N+G+hW, e = c+W).  The windowed cache stores exactly that key set per
+ * (sequence, KV head), merged and in ascending key order, in a contiguous
+ * bf16 tensor [B, rows, Hkv, d] with rows = cowa_wcache_rows(quad, R);
+ * unused rows are zero.  h is the GLOBAL head (local + kv_head_offset).
+ *
+ * cowa_wcache_rows: S + N + W + 2R, an upper bound of every head's key set
+ *   (0 for a negative field or R <= 0, or if the result reaches 2^30).
+ * cowa_wcache_build: from a full cache k_full/v_full [B, Lk, Hkv, d]
+ *   (shape->Lk, shape->k_stride, shape->v_stride; Lq, Hq, q/o strides are
+ *   ignored) and device int32 origin[B] (origin[b] < Lk: the position of the
+ *   query at build time, so keys 0..origin[b] exist), fills k_win/v_win.
+ *   Keys above origin[b] are left zero for cowa_wcache_append.
+ * cowa_wcache_append: writes the K/V of the token at device int32 pos[b]
+ *   (k_new/v_new [B, Hkv, d]; shape->k_stride[0] / [2] and v_stride[0] / [2]
+ *   are their batch and head strides) into the rows that hold it.
+ * cowa_decode_windowed: as cowa_decode over a windowed cache (shape->Lk =
+ *   rows, k/v strides those of the contiguous windowed tensors); the query
+ *   of sequence b sits at seqlens[b] - 1, which must lie in
+ *   [origin[b], origin[b] + R).  Workspace: cowa_decode_workspace_size.
+ * Errors: as cowa_decode; a device-side position outside the horizon (or an
+ * origin outside the source) sets COWA_ERR_DEVICE for cowa_get_device_error
+ * and the sequence reads or writes nothing.
+ */
+COWA_API int64_t cowa_wcache_rows(cowa_quad_t quad, int32_t horizon);
+COWA_API int cowa_wcache_build(const cowa_shape_t *shape, cowa_quad_t quad, int32_t horizon,
+                               const int32_t *origin, const void *k_full, const void *v_full,
+                               void *k_win, void *v_win, void *stream);
+COWA_API int cowa_wcache_append(const cowa_shape_t *shape, cowa_quad_t quad, int32_t horizon,
+                                const int32_t *origin, const int32_t *pos, const void *k_new,
+                                const void *v_new, void *k_win, void *v_win, void *stream);
+COWA_API int cowa_decode_windowed(const cowa_shape_t *shape, cowa_quad_t quad, float softmax_scale,
+                                  int32_t horizon, const int32_t *origin, const void *q,
+                                  const void *k_win, const void *v_win, const int32_t *seqlens,
+                                  void *o, float *lse, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/*
  * Kernel trace, a measurement aid with no counterpart in the paper.
  * cowa_trace_start(capacity, only) creates `capacity` CUDA event pairs on
  * the current device and turns tracing on (capacity 0 turns it off and frees

@@ -29,6 +29,7 @@ __all__ = ["CowaError", "cowa_fwd", "cowa_bwd", "cowa_decode", "cowa_default_qua
            "cowa_tile_classes", "cowa_fwd_workspace_size", "cowa_bwd_workspace_size",
            "cowa_decode_workspace_size", "cowa_get_device_error", "cowa_launch_count",
            "cowa_decode_noalloc", "cowa_trace_start", "cowa_trace_stop", "cowa_trace_entries",
+           "cowa_wcache_rows", "cowa_wcache_build", "cowa_wcache_append", "cowa_decode_windowed",
            "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -101,6 +102,14 @@ def lib():
         L.cowa_tile_classes.argtypes = [i64, i64, i64, Quad, i32, i32, ctypes.c_int, vp, vp, sz, vp]
         L.cowa_get_device_error.restype = ctypes.c_int
         L.cowa_get_device_error.argtypes = [vp]
+        L.cowa_wcache_rows.restype = i64
+        L.cowa_wcache_rows.argtypes = [Quad, i32]
+        L.cowa_wcache_build.restype = ctypes.c_int
+        L.cowa_wcache_build.argtypes = [SP, Quad, i32, vp, vp, vp, vp, vp, vp]
+        L.cowa_wcache_append.restype = ctypes.c_int
+        L.cowa_wcache_append.argtypes = [SP, Quad, i32, vp, vp, vp, vp, vp, vp, vp]
+        L.cowa_decode_windowed.restype = ctypes.c_int
+        L.cowa_decode_windowed.argtypes = [SP, Quad, ctypes.c_float, i32] + [vp] * 7 + [vp, sz, vp]
         L.cowa_trace_start.restype = ctypes.c_int
         L.cowa_trace_start.argtypes = [i64, ctypes.c_char_p]
         L.cowa_trace_stop.restype = ctypes.c_int
@@ -272,6 +281,86 @@ def cowa_decode(q, k_cache, v_cache, seqlens, quad, softmax_scale=None, kv_head_
     _check(L.cowa_decode(ctypes.byref(shape), qd, scale, _ptr(q4), _ptr(k_cache), _ptr(v_cache),
                          _ptr(seqlens), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                          _stream(q4.device)))
+    return out, lse
+
+
+def _int32_cuda(t, name):
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError("%s must be a contiguous int32 CUDA tensor" % name)
+
+
+def cowa_wcache_rows(quad, horizon) -> int:
+    """Rows of a windowed decode cache serving ``horizon`` query positions."""
+    return int(lib().cowa_wcache_rows(_quad(quad), int(horizon)))
+
+
+def cowa_wcache_build(k_cache, v_cache, origin, quad, horizon, kv_head_offset=0):
+    """Windowed decode cache ``(k_win, v_win)`` [B, rows, Hkv, d] from a full
+    cache [B, L, Hkv, d] for query positions [origin[b], origin[b] + horizon)
+    of each sequence (origin: int32 CUDA [B]; keys 0..origin[b] must be in
+    the full cache)."""
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _bf16_cuda(t, n)
+    _int32_cuda(origin, "origin")
+    B, Lk, Hkv, d = k_cache.shape
+    rows = cowa_wcache_rows(quad, horizon)
+    if rows <= 0:
+        raise ValueError("bad quadruple or horizon")
+    kw = torch.empty((B, rows, Hkv, d), dtype=torch.bfloat16, device=k_cache.device)
+    vw = torch.empty_like(kw)
+    shape = Shape(B, 1, Lk, Hkv, Hkv, d, _strides(k_cache), _strides(k_cache), _strides(v_cache),
+                  _strides(k_cache), int(kv_head_offset))
+    _check(lib().cowa_wcache_build(ctypes.byref(shape), _quad(quad), int(horizon), _ptr(origin),
+                                   _ptr(k_cache), _ptr(v_cache), _ptr(kw), _ptr(vw), _stream(k_cache.device)))
+    return kw, vw
+
+
+def cowa_wcache_append(k_win, v_win, k_new, v_new, pos, origin, quad, horizon, kv_head_offset=0):
+    """Write the K/V rows k_new/v_new [B, Hkv, d] of the tokens at positions
+    pos (int32 CUDA [B]) into the windowed cache (in place)."""
+    for t, n in ((k_win, "k_win"), (v_win, "v_win")):
+        _bf16_cuda(t, n)
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 3 \
+                or t.stride(2) != 1:
+            raise TypeError("%s must be a bf16 CUDA tensor [B, Hkv, d] with a contiguous last dimension" % n)
+    _int32_cuda(pos, "pos")
+    _int32_cuda(origin, "origin")
+    B, rows, Hkv, d = k_win.shape
+    ks = (ctypes.c_int64 * 3)(k_new.stride(0), 0, k_new.stride(1))
+    vs = (ctypes.c_int64 * 3)(v_new.stride(0), 0, v_new.stride(1))
+    shape = Shape(B, 1, rows, Hkv, Hkv, d, ks, ks, vs, ks, int(kv_head_offset))
+    _check(lib().cowa_wcache_append(ctypes.byref(shape), _quad(quad), int(horizon), _ptr(origin), _ptr(pos),
+                                    _ptr(k_new), _ptr(v_new), _ptr(k_win), _ptr(v_win), _stream(k_win.device)))
+
+
+def cowa_decode_windowed(q, k_win, v_win, seqlens, origin, quad, horizon, softmax_scale=None,
+                         kv_head_offset=0, out=None, lse=None, workspace=None):
+    """CoWA decode over a windowed cache; the query of sequence b sits at
+    seqlens[b] - 1, inside [origin[b], origin[b] + horizon).  Returns
+    ``(o [B, 1, Hq, d], lse [B, Hq])``."""
+    q4 = q if q.dim() == 4 else q.unsqueeze(1)
+    for t, n in ((q4, "q"), (k_win, "k_win"), (v_win, "v_win")):
+        _bf16_cuda(t, n)
+    _int32_cuda(seqlens, "seqlens")
+    _int32_cuda(origin, "origin")
+    B, _, Hq, d = q4.shape
+    if out is None:
+        out = torch.empty((B, 1, Hq, d), dtype=torch.bfloat16, device=q4.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q4.device)
+    _bf16_cuda(out, "out")
+    shape = _shape(q4, k_win, v_win, out, kv_head_offset)
+    qd = _quad(quad)
+    L = lib()
+    need = L.cowa_decode_workspace_size(ctypes.byref(shape), qd)
+    if need == 0:
+        _raise_size_error(L)
+    ws = _workspace(need, q4.device, workspace)
+    scale = 0.0 if softmax_scale is None else float(softmax_scale)
+    _check(L.cowa_decode_windowed(ctypes.byref(shape), qd, scale, int(horizon), _ptr(origin), _ptr(q4),
+                                  _ptr(k_win), _ptr(v_win), _ptr(seqlens), _ptr(out), _ptr(lse), _ptr(ws),
+                                  ws.numel(), _stream(q4.device)))
     return out, lse
 
 

@@ -483,9 +483,122 @@ int cowa_bwd(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const
     return COWA_OK;
 }
 
+static int decode_common(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const void *q,
+                         const void *k_cache, const void *v_cache, const int32_t *seqlens, void *o, float *lse,
+                         void *ws, size_t ws_bytes, void *stream, const int32_t *origin, int32_t horizon);
+
 int cowa_decode(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const void *q, const void *k_cache,
                 const void *v_cache, const int32_t *seqlens, void *o, float *lse, void *ws, size_t ws_bytes,
                 void *stream)
+{
+    return decode_common(s, quad, softmax_scale, q, k_cache, v_cache, seqlens, o, lse, ws, ws_bytes, stream,
+                         nullptr, 0);
+}
+
+int64_t cowa_wcache_rows(cowa_quad_t quad, int32_t horizon)
+{
+    if (quad.S < 0 || quad.N < 0 || quad.G < 0 || quad.W < 0 || horizon <= 0) return 0;
+    const long long rows = (long long)quad.S + quad.N + quad.W + 2ll * horizon;
+    return rows >= kMaxLen ? 0 : rows;
+}
+
+int cowa_decode_windowed(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, int32_t horizon,
+                         const int32_t *origin, const void *q, const void *k_win, const void *v_win,
+                         const int32_t *seqlens, void *o, float *lse, void *ws, size_t ws_bytes, void *stream)
+{
+    const int64_t rows = cowa_wcache_rows(quad, horizon);
+    if (rows == 0) return fail(COWA_ERR_INVALID_ARG, "bad quadruple or horizon %d", horizon);
+    if (s && s->Lk != rows)
+        return fail(COWA_ERR_INVALID_ARG, "windowed cache has %lld rows, expected %lld", (long long)s->Lk,
+                    (long long)rows);
+    if (s && s->B * s->Hq > 0 && !origin) return fail(COWA_ERR_INVALID_ARG, "origin is NULL");
+    return decode_common(s, quad, softmax_scale, q, k_win, v_win, seqlens, o, lse, ws, ws_bytes, stream, origin,
+                         horizon);
+}
+
+static int wcache_params(const cowa_shape_t *s, cowa_quad_t quad, int32_t horizon, const int32_t *origin,
+                         cowa::WCacheParams &p)
+{
+    if (!s) return fail(COWA_ERR_INVALID_ARG, "shape is NULL");
+    int r = check_quad(quad);
+    if (r) return r;
+    const int64_t rows = cowa_wcache_rows(quad, horizon);
+    if (rows == 0) return fail(COWA_ERR_INVALID_ARG, "bad horizon %d", horizon);
+    if (s->B < 0 || s->Hkv < 0 || s->Lk < 0 || s->kv_head_offset < 0 || s->B > 65535 || s->Hkv > 65535 ||
+        s->Lk >= kMaxLen)
+        return fail(COWA_ERR_INVALID_ARG, "bad sizes in shape");
+    if (s->d != 64 && s->d != 128)
+        return fail(COWA_ERR_UNSUPPORTED, "head dim %lld (supported: 64, 128)", (long long)s->d);
+    if ((r = check_strides(s->k_stride, "k")) || (r = check_strides(s->v_stride, "v"))) return r;
+    if (s->B * s->Hkv > 0 && !origin) return fail(COWA_ERR_INVALID_ARG, "origin is NULL");
+    p = cowa::WCacheParams{};
+    for (int a = 0; a < 3; ++a) {
+        p.ks[a] = s->k_stride[a];
+        p.vs[a] = s->v_stride[a];
+    }
+    p.origin = origin;
+    p.B = (int)s->B;
+    p.Hkv = (int)s->Hkv;
+    p.rows = (int)rows;
+    p.horizon = horizon;
+    p.Lsrc = (int)s->Lk;
+    p.S = quad.S;
+    p.N = quad.N;
+    p.G = quad.G;
+    p.W = quad.W;
+    p.kv_head_offset = (int)s->kv_head_offset;
+    p.err = device_error_word();
+    return COWA_OK;
+}
+
+int cowa_wcache_build(const cowa_shape_t *s, cowa_quad_t quad, int32_t horizon, const int32_t *origin,
+                      const void *k_full, const void *v_full, void *k_win, void *v_win, void *stream)
+{
+    cowa::WCacheParams p;
+    int r = wcache_params(s, quad, horizon, origin, p);
+    if (r) return r;
+    const bool work = s->B * s->Hkv > 0;
+    if ((r = check_ptr(k_full, work && s->Lk > 0, "k_full")) || (r = check_ptr(v_full, work && s->Lk > 0, "v_full")) ||
+        (r = check_ptr(k_win, work, "k_win")) || (r = check_ptr(v_win, work, "v_win")))
+        return r;
+    if (!work) return COWA_OK;
+    if ((r = check_device(nullptr))) return r;
+    p.err = device_error_word();
+    p.ksrc = k_full;
+    p.vsrc = v_full;
+    p.kw = k_win;
+    p.vw = v_win;
+    cudaError_t e = cowa::launch_wcache_build(p, (int)s->d, (cudaStream_t)stream);
+    return e == cudaSuccess ? COWA_OK : cuda_fail(e, "windowed cache build launch");
+}
+
+int cowa_wcache_append(const cowa_shape_t *s, cowa_quad_t quad, int32_t horizon, const int32_t *origin,
+                       const int32_t *pos, const void *k_new, const void *v_new, void *k_win, void *v_win,
+                       void *stream)
+{
+    cowa::WCacheParams p;
+    int r = wcache_params(s, quad, horizon, origin, p);
+    if (r) return r;
+    const bool work = s->B * s->Hkv > 0;
+    if ((r = check_ptr(k_new, work, "k_new")) || (r = check_ptr(v_new, work, "v_new")) ||
+        (r = check_ptr(k_win, work, "k_win")) || (r = check_ptr(v_win, work, "v_win")))
+        return r;
+    if (work && !pos) return fail(COWA_ERR_INVALID_ARG, "pos is NULL");
+    if (!work) return COWA_OK;
+    if ((r = check_device(nullptr))) return r;
+    p.err = device_error_word();
+    p.ksrc = k_new;
+    p.vsrc = v_new;
+    p.kw = k_win;
+    p.vw = v_win;
+    p.pos = pos;
+    cudaError_t e = cowa::launch_wcache_append(p, (int)s->d, (cudaStream_t)stream);
+    return e == cudaSuccess ? COWA_OK : cuda_fail(e, "windowed cache append launch");
+}
+
+static int decode_common(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const void *q,
+                         const void *k_cache, const void *v_cache, const int32_t *seqlens, void *o, float *lse,
+                         void *ws, size_t ws_bytes, void *stream, const int32_t *origin, int32_t horizon)
 {
     int r = check_shape(s, quad, true);
     if (r) return r;
@@ -511,6 +624,8 @@ int cowa_decode(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, co
     const size_t rows_p = (size_t)(s->B * s->Hq * p.splits);
     p.part_o = (float *)ws;
     p.part_lse = (float *)((char *)ws + align256(rows_p * s->d * sizeof(float)));
+    p.origin = origin;
+    p.horizon = horizon;
     cudaError_t e = cowa::launch_decode(p, (int)s->d, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     return COWA_OK;

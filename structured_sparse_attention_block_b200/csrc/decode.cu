@@ -25,9 +25,64 @@ __device__ __forceinline__ float ex2d(float x)
     return y;
 }
 
+// ------------------------------------------------------- windowed cache --
+// Keys a decode cache serving query positions [o, o + R) of one KV head must
+// hold: sink [0, S), near [o-N+1, o+R-1] and long [o-e+1, o+R-1-c], clipped
+// at 0, merged and stored back to back in ascending key order.  Every key
+// interval a query in that range sees lies inside one stored interval (the
+// stored intervals are separated by keys none of the queries sees).
+struct WindowStore {
+    int n;
+    int lo[3], len[3], off[3];
+};
+
+__device__ inline WindowStore window_store(int o, int R, const Win &w)
+{
+    Ranges r;
+    r.n = 0;
+    const long long top = (long long)o + R - 1;  // last query position served
+    if (R > 0 && top >= 0) {
+        if (w.S > 0) {
+            r.lo[r.n] = 0;
+            r.hi[r.n] = (int)min((long long)w.S, top + 1);
+            ++r.n;
+        }
+        if (w.N > 0) {
+            r.lo[r.n] = (int)max(0ll, (long long)o - w.N + 1);
+            r.hi[r.n] = (int)(top + 1);
+            ++r.n;
+        }
+        if (w.e > w.c && top - w.c >= 0) {
+            r.lo[r.n] = (int)max(0ll, (long long)o - w.e + 1);
+            r.hi[r.n] = (int)(top - w.c + 1);
+            ++r.n;
+        }
+        merge_ranges(r);
+    }
+    WindowStore ws;
+    ws.n = r.n;
+    int off = 0;
+    for (int a = 0; a < 3; ++a) {
+        ws.lo[a] = a < r.n ? r.lo[a] : 0;
+        ws.len[a] = a < r.n ? r.hi[a] - r.lo[a] : 0;
+        ws.off[a] = off;
+        off += ws.len[a];
+    }
+    return ws;
+}
+
+// stored row of the keys [j, j + n), or -1 unless one stored interval holds them all
+__device__ inline int window_row(const WindowStore &ws, int j, int n)
+{
+    for (int a = 0; a < ws.n; ++a)
+        if (j >= ws.lo[a] && j + n <= ws.lo[a] + ws.len[a]) return ws.off[a] + (j - ws.lo[a]);
+    return -1;
+}
+
 struct KeySpans {
     int n;
     int lo[3], len[3];
+    int row[3];  // cache row of lo[a]: lo[a] itself, or its row in a windowed cache
     int tiles[3];
     int total_tiles;
 };
@@ -51,6 +106,7 @@ __device__ inline KeySpans decode_spans(int p, const Win &w)
         ks.len[a] = a < r.n ? r.hi[a] - r.lo[a] : 0;
         ks.tiles[a] = (ks.len[a] + kDecBN - 1) / kDecBN;
         ks.total_tiles += ks.tiles[a];
+        ks.row[a] = ks.lo[a];
     }
     return ks;
 }
@@ -70,13 +126,31 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
     const int split = blockIdx.x, hl = blockIdx.y, b = blockIdx.z;
     const int g = p.g;
     int seq = p.seqlens[b];
-    if (seq < 0 || seq > p.Lcap) {  // never read outside the cache
+    const int org = p.origin ? p.origin[b] : 0;
+    // never read outside the cache: a full cache holds keys [0, Lcap); a
+    // windowed one serves query positions [origin, origin + horizon)
+    const bool bad = p.origin ? (org < 0 || seq - 1 < org || seq - 1 >= org + p.horizon)
+                              : (seq < 0 || seq > p.Lcap);
+    if (bad) {
         if (tid == 0 && split == 0) atomicExch(p.err, 7);
         seq = 0;
     }
     const int pq = seq - 1;
     const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
-    const KeySpans ks = decode_spans(pq, w);
+    KeySpans ks = decode_spans(pq, w);
+    if (p.origin && !bad) {
+        const WindowStore wst = window_store(org, p.horizon, w);
+        bool held = true;
+        for (int a = 0; a < 3; ++a) {
+            if (ks.len[a] == 0) continue;
+            ks.row[a] = window_row(wst, ks.lo[a], ks.len[a]);
+            held &= ks.row[a] >= 0 && ks.row[a] + ks.len[a] <= p.Lcap;
+        }
+        if (!held) {  // cannot happen for positions in the horizon; read nothing
+            if (tid == 0 && split == 0) atomicExch(p.err, 7);
+            ks = decode_spans(-1, w);
+        }
+    }
     const int t_begin = (int)((long long)ks.total_tiles * split / p.splits);
     const int t_end = (int)((long long)ks.total_tiles * (split + 1) / p.splits);
     const int ntiles = t_end - t_begin;
@@ -85,8 +159,8 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
     auto tile_at = [&](int t, int &k0, int &nk) {
         int a = 0;
         while (a < 2 && t >= ks.tiles[a]) { t -= ks.tiles[a]; ++a; }
-        k0 = ks.lo[a] + t * BN;
-        nk = min(BN, ks.lo[a] + ks.len[a] - k0);
+        k0 = ks.row[a] + t * BN;  // cache row of the tile's first key
+        nk = min(BN, ks.len[a] - t * BN);
     };
 
     const __nv_bfloat16 *kg = reinterpret_cast<const __nv_bfloat16 *>(p.kc) + b * p.ks[0] + hl * p.ks[2];
@@ -262,6 +336,97 @@ __global__ void decode_combine_kernel(const DecodeParams p)
     }
     if (threadIdx.x == 0)
         p.lse[row] = lsum > 0.f ? (m + __log2f(lsum)) * 0.69314718055994531f : -CUDART_INF_F;
+}
+
+// One thread per 16-byte piece of a row: row i of the windowed cache of
+// (b, h) takes key j of the source when the cache holds j and j <= origin
+// (a key the source has); other rows are zeroed (later appends fill them).
+template <int D>
+__global__ void __launch_bounds__(128) wcache_build_kernel(const WCacheParams p)
+{
+    constexpr int PIECES = D * 2 / 16, ROWS = 128 / PIECES;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int i = blockIdx.x * ROWS + threadIdx.x / PIECES, c = threadIdx.x % PIECES;
+    if (i >= p.rows) return;
+    const int o = p.origin[b];
+    int j = -1;
+    if (o >= 0 && o < p.Lsrc) {
+        const WindowStore ws = window_store(o, p.horizon, make_win(p.S, p.N, p.G, p.W, (long long)h + p.kv_head_offset));
+        for (int a = 0; a < ws.n; ++a)
+            if (i >= ws.off[a] && i < ws.off[a] + ws.len[a]) j = ws.lo[a] + (i - ws.off[a]);
+        if (j > o) j = -1;  // a future key: appended later
+    } else if (i == 0 && c == 0 && h == 0) {
+        atomicExch(p.err, 7);
+    }
+    const long long dst = (((long long)b * p.rows + i) * p.Hkv + h) * D + c * 8;
+    uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
+    if (j >= 0) {
+        kv = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(p.ksrc) + b * p.ks[0] +
+                                              (long long)j * p.ks[1] + h * p.ks[2] + c * 8);
+        vv = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(p.vsrc) + b * p.vs[0] +
+                                              (long long)j * p.vs[1] + h * p.vs[2] + c * 8);
+    }
+    *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.kw) + dst) = kv;
+    *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.vw) + dst) = vv;
+}
+
+// The K/V row of the token at pos[b] (source [B, Hkv, d], strides b and h)
+// goes to its row of every KV head's windowed cache that holds it; a
+// position outside [origin, origin + horizon) is refused on the device.
+template <int D>
+__global__ void __launch_bounds__(128) wcache_append_kernel(const WCacheParams p)
+{
+    constexpr int PIECES = D * 2 / 16, HEADS = 128 / PIECES;
+    const int b = blockIdx.y;
+    const int h = blockIdx.x * HEADS + threadIdx.x / PIECES, c = threadIdx.x % PIECES;
+    if (h >= p.Hkv) return;
+    const int o = p.origin[b], j = p.pos[b];
+    if (o < 0 || j < o || j >= o + p.horizon) {
+        if (h == 0 && c == 0) atomicExch(p.err, 7);
+        return;
+    }
+    const WindowStore ws = window_store(o, p.horizon, make_win(p.S, p.N, p.G, p.W, (long long)h + p.kv_head_offset));
+    const int i = window_row(ws, j, 1);
+    if (i < 0 || i >= p.rows) return;  // no query of the horizon sees key j through this head
+    const long long dst = (((long long)b * p.rows + i) * p.Hkv + h) * D + c * 8;
+    *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.kw) + dst) = *reinterpret_cast<const uint4 *>(
+        reinterpret_cast<const __nv_bfloat16 *>(p.ksrc) + b * p.ks[0] + h * p.ks[2] + c * 8);
+    *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.vw) + dst) = *reinterpret_cast<const uint4 *>(
+        reinterpret_cast<const __nv_bfloat16 *>(p.vsrc) + b * p.vs[0] + h * p.vs[2] + c * 8);
+}
+
+template <int D>
+static cudaError_t launch_wcache_build_d(const WCacheParams &p, cudaStream_t st)
+{
+    constexpr int ROWS = 128 / (D * 2 / 16);
+    dim3 grid((p.rows + ROWS - 1) / ROWS, p.Hkv, p.B);
+    launch_begin("wcache_build", st);
+    wcache_build_kernel<D><<<grid, 128, 0, st>>>(p);
+    launch_end(st);
+    return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_wcache_append_d(const WCacheParams &p, cudaStream_t st)
+{
+    constexpr int HEADS = 128 / (D * 2 / 16);
+    dim3 grid((p.Hkv + HEADS - 1) / HEADS, p.B);
+    launch_begin("wcache_append", st);
+    wcache_append_kernel<D><<<grid, 128, 0, st>>>(p);
+    launch_end(st);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_wcache_build(const WCacheParams &p, int D, cudaStream_t st)
+{
+    if (p.B == 0 || p.Hkv == 0 || p.rows == 0) return cudaSuccess;
+    return D == 128 ? launch_wcache_build_d<128>(p, st) : launch_wcache_build_d<64>(p, st);
+}
+
+cudaError_t launch_wcache_append(const WCacheParams &p, int D, cudaStream_t st)
+{
+    if (p.B == 0 || p.Hkv == 0 || p.rows == 0) return cudaSuccess;
+    return D == 128 ? launch_wcache_append_d<128>(p, st) : launch_wcache_append_d<64>(p, st);
 }
 
 template <int D>

@@ -39,7 +39,25 @@ struct DecodeParams {
     int kv_head_offset;
     float scale, scale_log2;
     int *err;
+    // windowed cache: per-sequence origin positions (nullptr for a full cache)
+    // and the horizon of query positions [origin, origin + horizon) it serves
+    const int *origin;
+    int horizon;
 };
+
+// Building and appending to a windowed decode cache (decode.cu).  The cache
+// is [B, rows, Hkv, d] contiguous bf16; the source is strided (b, l, h).
+struct WCacheParams {
+    const void *ksrc, *vsrc;
+    void *kw, *vw;
+    const int *origin, *pos;
+    long long ks[3], vs[3];
+    int B, Hkv, rows, horizon, Lsrc;
+    int S, N, G, W, kv_head_offset;
+    int *err;
+};
+cudaError_t launch_wcache_build(const WCacheParams &p, int D, cudaStream_t st);
+cudaError_t launch_wcache_append(const WCacheParams &p, int D, cudaStream_t st);
 
 // api.cu: every kernel launch of the library is bracketed by these two calls:
 // they count launches and, while tracing is on, record a CUDA event pair on

@@ -110,3 +110,23 @@ def test_trace_argument_errors(cowa):
     assert lib.cowa_trace_size() == 0
     name, ms = ctypes.c_char_p(), ctypes.c_float()
     assert lib.cowa_trace_entry(0, ctypes.byref(name), ctypes.byref(ms)) == 1
+
+
+def test_wcache_rows_and_argument_errors(cowa):
+    lib = cowa.lib()
+    assert cowa.cowa_wcache_rows((128, 8192, 0, 15360), 16) == 128 + 8192 + 15360 + 32
+    assert cowa.cowa_wcache_rows((1, 2, 0, 3), 0) == 0
+    assert cowa.cowa_wcache_rows((-1, 2, 0, 3), 4) == 0
+    p = ctypes.c_void_p(16)
+    shp = make_shape(cowa, Lq=1, Lk=1 + 2 + 3 + 8)
+    # a windowed decode whose cache rows do not match the quadruple and horizon
+    st = lib.cowa_decode_windowed(ctypes.byref(make_shape(cowa, Lq=1, Lk=99)), cowa.Quad(1, 2, 0, 3), 0.0, 4,
+                                  p, p, p, p, p, p, p, p, 1 << 20, None)
+    assert st == 1 and "rows" in lib.cowa_last_error_detail().decode()
+    st = lib.cowa_decode_windowed(ctypes.byref(shp), cowa.Quad(1, 2, 0, 3), 0.0, 4, None, p, p, p, p, p, p, p,
+                                  1 << 20, None)
+    assert st == 1  # origin is NULL
+    assert lib.cowa_wcache_build(ctypes.byref(make_shape(cowa, d=96)), cowa.Quad(1, 2, 0, 3), 4, p, p, p, p, p,
+                                 None) == 2
+    assert lib.cowa_wcache_append(ctypes.byref(make_shape(cowa)), cowa.Quad(1, 2, 0, 3), 4, p, None, p, p, p, p,
+                                  None) == 1  # pos is NULL

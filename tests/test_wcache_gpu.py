@@ -49,7 +49,7 @@ def test_build_stores_the_oracle_key_set(oracle_mod, B, Lcap, Hq, Hkv, d, quad, 
 @pytest.mark.parametrize("d", [64, 128])
 def test_decode_over_horizon_matches_full_cache(oracle_mod, d):
     import structured_sparse_attention_block_b200 as cowa
-    from structured_sparse_attention_block_b200.inputs import decode_inputs
+    from structured_sparse_attention_block_b200.inputs import bf16_bits, decode_inputs
     B, Lcap, Hq, Hkv, horizon = 3, 900, 8, 4, 6
     quad = (16, 48, 0, 160)
     origins = [880, 511, 200]
@@ -68,14 +68,15 @@ def test_decode_over_horizon_matches_full_cache(oracle_mod, d):
         o_w, lse_w = cowa.cowa_decode_windowed(qs, kw, vw, seq, org, quad, horizon)
         torch.cuda.synchronize()
         cowa.cowa_get_device_error()
-        o_ref, lse_ref = oracle_mod.decode(qs[:, 0].cpu(), kc.cpu(), vc.cpu(), seq.cpu().numpy(), quad)
+        o_ref, lse_ref = oracle_mod.decode(bf16_bits(qs[:, 0]), bf16_bits(kc), bf16_bits(vc), seq.cpu().numpy(),
+                                           quad)
         assert_o(o_w[:, 0], o_ref, what="windowed decode O, step %d" % step)
         assert np.abs(lse_w.cpu().numpy() - lse_ref).max() <= LSE_ABS
 
 
 def test_query_outside_the_horizon_is_flagged():
     import structured_sparse_attention_block_b200 as cowa
-    B, Lcap, Hq, Hkv, d, horizon = 2, 400, 4, 2, 64
+    B, Lcap, Hq, Hkv, d, horizon = 2, 400, 4, 2, 64, 6
     quad = (8, 32, 0, 100)
     origins = [300, 100]
     q, kc, vc, org, kw, vw = _full_and_windowed(cowa, B, Lcap, Hq, Hkv, d, quad, origins, horizon, seed=3)
