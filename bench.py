@@ -405,6 +405,8 @@ def run_cowa(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": int(launches),
     }
+    if args.packed:
+        result["packed_workload"] = run_packed_workload(args, cowa, wl, dev, stream, flush, world, peaks)
     if args.full_mask:
         result["full_mask_control"] = run_full_mask(args, cowa, wl, q, k, v, do, qd, seqlens, dev, stream,
                                                     flush, world, (t_fwd, t_bwd, t_dec))
@@ -509,6 +511,62 @@ def run_full_mask(args, cowa, wl, q, k, v, do, qd, seqlens, dev, stream, flush, 
             "speedup_decode": round(t[2] / t_cowa[2], 3),
             "visible_work_ratio_fwd_bwd": round(full_pairs / cowa_pairs, 3),
             "visible_work_ratio_decode": round(full_keys / cowa_keys, 3)}
+
+
+def packed_lengths(total, lo, hi, seed):
+    """Seeded ragged sequence lengths, log-uniform in [lo, hi], summing to total."""
+    rng = np.random.default_rng(seed)
+    out = []
+    while sum(out) < total:
+        n = int(round(float(np.exp(rng.uniform(np.log(lo), np.log(hi))))))
+        out.append(min(n, total - sum(out)))
+    return out
+
+
+def run_packed_workload(args, cowa, wl, dev, stream, flush, world, peaks):
+    """A packed (variable-length) batch with the workload's heads and window
+    quadruple: as many tokens as the workload's batch, in sequences of
+    log-uniform lengths between 1/16 and 1x the workload's length."""
+    import torch.distributed as dist
+    from structured_sparse_attention_block_b200.inputs import training_inputs
+    lens = packed_lengths(wl.B * wl.Lq, max(1, wl.Lq // 16), wl.Lq, seed=17)
+    T = sum(lens)
+    q, k, v, do = (t[0] for t in training_inputs(1, T, T, wl.Hq, wl.Hkv, wl.d, device=dev, seed=23))
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), device=dev)
+    mx = max(lens)
+    pairs = sum(visible_pairs(1, n, n, wl.Hq, wl.Hkv, wl.quad) for n in lens)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(max(3, args.steps))]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        o, lse = cowa.cowa_fwd_varlen(q, k, v, cu, cu, mx, mx, wl.quad)
+        if ev is not None:
+            ev[1].record(stream)
+        cowa.cowa_bwd_varlen(q, k, v, o, lse, do, cu, cu, mx, mx, wl.quad)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    for ev in evs:
+        flush.zero_()
+        step(ev)
+    torch.cuda.synchronize()
+    cowa.cowa_get_device_error(dev)
+    t_f, t_b = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in evs) / len(evs),
+                               sum(e[1].elapsed_time(e[2]) for e in evs) / len(evs)], world, dev)
+    fwd_tf = pairs * 4 * wl.d / (t_f * 1e-3) / 1e12
+    bwd_tf = pairs * 10 * wl.d / (t_b * 1e-3) / 1e12
+    return {"sequences": len(lens), "tokens": T, "min_len": min(lens), "max_len": mx,
+            "visible_pairs": pairs, "fwd_ms": round(t_f, 4), "bwd_ms": round(t_b, 4),
+            "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": round(bwd_tf, 2),
+            "fwd_frac": round(fwd_tf / peaks["bf16_tflops"], 4), "bwd_frac": round(bwd_tf / peaks["bf16_tflops"], 4),
+            "lengths": "log-uniform in [L/16, L], seed 17"}
 
 
 def run_decode_workload(args, cowa, dev, stream, flush, world, peaks, peak_src):
@@ -641,6 +699,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=512, help="query rows per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-workload", dest="decode_workload", action="store_false")
+    ap.add_argument("--no-packed", dest="packed", action="store_false",
+                    help="skip the packed variable-length batch of the workload's heads and windows")
     ap.add_argument("--no-full-mask", dest="full_mask", action="store_false",
                     help="skip the full-causal-mask control run of the same step")
     args = ap.parse_args()

@@ -99,6 +99,41 @@ COWA_API int cowa_abi_version(void);
 COWA_API uint64_t cowa_launch_count(void);
 
 /*
+ * Packed (variable-length) batches for training (chunked prefill included):
+ * sequence b owns query rows [cu_q[b], cu_q[b+1]) of q / o / dq / dO and key
+ * rows [cu_k[b], cu_k[b+1]) of k / v / dk / dv, each tensor [total, H, d]
+ * bf16 with the given (token, head) strides in elements (multiples of 8, last
+ * dim contiguous, 16-byte aligned bases).  cu_q / cu_k are device int32
+ * arrays of B + 1 ascending offsets; max_q / max_k bound every sequence's
+ * length.  Each sequence is aligned bottom-right on its own (p = i + Lk_b -
+ * Lq_b), exactly as a batch of one (paper digest, method key points: the
+ * same position rule for training, prefill and decoding).  LSE is fp32
+ * [Hq, total_q].  A sequence whose offsets do not fit the tensors or exceed
+ * max_q / max_k is treated as empty and reported by cowa_get_device_error
+ * (COWA_ERR_DEVICE); no access leaves the tensors.  Batches without any key
+ * (or, for the backward, any query) are refused with COWA_ERR_UNSUPPORTED.
+ */
+typedef struct {
+    int64_t B;                   /* sequences */
+    int64_t total_q, total_k;    /* rows of the packed query / key tensors */
+    int64_t max_q, max_k;        /* longest query / key sequence */
+    int64_t Hq, Hkv, d;
+    int64_t q_stride[2], k_stride[2], v_stride[2], o_stride[2]; /* token, head */
+    int64_t kv_head_offset;
+} cowa_varlen_shape_t;
+
+COWA_API size_t cowa_fwd_varlen_workspace_size(const cowa_varlen_shape_t *shape, cowa_quad_t quad);
+COWA_API size_t cowa_bwd_varlen_workspace_size(const cowa_varlen_shape_t *shape, cowa_quad_t quad);
+COWA_API int cowa_fwd_varlen(const cowa_varlen_shape_t *shape, cowa_quad_t quad, float softmax_scale,
+                             const int32_t *cu_q, const int32_t *cu_k, const void *q, const void *k,
+                             const void *v, void *o, float *lse, void *workspace, size_t workspace_bytes,
+                             void *stream);
+COWA_API int cowa_bwd_varlen(const cowa_varlen_shape_t *shape, cowa_quad_t quad, float softmax_scale,
+                             const int32_t *cu_q, const int32_t *cu_k, const void *q, const void *k,
+                             const void *v, const void *o, const float *lse, const void *dout, void *dq,
+                             void *dk, void *dv, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Windowed decode cache (paper: decoding reads only each head's windows;
  * Digest, execution notes, and the decode memory saving of the abstract).
  * For a horizon of R query positions [origin[b], origin[b] + R) of sequence

@@ -30,6 +30,7 @@ __all__ = ["CowaError", "cowa_fwd", "cowa_bwd", "cowa_decode", "cowa_default_qua
            "cowa_decode_workspace_size", "cowa_get_device_error", "cowa_launch_count",
            "cowa_decode_noalloc", "cowa_trace_start", "cowa_trace_stop", "cowa_trace_entries",
            "cowa_wcache_rows", "cowa_wcache_build", "cowa_wcache_append", "cowa_decode_windowed",
+           "cowa_fwd_varlen", "cowa_bwd_varlen",
            "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -51,6 +52,15 @@ class CowaError(RuntimeError):
 class Quad(ctypes.Structure):
     _fields_ = [("S", ctypes.c_int32), ("N", ctypes.c_int32), ("G", ctypes.c_int32),
                 ("W", ctypes.c_int32)]
+
+
+class VarlenShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("total_q", ctypes.c_int64), ("total_k", ctypes.c_int64),
+                ("max_q", ctypes.c_int64), ("max_k", ctypes.c_int64), ("Hq", ctypes.c_int64),
+                ("Hkv", ctypes.c_int64), ("d", ctypes.c_int64),
+                ("q_stride", ctypes.c_int64 * 2), ("k_stride", ctypes.c_int64 * 2),
+                ("v_stride", ctypes.c_int64 * 2), ("o_stride", ctypes.c_int64 * 2),
+                ("kv_head_offset", ctypes.c_int64)]
 
 
 class Shape(ctypes.Structure):
@@ -102,6 +112,15 @@ def lib():
         L.cowa_tile_classes.argtypes = [i64, i64, i64, Quad, i32, i32, ctypes.c_int, vp, vp, sz, vp]
         L.cowa_get_device_error.restype = ctypes.c_int
         L.cowa_get_device_error.argtypes = [vp]
+        VP = ctypes.POINTER(VarlenShape)
+        for name in ("cowa_fwd_varlen_workspace_size", "cowa_bwd_varlen_workspace_size"):
+            f = getattr(L, name)
+            f.restype = sz
+            f.argtypes = [VP, Quad]
+        L.cowa_fwd_varlen.restype = ctypes.c_int
+        L.cowa_fwd_varlen.argtypes = [VP, Quad, ctypes.c_float] + [vp] * 7 + [vp, sz, vp]
+        L.cowa_bwd_varlen.restype = ctypes.c_int
+        L.cowa_bwd_varlen.argtypes = [VP, Quad, ctypes.c_float] + [vp] * 11 + [vp, sz, vp]
         L.cowa_wcache_rows.restype = i64
         L.cowa_wcache_rows.argtypes = [Quad, i32]
         L.cowa_wcache_build.restype = ctypes.c_int
@@ -282,6 +301,75 @@ def cowa_decode(q, k_cache, v_cache, seqlens, quad, softmax_scale=None, kv_head_
                          _ptr(seqlens), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                          _stream(q4.device)))
     return out, lse
+
+
+def _packed(t, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16:
+        raise TypeError("%s must be a bf16 CUDA tensor" % name)
+    if t.dim() != 3 or (t.numel() > 0 and t.stride(2) != 1):
+        raise ValueError("%s must be [total, H, d] with a contiguous last dimension" % name)
+
+
+def _varlen_shape(q, k, v, o, cu_q, max_q, max_k, kv_head_offset):
+    s2 = lambda t: (ctypes.c_int64 * 2)(t.stride(0), t.stride(1))
+    return VarlenShape(cu_q.numel() - 1, q.shape[0], k.shape[0], int(max_q), int(max_k), q.shape[1], k.shape[1],
+                       q.shape[2], s2(q), s2(k), s2(v), s2(o), int(kv_head_offset))
+
+
+def cowa_fwd_varlen(q, k, v, cu_q, cu_k, max_q, max_k, quad, softmax_scale=None, kv_head_offset=0,
+                    out=None, lse=None, workspace=None):
+    """CoWA forward over a packed batch: q [total_q, Hq, d], k/v [total_k, Hkv, d],
+    cu_q / cu_k int32 CUDA [B + 1] offsets, max_q / max_k the longest
+    sequences.  Returns ``(o [total_q, Hq, d], lse [Hq, total_q])``."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _packed(t, n)
+    _int32_cuda(cu_q, "cu_q")
+    _int32_cuda(cu_k, "cu_k")
+    if cu_k.numel() != cu_q.numel():
+        raise ValueError("cu_q and cu_k must have the same length")
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if lse is None:
+        lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+    _packed(out, "out")
+    shape = _varlen_shape(q, k, v, out, cu_q, max_q, max_k, kv_head_offset)
+    qd = _quad(quad)
+    L = lib()
+    need = L.cowa_fwd_varlen_workspace_size(ctypes.byref(shape), qd)
+    if need == 0:
+        _raise_size_error(L)
+    ws = _workspace(need, q.device, workspace)
+    scale = 0.0 if softmax_scale is None else float(softmax_scale)
+    _check(L.cowa_fwd_varlen(ctypes.byref(shape), qd, scale, _ptr(cu_q), _ptr(cu_k), _ptr(q), _ptr(k), _ptr(v),
+                             _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)))
+    return out, lse
+
+
+def cowa_bwd_varlen(q, k, v, o, lse, dout, cu_q, cu_k, max_q, max_k, quad, softmax_scale=None,
+                    kv_head_offset=0, workspace=None):
+    """CoWA backward over a packed batch; returns ``(dq, dk, dv)`` shaped like
+    q, k, v (dO must have o's strides)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _packed(t, n)
+    _int32_cuda(cu_q, "cu_q")
+    _int32_cuda(cu_k, "cu_k")
+    if dout.stride() != o.stride():
+        raise ValueError("dout must have the strides of o")
+    dq = torch.empty_strided(q.shape, q.stride(), dtype=q.dtype, device=q.device)
+    dk = torch.empty_strided(k.shape, k.stride(), dtype=k.dtype, device=k.device)
+    dv = torch.empty_strided(v.shape, v.stride(), dtype=v.dtype, device=v.device)
+    shape = _varlen_shape(q, k, v, o, cu_q, max_q, max_k, kv_head_offset)
+    qd = _quad(quad)
+    L = lib()
+    need = L.cowa_bwd_varlen_workspace_size(ctypes.byref(shape), qd)
+    if need == 0:
+        _raise_size_error(L)
+    ws = _workspace(need, q.device, workspace)
+    scale = 0.0 if softmax_scale is None else float(softmax_scale)
+    _check(L.cowa_bwd_varlen(ctypes.byref(shape), qd, scale, _ptr(cu_q), _ptr(cu_k), _ptr(q), _ptr(k), _ptr(v),
+                             _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
+                             _stream(q.device)))
+    return dq, dk, dv
 
 
 def _int32_cuda(t, name):

@@ -401,6 +401,7 @@ int cowa_fwd(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const
     fill_common(p, s, quad, softmax_scale);
     p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
     p.B = (int)s->B; p.Lq = (int)s->Lq; p.Lk = (int)s->Lk;
+    p.lse_ld = s->Lq;
     // tensor-core path (TMA + tcgen05); with no keys at all there is nothing
     // to map, and the warp-level kernel writes the empty rows
     const bool tc = s->Lk > 0;
@@ -441,6 +442,7 @@ int cowa_bwd(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const
     p.q = q; p.k = k; p.v = v; p.o = (void *)o; p.lse_in = lse; p.dout = dout;
     p.dq = dq; p.dk = dk; p.dv = dv;
     p.B = (int)s->B; p.Lq = (int)s->Lq; p.Lk = (int)s->Lk;
+    p.lse_ld = s->Lq;
     char *w = (char *)ws;
     char *rows_ws = w;
     w += align256((size_t)(s->B * s->Hq * cowa::bwd5_lq_pad(s->Lq)) * sizeof(float2));
@@ -628,6 +630,165 @@ static int decode_common(const cowa_shape_t *s, cowa_quad_t quad, float softmax_
     p.horizon = horizon;
     cudaError_t e = cowa::launch_decode(p, (int)s->d, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return COWA_OK;
+}
+
+// ------------------------------------------------------- packed batches --
+static int check_varlen(const cowa_varlen_shape_t *s, cowa_quad_t q)
+{
+    if (!s) return fail(COWA_ERR_INVALID_ARG, "shape is NULL");
+    if (s->B < 0 || s->total_q < 0 || s->total_k < 0 || s->max_q < 0 || s->max_k < 0 || s->Hq < 0 ||
+        s->Hkv < 0 || s->kv_head_offset < 0)
+        return fail(COWA_ERR_INVALID_ARG, "negative size in shape");
+    if (s->total_q >= kMaxLen || s->total_k >= kMaxLen || s->B > 65535 || s->Hq > 65535 || s->Hkv > 65535)
+        return fail(COWA_ERR_UNSUPPORTED, "token counts must be < 2^30, sequences/heads <= 65535");
+    if (s->max_q > s->total_q || s->max_k > s->total_k)
+        return fail(COWA_ERR_INVALID_ARG, "longest sequence exceeds the token count");
+    if (s->Hq > 0 && (s->Hkv == 0 || s->Hq % s->Hkv))
+        return fail(COWA_ERR_INVALID_ARG, "Hq=%lld is not a multiple of Hkv=%lld", (long long)s->Hq,
+                    (long long)s->Hkv);
+    if (s->d != 64 && s->d != 128)
+        return fail(COWA_ERR_UNSUPPORTED, "head dim %lld (supported: 64, 128)", (long long)s->d);
+    if (s->kv_head_offset + s->Hkv > kMaxLen) return fail(COWA_ERR_INVALID_ARG, "kv_head_offset too large");
+    if (s->B * s->Hq * cdiv(s->max_q, 32) > 0x7fffffffll || s->B * s->Hkv * cdiv(s->max_k, 32) > 0x7fffffffll)
+        return fail(COWA_ERR_UNSUPPORTED, "sequences * heads * length / 32 exceeds 2^31 - 1");
+    int r = check_quad(q);
+    if (r) return r;
+    const int64_t *st[4] = {s->q_stride, s->k_stride, s->v_stride, s->o_stride};
+    const char *nm[4] = {"q", "k", "v", "o"};
+    for (int t = 0; t < 4; ++t)
+        for (int a = 0; a < 2; ++a)
+            if (st[t][a] < 0 || st[t][a] % 8)
+                return fail(COWA_ERR_ALIGNMENT, "%s stride[%d] = %lld is not a non-negative multiple of 8 elements",
+                            nm[t], a, (long long)st[t][a]);
+    return COWA_OK;
+}
+
+// AttnParams of a packed batch: one batch entry of total rows, per-sequence
+// offsets from cu_q / cu_k, schedules per sequence
+static void fill_varlen(cowa::AttnParams &p, const cowa_varlen_shape_t *s, cowa_quad_t q, float scale,
+                        const int32_t *cu_q, const int32_t *cu_k)
+{
+    for (int a = 0; a < 2; ++a) {
+        p.qs[a + 1] = s->q_stride[a];
+        p.ks[a + 1] = s->k_stride[a];
+        p.vs[a + 1] = s->v_stride[a];
+        p.os[a + 1] = s->o_stride[a];
+    }
+    p.qs[0] = p.ks[0] = p.vs[0] = p.os[0] = 0;
+    p.Hq = (int)s->Hq;
+    p.Hkv = (int)s->Hkv;
+    p.g = s->Hkv > 0 ? (int)(s->Hq / s->Hkv) : 1;
+    p.S = q.S; p.N = q.N; p.G = q.G; p.W = q.W;
+    p.kv_head_offset = (int)s->kv_head_offset;
+    p.scale = resolve_scale(scale, s->d);
+    p.scale_log2 = p.scale * 1.4426950408889634f;
+    p.err = device_error_word();
+    p.B = (int)s->B;
+    p.Lq = (int)s->max_q;
+    p.Lk = (int)s->max_k;
+    p.cu_q = cu_q;
+    p.cu_k = cu_k;
+    p.total_q = (int)s->total_q;
+    p.total_k = (int)s->total_k;
+    p.lse_ld = s->total_q;
+}
+
+size_t cowa_fwd_varlen_workspace_size(const cowa_varlen_shape_t *s, cowa_quad_t q)
+{
+    if (check_varlen(s, q)) return 0;
+    return sched_bytes(s->B * s->Hkv, cdiv(s->max_q, cowa::kFwd5BM)) + 256;
+}
+
+size_t cowa_bwd_varlen_workspace_size(const cowa_varlen_shape_t *s, cowa_quad_t q)
+{
+    if (check_varlen(s, q)) return 0;
+    return align256((size_t)(s->B * s->Hq * cowa::bwd5_lq_pad(s->max_q)) * sizeof(float2)) +
+           sched_bytes(s->B * s->Hkv, cdiv(s->max_q, 64)) + sched_bytes(s->B * s->Hkv, cdiv(s->max_k, 64)) + 256;
+}
+
+int cowa_fwd_varlen(const cowa_varlen_shape_t *s, cowa_quad_t quad, float softmax_scale, const int32_t *cu_q,
+                    const int32_t *cu_k, const void *q, const void *k, const void *v, void *o, float *lse, void *ws,
+                    size_t ws_bytes, void *stream)
+{
+    int r = check_varlen(s, quad);
+    if (r) return r;
+    const bool qrows = s->B * s->total_q * s->Hq > 0 && s->max_q > 0;
+    if (!qrows) return COWA_OK;
+    if (s->total_k == 0 || s->max_k == 0)
+        return fail(COWA_ERR_UNSUPPORTED, "packed batch without keys (every output would be empty)");
+    if ((r = check_ptr(q, true, "q")) || (r = check_ptr(k, true, "k")) || (r = check_ptr(v, true, "v")) ||
+        (r = check_ptr(o, true, "o")) || (r = check_ptr(lse, true, "lse")))
+        return r;
+    if (!cu_q || !cu_k) return fail(COWA_ERR_INVALID_ARG, "cu_q / cu_k is NULL");
+    if ((r = check_device(nullptr))) return r;
+    const size_t need = cowa_fwd_varlen_workspace_size(s, quad);
+    if (!ws || ws_bytes < need || (uintptr_t)ws % 256)
+        return fail(COWA_ERR_WORKSPACE, "fwd workspace needs %zu bytes, 256-byte aligned (got %zu)", need, ws_bytes);
+    cudaStream_t st = (cudaStream_t)stream;
+    cowa::AttnParams p{};
+    fill_varlen(p, s, quad, softmax_scale, cu_q, cu_k);
+    p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
+    const int BN = cowa::fwd5_bn((int)s->d);
+    p.nqt = (int)cdiv(s->max_q, cowa::kFwd5BM);
+    p.nkt = (int)cdiv(s->max_k, BN);
+    p.sched = (int *)ws;
+    p.sched_bs = (long long)p.Hkv * p.nqt * cowa::kSchedInts;
+    cudaError_t e = cowa::launch_schedule((int *)ws, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W,
+                                          cowa::kFwd5BM, BN, 0, st, cu_q, cu_k, p.B, p.total_q, p.total_k, p.err);
+    if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+    e = cowa::launch_fwd_sm100(p, (int)s->d, st);
+    if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
+    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    return COWA_OK;
+}
+
+int cowa_bwd_varlen(const cowa_varlen_shape_t *s, cowa_quad_t quad, float softmax_scale, const int32_t *cu_q,
+                    const int32_t *cu_k, const void *q, const void *k, const void *v, const void *o,
+                    const float *lse, const void *dout, void *dq, void *dk, void *dv, void *ws, size_t ws_bytes,
+                    void *stream)
+{
+    int r = check_varlen(s, quad);
+    if (r) return r;
+    if (s->B == 0 || s->Hq == 0 || (s->total_q == 0 && s->total_k == 0)) return COWA_OK;
+    if (s->total_q == 0 || s->total_k == 0 || s->max_q == 0 || s->max_k == 0)
+        return fail(COWA_ERR_UNSUPPORTED, "packed batch without queries or keys (every gradient would be zero)");
+    if ((r = check_ptr(q, true, "q")) || (r = check_ptr(k, true, "k")) || (r = check_ptr(v, true, "v")) ||
+        (r = check_ptr(o, true, "o")) || (r = check_ptr(lse, true, "lse")) || (r = check_ptr(dout, true, "dout")) ||
+        (r = check_ptr(dq, true, "dq")) || (r = check_ptr(dk, true, "dk")) || (r = check_ptr(dv, true, "dv")))
+        return r;
+    if (!cu_q || !cu_k) return fail(COWA_ERR_INVALID_ARG, "cu_q / cu_k is NULL");
+    if ((r = check_device(nullptr))) return r;
+    const size_t need = cowa_bwd_varlen_workspace_size(s, quad);
+    if (!ws || ws_bytes < need || (uintptr_t)ws % 256)
+        return fail(COWA_ERR_WORKSPACE, "bwd workspace needs %zu bytes, 256-byte aligned (got %zu)", need, ws_bytes);
+    cudaStream_t st = (cudaStream_t)stream;
+    cowa::AttnParams p{};
+    fill_varlen(p, s, quad, softmax_scale, cu_q, cu_k);
+    p.q = q; p.k = k; p.v = v; p.o = (void *)o; p.lse_in = lse; p.dout = dout;
+    p.dq = dq; p.dk = dk; p.dv = dv;
+    char *w = (char *)ws;
+    char *rows_ws = w;
+    const long long lq_pad = cowa::bwd5_lq_pad(s->max_q);
+    w += align256((size_t)(s->B * s->Hq * lq_pad) * sizeof(float2));
+    int *sched_q = (int *)w;
+    w += sched_bytes(s->B * s->Hkv, cdiv(s->max_q, 64));
+    int *sched_t = (int *)w;
+    const int D = (int)s->d;
+    const int kv_bm = cowa::bwd5_kv_bm(D), dq_bn = cowa::bwd5_dq_bn(D);
+    const int nqt = (int)cdiv(s->max_q, cowa::kBwd5QTile), nkt = (int)cdiv(s->max_k, cowa::kBwd5KeyTile);
+    p.sched_bs = (long long)p.Hkv * nqt * cowa::kSchedInts;
+    p.sched_t_bs = (long long)p.Hkv * nkt * cowa::kSchedInts;
+    cudaError_t e = cowa::launch_schedule(sched_q, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W,
+                                          cowa::kBwd5QTile, dq_bn, 0, st, cu_q, cu_k, p.B, p.total_q, p.total_k,
+                                          p.err);
+    if (e == cudaSuccess)
+        e = cowa::launch_schedule(sched_t, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W, kv_bm,
+                                  cowa::kBwd5KeyTile, 1, st, cu_q, cu_k, p.B, p.total_q, p.total_k, p.err);
+    if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+    e = cowa::launch_bwd_sm100(p, D, (float2 *)rows_ws, (int)lq_pad, sched_q, nqt, sched_t, nkt, st);
+    if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return COWA_OK;
 }
 

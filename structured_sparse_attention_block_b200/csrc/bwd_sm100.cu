@@ -57,12 +57,13 @@ __global__ void bwd_prep_kernel(const AttnParams p, float2 *lsd, int lq_pad)
     const int i = (int)(row % lq_pad);
     const long long bh = row / lq_pad;  // b * Hq + hq
     const int hq = (int)(bh % p.Hq), b = (int)(bh / p.Hq);
+    const SeqGeom sg = seq_geom(p, b);
     float s = 0.f, nl = -CUDART_INF_F;
-    if (i < p.Lq) {
-        const __nv_bfloat16 *o = reinterpret_cast<const __nv_bfloat16 *>(p.o) + b * p.os[0] +
-                                 (long long)i * p.os[1] + hq * p.os[2];
-        const __nv_bfloat16 *dout = reinterpret_cast<const __nv_bfloat16 *>(p.dout) + b * p.os[0] +
-                                    (long long)i * p.os[1] + hq * p.os[2];
+    if (i < sg.Lq) {
+        const __nv_bfloat16 *o = reinterpret_cast<const __nv_bfloat16 *>(p.o) + sg.tb * p.os[0] +
+                                 (long long)(sg.qoff + i) * p.os[1] + hq * p.os[2];
+        const __nv_bfloat16 *dout = reinterpret_cast<const __nv_bfloat16 *>(p.dout) + sg.tb * p.os[0] +
+                                    (long long)(sg.qoff + i) * p.os[1] + hq * p.os[2];
         constexpr int PER = D / 32;
 #pragma unroll
         for (int x = 0; x < PER; x += 2) {
@@ -70,7 +71,7 @@ __global__ void bwd_prep_kernel(const AttnParams p, float2 *lsd, int lq_pad)
             const __nv_bfloat162 c = *reinterpret_cast<const __nv_bfloat162 *>(dout + lane * PER + x);
             s += __bfloat162float(a.x) * __bfloat162float(c.x) + __bfloat162float(a.y) * __bfloat162float(c.y);
         }
-        const float lv = p.lse_in[bh * p.Lq + i];
+        const float lv = p.lse_in[((long long)sg.tb * p.Hq + hq) * p.lse_ld + sg.qoff + i];
         nl = lv == -CUDART_INF_F ? -CUDART_INF_F : -lv * 1.4426950408889634f;
     }
 #pragma unroll
@@ -146,11 +147,13 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const TilePos pos = tile_pos(p.Hkv, p.B);
     const int kt = pos.step, hl = pos.slot, b = pos.b;  // sink keys first
-    const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
-    const int delta_pos = p.Lk - p.Lq;
+    const SeqGeom sg = seq_geom(p, b);
     const int c0 = kt * BN;
+    if (c0 >= sg.Lk) return;  // past the end of this sequence of a packed batch
+    const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
+    const int delta_pos = sg.Lk - sg.Lq;
 
-    const int4 *e4 = reinterpret_cast<const int4 *>(p.sched_t + ((size_t)hl * p.nkt + kt) * kSchedInts);
+    const int4 *e4 = reinterpret_cast<const int4 *>(p.sched_t + b * p.sched_t_bs + ((size_t)hl * p.nkt + kt) * kSchedInts);
     const int4 e0 = e4[0], e1 = e4[1];
     const int nr = e0.x;
     const int lo0 = e0.y, lo1 = e0.w, lo2 = e1.y;
@@ -203,8 +206,8 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
         if (lane == 0) {
             mbar_expect_tx(KV_LOADED, 2 * C::KV_BYTES);
             for (int kb = 0; kb < KB; ++kb) {
-                tma_load_4d(sK + kb * BN * 128, &a.tk, KV_LOADED, kb * 64, c0, hl, b);
-                tma_load_4d(sV + kb * BN * 128, &a.tv, KV_LOADED, kb * 64, c0, hl, b);
+                tma_load_4d(sK + kb * BN * 128, &a.tk, KV_LOADED, kb * 64, sg.koff + c0, hl, sg.tb);
+                tma_load_4d(sV + kb * BN * 128, &a.tv, KV_LOADED, kb * 64, sg.koff + c0, hl, sg.tb);
             }
             int issued = 0;
             for (int u = 0; u < ntask; ++u) {
@@ -214,8 +217,8 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
                 task(u, hq, qt);
                 mbar_expect_tx(Q_FULL(s), 2 * C::QT_BYTES + C::LSD_BYTES);
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_4d(stage_q(s) + kb * BM * 128, &a.tq, Q_FULL(s), kb * 64, qt * BM, hq, b);
-                    tma_load_4d(stage_do(s) + kb * BM * 128, &a.tdo, Q_FULL(s), kb * 64, qt * BM, hq, b);
+                    tma_load_4d(stage_q(s) + kb * BM * 128, &a.tq, Q_FULL(s), kb * 64, sg.qoff + qt * BM, hq, sg.tb);
+                    tma_load_4d(stage_do(s) + kb * BM * 128, &a.tdo, Q_FULL(s), kb * 64, sg.qoff + qt * BM, hq, sg.tb);
                 }
                 bulk_load(stage_q(s) + 2 * C::QT_BYTES,
                           a.lsd + ((long long)b * p.Hq + hq) * a.lq_pad + (long long)qt * BM, C::LSD_BYTES,
@@ -301,7 +304,7 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
         // aligned positions p that see key jg: sink [jg, Lk-1], near
         // [jg, jg+N-1], long [jg+c, jg+e-1], as 32-bit bounds (an empty
         // interval has hi < lo; every position is below 2^30)
-        const long long pmax = (long long)p.Lk - 1;
+        const long long pmax = (long long)sg.Lk - 1;
         const int snk_hi = jg < w.S ? (int)pmax : -1;
         const int nr_hi = w.N > 0 ? (int)min((long long)jg + w.N - 1, pmax) : -1;
         const int lg_lo = (int)min((long long)jg + w.c, pmax + 1);
@@ -323,9 +326,9 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
                 ++gi;
             }
             const int q0 = qt * BM;
-            const int nrows = min(BM, p.Lq - q0);
+            const int nrows = min(BM, sg.Lq - q0);
             const int pa = q0 + delta_pos;
-            const bool full = tile_full(pa, pa + nrows - 1, c0, BN, p.Lk, w);
+            const bool full = tile_full(pa, pa + nrows - 1, c0, BN, sg.Lk, w);
             uint32_t vis[BM / 32];
 #pragma unroll
             for (int c = 0; c < BM / 32; ++c) {
@@ -393,8 +396,10 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
         const float f = x == 0 ? p.scale : 1.f;
         const uint32_t tg = tmem + (x == 0 ? C::T_DK : C::T_DV) + lane_off;
         __nv_bfloat16 *grow_ = x == 0
-            ? reinterpret_cast<__nv_bfloat16 *>(p.dk) + b * p.ks[0] + (long long)jg * p.ks[1] + hl * p.ks[2]
-            : reinterpret_cast<__nv_bfloat16 *>(p.dv) + b * p.vs[0] + (long long)jg * p.vs[1] + hl * p.vs[2];
+            ? reinterpret_cast<__nv_bfloat16 *>(p.dk) + sg.tb * p.ks[0] + (long long)(sg.koff + jg) * p.ks[1] +
+                  hl * p.ks[2]
+            : reinterpret_cast<__nv_bfloat16 *>(p.dv) + sg.tb * p.vs[0] + (long long)(sg.koff + jg) * p.vs[1] +
+                  hl * p.vs[2];
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) {
             uint32_t g[16];
@@ -408,7 +413,7 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
             uint32_t pk[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) pk[e] = pack2(__uint_as_float(g[2 * e]) * f, __uint_as_float(g[2 * e + 1]) * f);
-            if (jg < p.Lk) {
+            if (jg < sg.Lk) {
                 uint4 *dst = reinterpret_cast<uint4 *>(grow_ + c * 16);
                 dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
@@ -475,13 +480,15 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
     const int hq0 = hl * p.g + NSLOT * pair;
     const int nslot = min(NSLOT, p.g - NSLOT * pair);
     const int b = pos.b;
-    const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
-    const int delta_pos = p.Lk - p.Lq;
+    const SeqGeom sg = seq_geom(p, b);
     const int i0 = qt * BM;
-    const int nrows = min(BM, p.Lq - i0);
+    if (i0 >= sg.Lq) return;  // past the end of this sequence of a packed batch
+    const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
+    const int delta_pos = sg.Lk - sg.Lq;
+    const int nrows = min(BM, sg.Lq - i0);
     const int pa = i0 + delta_pos, pb = i0 + nrows - 1 + delta_pos;
 
-    const int4 *e4 = reinterpret_cast<const int4 *>(p.sched + ((size_t)hl * p.nqt + qt) * kSchedInts);
+    const int4 *e4 = reinterpret_cast<const int4 *>(p.sched + b * p.sched_bs + ((size_t)hl * p.nqt + qt) * kSchedInts);
     const int4 e0 = e4[0], e1 = e4[1];
     const int nr = e0.x;
     const int lo0 = e0.y, lo1 = e0.w, lo2 = e1.y;
@@ -531,8 +538,8 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
             mbar_expect_tx(BAR_Q, nslot * 2 * C::QT_BYTES);
             for (int x = 0; x < nslot; ++x)
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_4d(sQ(x) + kb * BM * 128, &a.tq, BAR_Q, kb * 64, i0, hq0 + x, b);
-                    tma_load_4d(sDO(x) + kb * BM * 128, &a.tdo, BAR_Q, kb * 64, i0, hq0 + x, b);
+                    tma_load_4d(sQ(x) + kb * BM * 128, &a.tq, BAR_Q, kb * 64, sg.qoff + i0, hq0 + x, sg.tb);
+                    tma_load_4d(sDO(x) + kb * BM * 128, &a.tdo, BAR_Q, kb * 64, sg.qoff + i0, hq0 + x, sg.tb);
                 }
             int issued = 0;
             for (int t = 0; t < ntiles; ++t) {
@@ -542,8 +549,8 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
                 mbar_expect_tx(KV_FULL(s), C::STAGE_BYTES);
                 const uint32_t sk = sStage + s * C::STAGE_BYTES, sv = sk + C::KV_BYTES;
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_4d(sk + kb * BN * 128, &a.tk, KV_FULL(s), kb * 64, kt * BN, hl, b);
-                    tma_load_4d(sv + kb * BN * 128, &a.tv, KV_FULL(s), kb * 64, kt * BN, hl, b);
+                    tma_load_4d(sk + kb * BN * 128, &a.tk, KV_FULL(s), kb * 64, sg.koff + kt * BN, hl, sg.tb);
+                    tma_load_4d(sv + kb * BN * 128, &a.tv, KV_FULL(s), kb * 64, sg.koff + kt * BN, hl, sg.tb);
                 }
                 issued = t + 1;
             }
@@ -624,7 +631,7 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
         const bool active = x < nslot;
         const int hq = hq0 + x;
         float nl = -CUDART_INF_F, nd = 0.f;
-        if (active && i0 + r < p.Lq) {
+        if (active && i0 + r < sg.Lq) {
             const float2 v = a.lsd[((long long)b * p.Hq + hq) * a.lq_pad + i0 + r];
             nl = v.x;
             nd = v.y;
@@ -635,7 +642,7 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
         for (int t = 0; active && t < ntiles; ++t) {
             // tile set-up, independent of the scores: done while they land
             const int kt = tile_of(t);
-            const bool full = tile_full(pa, pb, kt * BN, BN, p.Lk, w);
+            const bool full = tile_full(pa, pb, kt * BN, BN, sg.Lk, w);
             uint32_t vis[BN / 32];
 #pragma unroll
             for (int c = 0; c < BN / 32; ++c) {
@@ -695,8 +702,8 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
         tc_fence_after();
         if (active) {
             const bool have = ok && ntiles > 0;
-            __nv_bfloat16 *drow = reinterpret_cast<__nv_bfloat16 *>(p.dq) + b * p.qs[0] +
-                                  (long long)(i0 + r) * p.qs[1] + hq * p.qs[2];
+            __nv_bfloat16 *drow = reinterpret_cast<__nv_bfloat16 *>(p.dq) + sg.tb * p.qs[0] +
+                                  (long long)(sg.qoff + i0 + r) * p.qs[1] + hq * p.qs[2];
 #pragma unroll
             for (int c = 0; c < D / 16; ++c) {
                 uint32_t g[16];
@@ -758,10 +765,13 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, c
     a.lsd = lsd;
     a.lq_pad = lq_pad;
     // dK/dV: query tiles of BM rows, key tiles of 128
-    if (!make_bshd_map(&a.tq, p.q, D, p.Lq, p.Hq, p.B, p.qs, K::BM) ||
-        !make_bshd_map(&a.tdo, p.dout, D, p.Lq, p.Hq, p.B, p.os, K::BM) ||
-        !make_bshd_map(&a.tk, p.k, D, p.Lk, p.Hkv, p.B, p.ks, K::BN) ||
-        !make_bshd_map(&a.tv, p.v, D, p.Lk, p.Hkv, p.B, p.vs, K::BN))
+    // a packed batch is one batch entry of total_q / total_k rows
+    const long long Lq_map = p.cu_q ? p.total_q : p.Lq, Lk_map = p.cu_q ? p.total_k : p.Lk;
+    const long long B_map = p.cu_q ? 1 : p.B;
+    if (!make_bshd_map(&a.tq, p.q, D, Lq_map, p.Hq, B_map, p.qs, K::BM) ||
+        !make_bshd_map(&a.tdo, p.dout, D, Lq_map, p.Hq, B_map, p.os, K::BM) ||
+        !make_bshd_map(&a.tk, p.k, D, Lk_map, p.Hkv, B_map, p.ks, K::BN) ||
+        !make_bshd_map(&a.tv, p.v, D, Lk_map, p.Hkv, B_map, p.vs, K::BN))
         return cudaErrorInvalidValue;
     a.p.sched_t = sched_kv;
     a.p.nkt = nkt_kv;
@@ -775,10 +785,10 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, c
         if (e != cudaSuccess) return e;
     }
     // dQ: query tiles of 128 rows, key tiles of BN
-    if (!make_bshd_map(&a.tq, p.q, D, p.Lq, p.Hq, p.B, p.qs, Q::BM) ||
-        !make_bshd_map(&a.tdo, p.dout, D, p.Lq, p.Hq, p.B, p.os, Q::BM) ||
-        !make_bshd_map(&a.tk, p.k, D, p.Lk, p.Hkv, p.B, p.ks, Q::BN) ||
-        !make_bshd_map(&a.tv, p.v, D, p.Lk, p.Hkv, p.B, p.vs, Q::BN))
+    if (!make_bshd_map(&a.tq, p.q, D, Lq_map, p.Hq, B_map, p.qs, Q::BM) ||
+        !make_bshd_map(&a.tdo, p.dout, D, Lq_map, p.Hq, B_map, p.os, Q::BM) ||
+        !make_bshd_map(&a.tk, p.k, D, Lk_map, p.Hkv, B_map, p.ks, Q::BN) ||
+        !make_bshd_map(&a.tv, p.v, D, Lk_map, p.Hkv, B_map, p.vs, Q::BN))
         return cudaErrorInvalidValue;
     a.p.sched = sched_dq;
     a.p.nqt = nqt_dq;

@@ -108,13 +108,15 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
     const int hq0 = hl * p.g + 2 * pair;
     const int nslot = (2 * pair + 1 < p.g) ? 2 : 1;  // an odd group leaves the last head alone
     const int b = pos.b;
-    const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
-    const int delta = p.Lk - p.Lq;
+    const SeqGeom sg = seq_geom(p, b);
     const int i0 = qt * BM;
-    const int nrows = min(BM, p.Lq - i0);
+    if (i0 >= sg.Lq) return;  // past the end of this sequence of a packed batch
+    const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
+    const int delta = sg.Lk - sg.Lq;
+    const int nrows = min(BM, sg.Lq - i0);
     const int pa = i0 + delta, pb = i0 + nrows - 1 + delta;
 
-    const int4 *e4 = reinterpret_cast<const int4 *>(p.sched + ((size_t)hl * p.nqt + qt) * kSchedInts);
+    const int4 *e4 = reinterpret_cast<const int4 *>(p.sched + b * p.sched_bs + ((size_t)hl * p.nqt + qt) * kSchedInts);
     const int4 e0 = e4[0], e1 = e4[1];
     const int nr = e0.x;
     const int lo0 = e0.y, lo1 = e0.w, lo2 = e1.y;
@@ -167,10 +169,12 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
     if (warp == 8) {
         // ------------------------------------------------------------ TMA
         if (lane == 0) {
+            const SeqGeom sp = seq_geom(p, b);  // row offsets in the tensors
             mbar_expect_tx(BAR_Q, nslot * C::Q_BYTES);
             for (int x = 0; x < nslot; ++x)
                 for (int kb = 0; kb < KB; ++kb)
-                    tma_load_4d(sQ + x * C::Q_BYTES + kb * BM * 128, &a.tq, BAR_Q, kb * 64, i0, hq0 + x, b);
+                    tma_load_4d(sQ + x * C::Q_BYTES + kb * BM * 128, &a.tq, BAR_Q, kb * 64, sp.qoff + i0, hq0 + x,
+                                sp.tb);
             int issued = 0;
             for (int t = 0; t < ntiles; ++t) {
                 const int s = t % ST;
@@ -179,8 +183,8 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                 mbar_expect_tx(KV_FULL(s), 2 * C::KV_BYTES);
                 const uint32_t sk = sStage + s * C::STAGE_BYTES, sv = sk + C::KV_BYTES;
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_4d(sk + kb * BN * 128, &a.tk, KV_FULL(s), kb * 64, kt * BN, hl, b);
-                    tma_load_4d(sv + kb * BN * 128, &a.tv, KV_FULL(s), kb * 64, kt * BN, hl, b);
+                    tma_load_4d(sk + kb * BN * 128, &a.tk, KV_FULL(s), kb * 64, sp.koff + kt * BN, hl, sp.tb);
+                    tma_load_4d(sv + kb * BN * 128, &a.tv, KV_FULL(s), kb * 64, sp.koff + kt * BN, hl, sp.tb);
                 }
                 issued = t + 1;
             }
@@ -265,6 +269,9 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             // Edge tiles build, per 32-key chunk, the bitmask of keys the row
             // sees: the union of its sink, near and long key intervals.
             const int kt = tile_of(t);
+            // (the longest key length serves for the sequence's own: no
+            // covering interval ends past pa <= Lk_b - 1, so a tile reaching
+            // past the sequence's last key is never full)
             const bool full = tile_full(pa, pb, kt * BN, BN, p.Lk, w);
             constexpr int NC = BN / 32;  // 32-column chunks of the row
             uint32_t vis[NC];
@@ -389,6 +396,8 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         tc_fence_after();
         // epilogue: O / (sum of the bf16 P) in bf16, LSE (natural log) from the fp32 sum
         if (active) {
+            // the sequence's offsets again, rather than live across the tile loop
+            const SeqGeom se = seq_geom(p, b);
             const bool have = ok && ntiles > 0;
             float lb = 0.f;  // sum of the bf16 P that O accumulated
             if (have) {
@@ -399,8 +408,8 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             }
             const float inv = (l > 0.f && lb > 0.f) ? 1.f / lb : 0.f;
             const int hq = hq0 + x;
-            __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + b * p.os[0] +
-                                  (long long)(i0 + r) * p.os[1] + hq * p.os[2];
+            __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + se.tb * p.os[0] +
+                                  (long long)(se.qoff + i0 + r) * p.os[1] + hq * p.os[2];
 #pragma unroll
             for (int c = 0; c < D / 16; ++c) {
                 uint32_t o[16];
@@ -422,7 +431,7 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                 }
             }
             if (r < nrows)
-                p.lse[((long long)b * p.Hq + hq) * p.Lq + i0 + r] =
+                p.lse[((long long)se.tb * p.Hq + hq) * p.lse_ld + se.qoff + i0 + r] =
                     l > 0.f ? m_run * 0.69314718055994531f + logf(l) : -CUDART_INF_F;
         }
     }
@@ -486,9 +495,12 @@ static cudaError_t launch_fwd5_d(const AttnParams &p, cudaStream_t st)
     memset(&a, 0, sizeof a);
     a.p = p;
     a.npair = (p.g + 1) / 2;
-    if (!make_bshd_map(&a.tq, p.q, D, p.Lq, p.Hq, p.B, p.qs, C::BM) ||
-        !make_bshd_map(&a.tk, p.k, D, p.Lk, p.Hkv, p.B, p.ks, C::BN) ||
-        !make_bshd_map(&a.tv, p.v, D, p.Lk, p.Hkv, p.B, p.vs, C::BN))
+    // a packed batch is one batch entry of total_q / total_k rows
+    const long long Lq_map = p.cu_q ? p.total_q : p.Lq, Lk_map = p.cu_q ? p.total_k : p.Lk;
+    const long long B_map = p.cu_q ? 1 : p.B;
+    if (!make_bshd_map(&a.tq, p.q, D, Lq_map, p.Hq, B_map, p.qs, C::BM) ||
+        !make_bshd_map(&a.tk, p.k, D, Lk_map, p.Hkv, B_map, p.ks, C::BN) ||
+        !make_bshd_map(&a.tv, p.v, D, Lk_map, p.Hkv, B_map, p.vs, C::BN))
         return cudaErrorInvalidValue;
     const unsigned blocks = tile_grid_blocks(p.nqt, (long long)p.Hkv * a.npair, p.B);
     if (!blocks) return cudaErrorInvalidConfiguration;

@@ -25,7 +25,46 @@ struct AttnParams {
     int nqt, nkt;           // tiles of the schedule in use
     float scale, scale_log2;
     int *err;               // device error word (status code of a failed device check)
+    // Packed (variable-length) batch: sequence b owns query rows
+    // [cu_q[b], cu_q[b+1]) and key rows [cu_k[b], cu_k[b+1]) of tensors with
+    // total_q / total_k rows; Lq / Lk are then the longest sequence.  With
+    // cu_q == nullptr the batch is uniform (B sequences of Lq / Lk rows).
+    const int *cu_q, *cu_k;
+    int total_q, total_k;
+    long long lse_ld;                 // LSE row pitch: Lq, or total_q when packed
+    long long sched_bs, sched_t_bs;   // schedule ints between sequences (0: shared)
 };
+
+// Lengths and row offsets of sequence b, and its batch coordinate (b for a
+// uniform batch, 0 for a packed one, whose rows are offsets into batch 0).
+// A packed sequence whose offsets do not fit its tensors or exceed the
+// longest length is reported and treated as empty.
+struct SeqGeom {
+    int Lq, Lk, qoff, koff, tb;
+};
+__device__ __forceinline__ SeqGeom seq_geom(const AttnParams &p, int b)
+{
+    SeqGeom g;
+    if (!p.cu_q) {
+        g.Lq = p.Lq;
+        g.Lk = p.Lk;
+        g.qoff = g.koff = 0;
+        g.tb = b;
+        return g;
+    }
+    g.qoff = p.cu_q[b];
+    g.koff = p.cu_k[b];
+    g.Lq = p.cu_q[b + 1] - g.qoff;
+    g.Lk = p.cu_k[b + 1] - g.koff;
+    g.tb = 0;
+    const bool ok = g.qoff >= 0 && g.koff >= 0 && g.Lq >= 0 && g.Lk >= 0 && g.Lq <= p.Lq && g.Lk <= p.Lk &&
+                    g.qoff <= p.total_q - g.Lq && g.koff <= p.total_k - g.Lk;
+    if (!ok) {
+        if (threadIdx.x == 0) atomicExch(p.err, 7);
+        g.Lq = g.Lk = g.qoff = g.koff = 0;
+    }
+    return g;
+}
 
 struct DecodeParams {
     const void *q, *kc, *vc;
@@ -66,9 +105,12 @@ void launch_begin(const char *name, cudaStream_t st);
 void launch_end(cudaStream_t st);
 
 // schedule.cu
+// (cu_q, cu_k, nseq, total_q, total_k, err describe a packed batch: one
+// schedule per sequence, Lq / Lk the longest; nullptr for a uniform batch)
 cudaError_t launch_schedule(int *sched, int Hkv, int kv_head_offset, int Lq,
                             int Lk, int S, int N, int G, int W, int BM, int BN, int transposed,
-                            cudaStream_t st);
+                            cudaStream_t st, const int *cu_q = nullptr, const int *cu_k = nullptr,
+                            int nseq = 1, int total_q = 0, int total_k = 0, int *err = nullptr);
 cudaError_t launch_tile_classes(const int *sched, uint8_t *out, int kv_head, int Lq, int Lk,
                                 int S, int N, int G, int W, int BM, int BN, int transposed,
                                 cudaStream_t st);

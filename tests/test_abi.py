@@ -130,3 +130,20 @@ def test_wcache_rows_and_argument_errors(cowa):
                                  None) == 2
     assert lib.cowa_wcache_append(ctypes.byref(make_shape(cowa)), cowa.Quad(1, 2, 0, 3), 4, p, None, p, p, p, p,
                                   None) == 1  # pos is NULL
+
+
+def test_varlen_argument_errors(cowa):
+    lib = cowa.lib()
+    s2 = lambda a, b: (ctypes.c_int64 * 2)(a, b)
+    def vshape(B=2, tq=100, tk=100, mq=60, mk=60, Hq=4, Hkv=2, d=64, qs=(256, 64)):
+        return cowa.VarlenShape(B, tq, tk, mq, mk, Hq, Hkv, d, s2(*qs), s2(128, 64), s2(128, 64), s2(256, 64), 0)
+    p = ctypes.c_void_p(16)
+    call = lambda sh: lib.cowa_fwd_varlen(ctypes.byref(sh), cowa.Quad(1, 2, 0, 3), 0.0, p, p, p, p, p, p, p, p,
+                                          1 << 20, None)
+    assert call(vshape(mq=101)) == 1          # longest sequence above the token count
+    assert call(vshape(d=96)) == 2
+    assert call(vshape(Hq=3)) == 1
+    assert call(vshape(qs=(250, 64))) == 3    # token stride not a multiple of 8
+    assert call(vshape(tk=0, mk=0)) == 2      # no keys at all
+    assert lib.cowa_fwd_varlen(ctypes.byref(vshape()), cowa.Quad(1, 2, 0, 3), 0.0, None, p, p, p, p, p, p, p,
+                               1 << 20, None) == 1  # cu_q is NULL
