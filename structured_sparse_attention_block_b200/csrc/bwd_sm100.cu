@@ -47,36 +47,39 @@ namespace cowa {
 using namespace sm100;
 
 // ------------------------------------------------------------- preprocess --
+// One row per D/8 lanes (16 bytes of O and of dO each), several rows per warp.
 template <int D>
-__global__ void bwd_prep_kernel(const AttnParams p, float2 *lsd, int lq_pad)
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const AttnParams p, float2 *lsd, int lq_pad)
 {
-    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
+    constexpr int LPR = D / 8, RPW = 32 / LPR;  // lanes per row, rows per warp
+    const int lane = threadIdx.x & 31, piece = lane % LPR;
+    const long long row = ((long long)blockIdx.x * 8 + (threadIdx.x >> 5)) * RPW + lane / LPR;
     const long long total = (long long)p.B * p.Hq * lq_pad;
-    if (row >= total) return;
-    const int i = (int)(row % lq_pad);
-    const long long bh = row / lq_pad;  // b * Hq + hq
-    const int hq = (int)(bh % p.Hq), b = (int)(bh / p.Hq);
-    const SeqGeom sg = seq_geom(p, b);
+    const bool live = row < total;
     float s = 0.f, nl = -CUDART_INF_F;
-    if (i < sg.Lq) {
-        const __nv_bfloat16 *o = reinterpret_cast<const __nv_bfloat16 *>(p.o) + sg.tb * p.os[0] +
-                                 (long long)(sg.qoff + i) * p.os[1] + hq * p.os[2];
-        const __nv_bfloat16 *dout = reinterpret_cast<const __nv_bfloat16 *>(p.dout) + sg.tb * p.os[0] +
-                                    (long long)(sg.qoff + i) * p.os[1] + hq * p.os[2];
-        constexpr int PER = D / 32;
+    if (live) {
+        const int i = (int)(row % lq_pad);
+        const long long bh = row / lq_pad;  // b * Hq + hq
+        const int hq = (int)(bh % p.Hq), b = (int)(bh / p.Hq);
+        const SeqGeom sg = seq_geom(p, b);
+        if (i < sg.Lq) {
+            const long long off = sg.tb * p.os[0] + (long long)(sg.qoff + i) * p.os[1] + hq * p.os[2] + piece * 8;
+            const uint4 ov = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(p.o) + off);
+            const uint4 dv = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(p.dout) + off);
+            const uint32_t oa[4] = {ov.x, ov.y, ov.z, ov.w}, da[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
-        for (int x = 0; x < PER; x += 2) {
-            const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(o + lane * PER + x);
-            const __nv_bfloat162 c = *reinterpret_cast<const __nv_bfloat162 *>(dout + lane * PER + x);
-            s += __bfloat162float(a.x) * __bfloat162float(c.x) + __bfloat162float(a.y) * __bfloat162float(c.y);
+            for (int e = 0; e < 4; ++e) {
+                const float2 of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&oa[e]));
+                const float2 df = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&da[e]));
+                s += of.x * df.x + of.y * df.y;
+            }
+            const float lv = p.lse_in[((long long)sg.tb * p.Hq + hq) * p.lse_ld + sg.qoff + i];
+            nl = lv == -CUDART_INF_F ? -CUDART_INF_F : -lv * 1.4426950408889634f;
         }
-        const float lv = p.lse_in[((long long)sg.tb * p.Hq + hq) * p.lse_ld + sg.qoff + i];
-        nl = lv == -CUDART_INF_F ? -CUDART_INF_F : -lv * 1.4426950408889634f;
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) lsd[row] = make_float2(nl, nl == -CUDART_INF_F ? 0.f : -s);
+    for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (live && piece == 0) lsd[row] = make_float2(nl, nl == -CUDART_INF_F ? 0.f : -s);
 }
 
 // bitmask of bit positions [lo, hi] within 0..31 (empty when lo > hi)
@@ -751,9 +754,10 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, c
         configured[dev & 63] = true;
     }
     const long long rows = (long long)p.B * p.Hq * lq_pad;
+    constexpr int PREP_ROWS = 8 * (32 / (D / 8));  // rows per 256-thread block
     if (rows > 0) {
         launch_begin("bwd_prep", st);
-        bwd_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p, lsd, lq_pad);
+        bwd_prep_kernel<D><<<(unsigned)((rows + PREP_ROWS - 1) / PREP_ROWS), 256, 0, st>>>(p, lsd, lq_pad);
         launch_end(st);
     }
     cudaError_t e = cudaGetLastError();
