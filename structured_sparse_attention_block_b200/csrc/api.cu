@@ -408,11 +408,14 @@ int cowa_fwd(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const
     const int BN = tc ? cowa::fwd5_bn((int)s->d) : cowa::kFwdBN;
     p.nqt = (int)cdiv(s->Lq, cowa::kFwdBM);
     p.nkt = (int)cdiv(s->Lk, BN);
-    int *sched = (int *)ws;
-    p.sched = sched;
-    cudaError_t e = cowa::launch_schedule(sched, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W,
-                                          cowa::kFwdBM, BN, 0, st);
-    if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+    cudaError_t e;
+    if (!tc) {  // the warp-level kernel reads a schedule; the tcgen05 one forms its own ranges
+        int *sched = (int *)ws;
+        p.sched = sched;
+        e = cowa::launch_schedule(sched, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W, cowa::kFwdBM,
+                                  BN, 0, st);
+        if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+    }
     e = tc ? cowa::launch_fwd_sm100(p, (int)s->d, st) : cowa::launch_fwd_mma(p, (int)s->d, st);
     if (e == cudaErrorInvalidValue && tc) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
     if (e != cudaSuccess) return cuda_fail(e, "forward launch");
@@ -453,14 +456,8 @@ int cowa_bwd(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const
     cudaError_t e;
     if (s->Lq > 0 && s->Lk > 0) {
         // tensor-core path: dK/dV over key tiles of 128, dQ over query tiles of 128
-        const int kv_bm = cowa::bwd5_kv_bm(D), dq_bn = cowa::bwd5_dq_bn(D);
+        // (the tcgen05 kernels form their tile ranges themselves: no schedule)
         const int nqt = (int)cdiv(s->Lq, cowa::kBwd5QTile), nkt = (int)cdiv(s->Lk, cowa::kBwd5KeyTile);
-        e = cowa::launch_schedule(sched_q, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W,
-                                  cowa::kBwd5QTile, dq_bn, 0, st);
-        if (e == cudaSuccess)
-            e = cowa::launch_schedule(sched_t, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W, kv_bm,
-                                      cowa::kBwd5KeyTile, 1, st);
-        if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
         e = cowa::launch_bwd_sm100(p, D, (float2 *)rows_ws, (int)cowa::bwd5_lq_pad(s->Lq), sched_q, nqt, sched_t,
                                    nkt, st);
         if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
@@ -697,14 +694,13 @@ static void fill_varlen(cowa::AttnParams &p, const cowa_varlen_shape_t *s, cowa_
 size_t cowa_fwd_varlen_workspace_size(const cowa_varlen_shape_t *s, cowa_quad_t q)
 {
     if (check_varlen(s, q)) return 0;
-    return sched_bytes(s->B * s->Hkv, cdiv(s->max_q, cowa::kFwd5BM)) + 256;
+    return 256;  // the kernels form their tile ranges themselves
 }
 
 size_t cowa_bwd_varlen_workspace_size(const cowa_varlen_shape_t *s, cowa_quad_t q)
 {
     if (check_varlen(s, q)) return 0;
-    return align256((size_t)(s->B * s->Hq * cowa::bwd5_lq_pad(s->max_q)) * sizeof(float2)) +
-           sched_bytes(s->B * s->Hkv, cdiv(s->max_q, 64)) + sched_bytes(s->B * s->Hkv, cdiv(s->max_k, 64)) + 256;
+    return align256((size_t)(s->B * s->Hq * cowa::bwd5_lq_pad(s->max_q)) * sizeof(float2)) + 256;
 }
 
 int cowa_fwd_varlen(const cowa_varlen_shape_t *s, cowa_quad_t quad, float softmax_scale, const int32_t *cu_q,
@@ -732,12 +728,7 @@ int cowa_fwd_varlen(const cowa_varlen_shape_t *s, cowa_quad_t quad, float softma
     const int BN = cowa::fwd5_bn((int)s->d);
     p.nqt = (int)cdiv(s->max_q, cowa::kFwd5BM);
     p.nkt = (int)cdiv(s->max_k, BN);
-    p.sched = (int *)ws;
-    p.sched_bs = (long long)p.Hkv * p.nqt * cowa::kSchedInts;
-    cudaError_t e = cowa::launch_schedule((int *)ws, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W,
-                                          cowa::kFwd5BM, BN, 0, st, cu_q, cu_k, p.B, p.total_q, p.total_k, p.err);
-    if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
-    e = cowa::launch_fwd_sm100(p, (int)s->d, st);
+    cudaError_t e = cowa::launch_fwd_sm100(p, (int)s->d, st);
     if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
     if (e != cudaSuccess) return cuda_fail(e, "forward launch");
     return COWA_OK;
@@ -767,26 +758,11 @@ int cowa_bwd_varlen(const cowa_varlen_shape_t *s, cowa_quad_t quad, float softma
     fill_varlen(p, s, quad, softmax_scale, cu_q, cu_k);
     p.q = q; p.k = k; p.v = v; p.o = (void *)o; p.lse_in = lse; p.dout = dout;
     p.dq = dq; p.dk = dk; p.dv = dv;
-    char *w = (char *)ws;
-    char *rows_ws = w;
+    char *rows_ws = (char *)ws;
     const long long lq_pad = cowa::bwd5_lq_pad(s->max_q);
-    w += align256((size_t)(s->B * s->Hq * lq_pad) * sizeof(float2));
-    int *sched_q = (int *)w;
-    w += sched_bytes(s->B * s->Hkv, cdiv(s->max_q, 64));
-    int *sched_t = (int *)w;
     const int D = (int)s->d;
-    const int kv_bm = cowa::bwd5_kv_bm(D), dq_bn = cowa::bwd5_dq_bn(D);
     const int nqt = (int)cdiv(s->max_q, cowa::kBwd5QTile), nkt = (int)cdiv(s->max_k, cowa::kBwd5KeyTile);
-    p.sched_bs = (long long)p.Hkv * nqt * cowa::kSchedInts;
-    p.sched_t_bs = (long long)p.Hkv * nkt * cowa::kSchedInts;
-    cudaError_t e = cowa::launch_schedule(sched_q, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W,
-                                          cowa::kBwd5QTile, dq_bn, 0, st, cu_q, cu_k, p.B, p.total_q, p.total_k,
-                                          p.err);
-    if (e == cudaSuccess)
-        e = cowa::launch_schedule(sched_t, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W, kv_bm,
-                                  cowa::kBwd5KeyTile, 1, st, cu_q, cu_k, p.B, p.total_q, p.total_k, p.err);
-    if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
-    e = cowa::launch_bwd_sm100(p, D, (float2 *)rows_ws, (int)lq_pad, sched_q, nqt, sched_t, nkt, st);
+    cudaError_t e = cowa::launch_bwd_sm100(p, D, (float2 *)rows_ws, (int)lq_pad, nullptr, nqt, nullptr, nkt, st);
     if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return COWA_OK;

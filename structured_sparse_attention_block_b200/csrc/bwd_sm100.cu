@@ -156,11 +156,12 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
     const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
     const int delta_pos = sg.Lk - sg.Lq;
 
-    const int4 *e4 = reinterpret_cast<const int4 *>(p.sched_t + b * p.sched_t_bs + ((size_t)hl * p.nkt + kt) * kSchedInts);
-    const int4 e0 = e4[0], e1 = e4[1];
-    const int nr = e0.x;
-    const int lo0 = e0.y, lo1 = e0.w, lo2 = e1.y;
-    const int len0 = e0.z - e0.y, len1 = e1.x - e0.w, len2 = e1.z - e1.y;
+    // the query tiles that see this key tile, from the same closed form as
+    // the schedule builder
+    const TileRanges tr = key_tile_ranges(c0, min(c0 + BN, sg.Lk) - 1, sg.Lq, sg.Lk, w, BM);
+    const int nr = tr.n;
+    const int lo0 = tr.lo0, lo1 = tr.lo1, lo2 = tr.lo2;
+    const int len0 = tr.len0, len1 = tr.len1, len2 = tr.len2;
     const int nq = (nr > 0 ? len0 : 0) + (nr > 1 ? len1 : 0) + (nr > 2 ? len2 : 0);
     const int ntask = nq * p.g;
     auto task = [&](int u, int &hq, int &qt) {
@@ -491,11 +492,12 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
     const int nrows = min(BM, sg.Lq - i0);
     const int pa = i0 + delta_pos, pb = i0 + nrows - 1 + delta_pos;
 
-    const int4 *e4 = reinterpret_cast<const int4 *>(p.sched + b * p.sched_bs + ((size_t)hl * p.nqt + qt) * kSchedInts);
-    const int4 e0 = e4[0], e1 = e4[1];
-    const int nr = e0.x;
-    const int lo0 = e0.y, lo1 = e0.w, lo2 = e1.y;
-    const int len0 = e0.z - e0.y, len1 = e1.x - e0.w, len2 = e1.z - e1.y;
+    // the key tiles this query tile visits, from the same closed form as the
+    // schedule builder
+    const TileRanges tr = query_tile_ranges(pa, pb, w, BN);
+    const int nr = tr.n;
+    const int lo0 = tr.lo0, lo1 = tr.lo1, lo2 = tr.lo2;
+    const int len0 = tr.len0, len1 = tr.len1, len2 = tr.len2;
     const int ntiles = (nr > 0 ? len0 : 0) + (nr > 1 ? len1 : 0) + (nr > 2 ? len2 : 0);
     auto tile_of = [&](int t) {
         if (t < len0 || nr == 1) return lo0 + t;

@@ -70,63 +70,119 @@ __host__ __device__ inline void merge_ranges(Ranges &r)
     r.n = m;
 }
 
-__host__ __device__ __forceinline__ void push_keys(Ranges &r, int a, int b, int BN)
-{
-    // key interval [a, b] inclusive -> tile range
-    if (a <= b) {
-        r.lo[r.n] = a / BN;
-        r.hi[r.n] = b / BN + 1;
-        ++r.n;
-    }
-}
-
 // Key tiles visited by a query tile whose in-range rows have aligned
 // positions pa..pb: the union over rows of the sink, near and long key
 // intervals, each contiguous, so every listed tile holds a visible pair.
-__host__ __device__ inline Ranges query_tile_ranges(int pa, int pb, const Win &w, int BN)
+// The ranges as the tile loops read them: n, then three [lo, lo + len)
+// ranges, ascending and disjoint, with the unused ones zero.
+struct TileRanges {
+    int n, lo0, len0, lo1, len1, lo2, len2;
+};
+
+// Sort three half-open ranges (hi <= lo: absent) and merge those that overlap
+// or touch, in scalars only (a runtime-indexed array would live in local
+// memory on the device).
+__host__ __device__ inline TileRanges merge3(int l0, int h0, int l1, int h1, int l2, int h2)
 {
-    Ranges r;
-    r.n = 0;
-    if (pb < 0) return r;
-    const int pa0 = pa > 0 ? pa : 0;
-    if (w.S > 0) push_keys(r, 0, w.S - 1 < pb ? w.S - 1 : pb, BN);
-    if (w.N > 0) push_keys(r, pa0 - w.N + 1 > 0 ? pa0 - w.N + 1 : 0, pb, BN);
-    if (w.e > w.c && pb - w.c >= 0) {
-        const int a = pa0 - (w.e - 1);
-        push_keys(r, a > 0 ? a : 0, pb - w.c, BN);
+    const int none = 0x7fffffff;
+    if (h0 <= l0) l0 = h0 = none;
+    if (h1 <= l1) l1 = h1 = none;
+    if (h2 <= l2) l2 = h2 = none;
+    auto cswap = [](int &la, int &ha, int &lb, int &hb) {
+        if (lb < la) {
+            const int tl = la, th = ha;
+            la = lb;
+            ha = hb;
+            lb = tl;
+            hb = th;
+        }
+    };
+    cswap(l0, h0, l1, h1);
+    cswap(l1, h1, l2, h2);
+    cswap(l0, h0, l1, h1);
+    TileRanges t{0, 0, 0, 0, 0, 0, 0};
+    if (l0 == none) return t;
+    int cl = l0, ch = h0;
+    auto emit = [&](int lo, int hi) {
+        if (t.n == 0) {
+            t.lo0 = lo;
+            t.len0 = hi - lo;
+        } else if (t.n == 1) {
+            t.lo1 = lo;
+            t.len1 = hi - lo;
+        } else {
+            t.lo2 = lo;
+            t.len2 = hi - lo;
+        }
+        ++t.n;
+    };
+    if (l1 != none) {
+        if (l1 <= ch) {
+            ch = h1 > ch ? h1 : ch;
+        } else {
+            emit(cl, ch);
+            cl = l1;
+            ch = h1;
+        }
     }
-    merge_ranges(r);
-    return r;
+    if (l2 != none) {
+        if (l2 <= ch) {
+            ch = h2 > ch ? h2 : ch;
+        } else {
+            emit(cl, ch);
+            cl = l2;
+            ch = h2;
+        }
+    }
+    emit(cl, ch);
+    return t;
 }
 
-__host__ __device__ __forceinline__ void push_rows(Ranges &r, long long lo, long long hi,
-                                                   long long pmin, long long pmax,
-                                                   long long delta, int BM)
+// Key tiles (of BN) a query tile with aligned positions [pa, pb] visits:
+// sink [0, S-1], near [pa-N+1, pb], long [pa-e+1, pb-c], clipped at 0.
+__host__ __device__ inline TileRanges query_tile_ranges(int pa, int pb, const Win &w, int BN)
 {
-    // aligned-position interval [lo, hi] -> query tile range
-    if (lo < pmin) lo = pmin;
-    if (hi > pmax) hi = pmax;
-    if (lo <= hi) {
-        r.lo[r.n] = (int)((lo - delta) / BM);
-        r.hi[r.n] = (int)((hi - delta) / BM) + 1;
-        ++r.n;
+    int l0 = 0, h0 = 0, l1 = 0, h1 = 0, l2 = 0, h2 = 0;
+    if (pb >= 0) {
+        const int pa0 = pa > 0 ? pa : 0;
+        if (w.S > 0) {
+            l0 = 0;
+            h0 = (w.S - 1 < pb ? w.S - 1 : pb) / BN + 1;
+        }
+        if (w.N > 0) {
+            const int a = pa0 - w.N + 1 > 0 ? pa0 - w.N + 1 : 0;
+            l1 = a / BN;
+            h1 = pb / BN + 1;
+        }
+        if (w.e > w.c && pb - w.c >= 0) {
+            const int a = pa0 - (w.e - 1) > 0 ? pa0 - (w.e - 1) : 0;
+            l2 = a / BN;
+            h2 = (pb - w.c) / BN + 1;
+        }
     }
+    return merge3(l0, h0, l1, h1, l2, h2);
 }
 
-// Query tiles that see key tile [c0, c1] (c1 clipped to Lk-1).  Rows sit at
-// p = i + delta with delta = Lk - Lq; valid p is [max(delta, 0), Lk-1].
-__host__ __device__ inline Ranges key_tile_ranges(int c0, int c1, int Lq, int Lk,
-                                                  const Win &w, int BM)
+// Query tiles (of BM) whose rows see some key of [c0, c1]: aligned
+// positions sink [c0, Lk-1] (keys < S), near [c0, c1+N-1], long
+// [c0+c, c1+e-1], within the rows' positions [max(Lk-Lq, 0), Lk-1].
+__host__ __device__ inline TileRanges key_tile_ranges(int c0, int c1, int Lq, int Lk, const Win &w, int BM)
 {
-    Ranges r;
-    r.n = 0;
     const long long delta = (long long)Lk - Lq;
     const long long pmin = delta > 0 ? delta : 0, pmax = (long long)Lk - 1;
-    if (c0 < w.S) push_rows(r, c0, pmax, pmin, pmax, delta, BM);
-    if (w.N > 0) push_rows(r, c0, (long long)c1 + w.N - 1, pmin, pmax, delta, BM);
-    if (w.e > w.c) push_rows(r, (long long)c0 + w.c, (long long)c1 + w.e - 1, pmin, pmax, delta, BM);
-    merge_ranges(r);
-    return r;
+    auto rows = [&](long long a, long long b, int &l, int &h) {
+        if (a < pmin) a = pmin;
+        if (b > pmax) b = pmax;
+        if (a <= b) {
+            l = (int)((a - delta) / BM);
+            h = (int)((b - delta) / BM) + 1;
+        }
+    };
+    int l0 = 0, h0 = 0, l1 = 0, h1 = 0, l2 = 0, h2 = 0;
+    if (c0 < w.S) rows(c0, pmax, l0, h0);
+    if (w.N > 0) rows(c0, (long long)c1 + w.N - 1, l1, h1);
+    if (w.e > w.c) rows((long long)c0 + w.c, (long long)c1 + w.e - 1, l2, h2);
+    return merge3(l0, h0, l1, h1, l2, h2);
 }
 
 // True when every pair of the tile (rows pa..pb, all in range; columns

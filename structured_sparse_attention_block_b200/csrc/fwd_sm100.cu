@@ -116,11 +116,12 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
     const int nrows = min(BM, sg.Lq - i0);
     const int pa = i0 + delta, pb = i0 + nrows - 1 + delta;
 
-    const int4 *e4 = reinterpret_cast<const int4 *>(p.sched + b * p.sched_bs + ((size_t)hl * p.nqt + qt) * kSchedInts);
-    const int4 e0 = e4[0], e1 = e4[1];
-    const int nr = e0.x;
-    const int lo0 = e0.y, lo1 = e0.w, lo2 = e1.y;
-    const int len0 = e0.z - e0.y, len1 = e1.x - e0.w, len2 = e1.z - e1.y;
+    // the key tiles this query tile visits (sink, near, long; at most three
+    // merged ranges), from the same closed form as the schedule builder
+    const TileRanges tr = query_tile_ranges(pa, pb, w, BN);
+    const int nr = tr.n;
+    const int lo0 = tr.lo0, lo1 = tr.lo1, lo2 = tr.lo2;
+    const int len0 = tr.len0, len1 = tr.len1, len2 = tr.len2;
     const int ntiles = (nr > 0 ? len0 : 0) + (nr > 1 ? len1 : 0) + (nr > 2 ? len2 : 0);
     auto tile_of = [&](int t) {
         if (t < len0 || nr == 1) return lo0 + t;

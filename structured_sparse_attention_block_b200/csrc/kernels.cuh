@@ -32,7 +32,6 @@ struct AttnParams {
     const int *cu_q, *cu_k;
     int total_q, total_k;
     long long lse_ld;                 // LSE row pitch: Lq, or total_q when packed
-    long long sched_bs, sched_t_bs;   // schedule ints between sequences (0: shared)
 };
 
 // Lengths and row offsets of sequence b, and its batch coordinate (b for a
@@ -105,12 +104,9 @@ void launch_begin(const char *name, cudaStream_t st);
 void launch_end(cudaStream_t st);
 
 // schedule.cu
-// (cu_q, cu_k, nseq, total_q, total_k, err describe a packed batch: one
-// schedule per sequence, Lq / Lk the longest; nullptr for a uniform batch)
 cudaError_t launch_schedule(int *sched, int Hkv, int kv_head_offset, int Lq,
                             int Lk, int S, int N, int G, int W, int BM, int BN, int transposed,
-                            cudaStream_t st, const int *cu_q = nullptr, const int *cu_k = nullptr,
-                            int nseq = 1, int total_q = 0, int total_k = 0, int *err = nullptr);
+                            cudaStream_t st);
 cudaError_t launch_tile_classes(const int *sched, uint8_t *out, int kv_head, int Lq, int Lk,
                                 int S, int N, int G, int W, int BM, int BN, int transposed,
                                 cudaStream_t st);

@@ -8,56 +8,47 @@
 // ranges, merged into at most three disjoint sorted ranges; the key-tile
 // major form (for dK/dV) lists, for every key tile, the query tiles that see
 // it.  Whether a visited tile needs the element mask is decided per tile by
-// tile_full() in the consumers.
+// tile_full() in the consumers.  The tcgen05 kernels evaluate the same closed
+// form per CTA (query_tile_ranges / key_tile_ranges) instead of reading this
+// table; it serves the warp-level kernels of the degenerate shapes and
+// cowa_tile_classes, the schedule as the kernels see it.
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace cowa {
 
 __global__ void schedule_kernel(int *sched, int kv_head_offset, int Lq, int Lk, int S, int N,
-                                int G, int W, int BM, int BN, int transposed, int ntile,
-                                const int *cu_q, const int *cu_k, int total_q, int total_k, int *err)
+                                int G, int W, int BM, int BN, int transposed, int ntile)
 {
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    const int h = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.y;
     if (t >= ntile) return;
-    if (cu_q) {  // sequence b of a packed batch (bounds as in seq_geom)
-        const int qoff = cu_q[b], koff = cu_k[b], lq = cu_q[b + 1] - qoff, lk = cu_k[b + 1] - koff;
-        const bool ok = qoff >= 0 && koff >= 0 && lq >= 0 && lk >= 0 && lq <= Lq && lk <= Lk &&
-                        qoff <= total_q - lq && koff <= total_k - lk;
-        if (!ok && t == 0 && h == 0) atomicExch(err, 7);
-        Lq = ok ? lq : 0;
-        Lk = ok ? lk : 0;
-        sched += (size_t)b * gridDim.y * ntile * kSchedInts;
-    }
     const Win w = make_win(S, N, G, W, (long long)h + kv_head_offset);
-    Ranges r;
-    r.n = 0;
+    TileRanges tr;
     if (!transposed) {
         const int i0 = t * BM;
         const int i1 = (i0 + BM < Lq ? i0 + BM : Lq) - 1;
         const int delta = Lk - Lq;
-        if (i0 < Lq) r = query_tile_ranges(i0 + delta, i1 + delta, w, BN);
+        tr = query_tile_ranges(i0 + delta, i1 + delta, w, BN);
     } else {
         const int c0 = t * BN;
         const int c1 = (c0 + BN < Lk ? c0 + BN : Lk) - 1;
-        if (c0 < Lk) r = key_tile_ranges(c0, c1, Lq, Lk, w, BM);
+        tr = key_tile_ranges(c0, c1, Lq, Lk, w, BM);
     }
     int4 *e = reinterpret_cast<int4 *>(sched + ((size_t)h * ntile + t) * kSchedInts);
-    e[0] = make_int4(r.n, r.n > 0 ? r.lo[0] : 0, r.n > 0 ? r.hi[0] : 0, r.n > 1 ? r.lo[1] : 0);
-    e[1] = make_int4(r.n > 1 ? r.hi[1] : 0, r.n > 2 ? r.lo[2] : 0, r.n > 2 ? r.hi[2] : 0, 0);
+    e[0] = make_int4(tr.n, tr.lo0, tr.lo0 + tr.len0, tr.lo1);
+    e[1] = make_int4(tr.lo1 + tr.len1, tr.lo2, tr.lo2 + tr.len2, 0);
 }
 
 cudaError_t launch_schedule(int *sched, int Hkv, int kv_head_offset, int Lq, int Lk, int S,
-                            int N, int G, int W, int BM, int BN, int transposed, cudaStream_t st,
-                            const int *cu_q, const int *cu_k, int nseq, int total_q, int total_k, int *err)
+                            int N, int G, int W, int BM, int BN, int transposed, cudaStream_t st)
 {
     const int ntile = transposed ? (Lk + BN - 1) / BN : (Lq + BM - 1) / BM;
-    if (ntile == 0 || Hkv == 0 || nseq == 0) return cudaSuccess;
-    dim3 grid((ntile + 127) / 128, Hkv, cu_q ? nseq : 1);
+    if (ntile == 0 || Hkv == 0) return cudaSuccess;
+    dim3 grid((ntile + 127) / 128, Hkv);
     launch_begin("schedule", st);
     schedule_kernel<<<grid, 128, 0, st>>>(sched, kv_head_offset, Lq, Lk, S, N, G, W, BM, BN,
-                                          transposed, ntile, cu_q, cu_k, total_q, total_k, err);
+                                          transposed, ntile);
     launch_end(st);
     return cudaGetLastError();
 }
