@@ -14,7 +14,6 @@
 
 namespace cowa {
 
-constexpr int kMaxRanges = 3;
 constexpr int kSchedInts = 8;  // n, lo0, hi0, lo1, hi1, lo2, hi2, pad
 
 // Per-head window geometry in 32-bit key units; [c, e) is the long window's
@@ -41,33 +40,6 @@ __host__ __device__ __forceinline__ bool visible(int p, int j, const Win &w)
 {
     const int d = p - j;
     return d >= 0 && (j < w.S || d < w.N || (d >= w.c && d < w.e));
-}
-
-struct Ranges {
-    int n;
-    int lo[kMaxRanges], hi[kMaxRanges];
-};
-
-// Sort up to three half-open tile ranges and merge those that overlap or touch.
-__host__ __device__ inline void merge_ranges(Ranges &r)
-{
-    for (int a = 0; a < r.n; ++a)
-        for (int b = a + 1; b < r.n; ++b)
-            if (r.lo[b] < r.lo[a]) {
-                int t = r.lo[a]; r.lo[a] = r.lo[b]; r.lo[b] = t;
-                t = r.hi[a]; r.hi[a] = r.hi[b]; r.hi[b] = t;
-            }
-    int m = 0;
-    for (int a = 0; a < r.n; ++a) {
-        if (m > 0 && r.lo[a] <= r.hi[m - 1]) {
-            if (r.hi[a] > r.hi[m - 1]) r.hi[m - 1] = r.hi[a];
-        } else {
-            r.lo[m] = r.lo[a];
-            r.hi[m] = r.hi[a];
-            ++m;
-        }
-    }
-    r.n = m;
 }
 
 // Key tiles visited by a query tile whose in-range rows have aligned

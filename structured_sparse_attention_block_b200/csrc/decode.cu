@@ -32,82 +32,83 @@ __device__ __forceinline__ float ex2d(float x)
 // interval a query in that range sees lies inside one stored interval (the
 // stored intervals are separated by keys none of the queries sees).
 struct WindowStore {
-    int n;
-    int lo[3], len[3], off[3];
+    TileRanges t;  // stored key intervals, ascending; row offsets 0, len0, len0 + len1
 };
 
 __device__ inline WindowStore window_store(int o, int R, const Win &w)
 {
-    Ranges r;
-    r.n = 0;
+    int l0 = 0, h0 = 0, l1 = 0, h1 = 0, l2 = 0, h2 = 0;
     const long long top = (long long)o + R - 1;  // last query position served
     if (R > 0 && top >= 0) {
-        if (w.S > 0) {
-            r.lo[r.n] = 0;
-            r.hi[r.n] = (int)min((long long)w.S, top + 1);
-            ++r.n;
-        }
+        if (w.S > 0) h0 = (int)min((long long)w.S, top + 1);
         if (w.N > 0) {
-            r.lo[r.n] = (int)max(0ll, (long long)o - w.N + 1);
-            r.hi[r.n] = (int)(top + 1);
-            ++r.n;
+            l1 = (int)max(0ll, (long long)o - w.N + 1);
+            h1 = (int)(top + 1);
         }
         if (w.e > w.c && top - w.c >= 0) {
-            r.lo[r.n] = (int)max(0ll, (long long)o - w.e + 1);
-            r.hi[r.n] = (int)(top - w.c + 1);
-            ++r.n;
+            l2 = (int)max(0ll, (long long)o - w.e + 1);
+            h2 = (int)(top - w.c + 1);
         }
-        merge_ranges(r);
     }
     WindowStore ws;
-    ws.n = r.n;
-    int off = 0;
-    for (int a = 0; a < 3; ++a) {
-        ws.lo[a] = a < r.n ? r.lo[a] : 0;
-        ws.len[a] = a < r.n ? r.hi[a] - r.lo[a] : 0;
-        ws.off[a] = off;
-        off += ws.len[a];
-    }
+    ws.t = merge3(l0, h0, l1, h1, l2, h2);
     return ws;
 }
 
 // stored row of the keys [j, j + n), or -1 unless one stored interval holds them all
 __device__ inline int window_row(const WindowStore &ws, int j, int n)
 {
-    for (int a = 0; a < ws.n; ++a)
-        if (j >= ws.lo[a] && j + n <= ws.lo[a] + ws.len[a]) return ws.off[a] + (j - ws.lo[a]);
+    const TileRanges &t = ws.t;
+    if (t.n > 0 && j >= t.lo0 && j + n <= t.lo0 + t.len0) return j - t.lo0;
+    if (t.n > 1 && j >= t.lo1 && j + n <= t.lo1 + t.len1) return t.len0 + (j - t.lo1);
+    if (t.n > 2 && j >= t.lo2 && j + n <= t.lo2 + t.len2) return t.len0 + t.len1 + (j - t.lo2);
     return -1;
 }
 
+// key of stored row i, or -1 past the stored keys
+__device__ inline int window_key(const WindowStore &ws, int i)
+{
+    const TileRanges &t = ws.t;
+    if (i < 0) return -1;
+    if (i < t.len0) return t.lo0 + i;
+    i -= t.len0;
+    if (i < t.len1) return t.lo1 + i;
+    i -= t.len1;
+    if (i < t.len2) return t.lo2 + i;
+    return -1;
+}
+
+// The keys the query at position p sees (at most three merged intervals, in
+// key units), each with the cache row of its first key and its tile count.
 struct KeySpans {
-    int n;
-    int lo[3], len[3];
-    int row[3];  // cache row of lo[a]: lo[a] itself, or its row in a windowed cache
-    int tiles[3];
-    int total_tiles;
+    TileRanges t;
+    int row0, row1, row2;  // cache row of each interval's first key
+    int tiles0, tiles1, tiles2, total_tiles;
 };
 
 __device__ inline KeySpans decode_spans(int p, const Win &w)
 {
-    KeySpans ks;
-    Ranges r;
-    r.n = 0;
+    int l0 = 0, h0 = 0, l1 = 0, h1 = 0, l2 = 0, h2 = 0;
     if (p >= 0) {
-        // exact key intervals, half-open, kept in key units (BN = 1 below)
-        if (w.S > 0) { r.lo[r.n] = 0; r.hi[r.n] = min(w.S, p + 1); ++r.n; }
-        if (w.N > 0) { r.lo[r.n] = max(0, p - w.N + 1); r.hi[r.n] = p + 1; ++r.n; }
-        if (w.e > w.c && p - w.c >= 0) { r.lo[r.n] = max(0, p - w.e + 1); r.hi[r.n] = p - w.c + 1; ++r.n; }
-        merge_ranges(r);
+        if (w.S > 0) h0 = min(w.S, p + 1);
+        if (w.N > 0) {
+            l1 = max(0, p - w.N + 1);
+            h1 = p + 1;
+        }
+        if (w.e > w.c && p - w.c >= 0) {
+            l2 = max(0, p - w.e + 1);
+            h2 = p - w.c + 1;
+        }
     }
-    ks.n = r.n;
-    ks.total_tiles = 0;
-    for (int a = 0; a < 3; ++a) {
-        ks.lo[a] = a < r.n ? r.lo[a] : 0;
-        ks.len[a] = a < r.n ? r.hi[a] - r.lo[a] : 0;
-        ks.tiles[a] = (ks.len[a] + kDecBN - 1) / kDecBN;
-        ks.total_tiles += ks.tiles[a];
-        ks.row[a] = ks.lo[a];
-    }
+    KeySpans ks;
+    ks.t = merge3(l0, h0, l1, h1, l2, h2);
+    ks.row0 = ks.t.lo0;
+    ks.row1 = ks.t.lo1;
+    ks.row2 = ks.t.lo2;
+    ks.tiles0 = (ks.t.len0 + kDecBN - 1) / kDecBN;
+    ks.tiles1 = (ks.t.len1 + kDecBN - 1) / kDecBN;
+    ks.tiles2 = (ks.t.len2 + kDecBN - 1) / kDecBN;
+    ks.total_tiles = ks.tiles0 + ks.tiles1 + ks.tiles2;
     return ks;
 }
 
@@ -141,10 +142,17 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
     if (p.origin && !bad) {
         const WindowStore wst = window_store(org, p.horizon, w);
         bool held = true;
-        for (int a = 0; a < 3; ++a) {
-            if (ks.len[a] == 0) continue;
-            ks.row[a] = window_row(wst, ks.lo[a], ks.len[a]);
-            held &= ks.row[a] >= 0 && ks.row[a] + ks.len[a] <= p.Lcap;
+        if (ks.t.n > 0) {
+            ks.row0 = window_row(wst, ks.t.lo0, ks.t.len0);
+            held &= ks.row0 >= 0 && ks.row0 + ks.t.len0 <= p.Lcap;
+        }
+        if (ks.t.n > 1) {
+            ks.row1 = window_row(wst, ks.t.lo1, ks.t.len1);
+            held &= ks.row1 >= 0 && ks.row1 + ks.t.len1 <= p.Lcap;
+        }
+        if (ks.t.n > 2) {
+            ks.row2 = window_row(wst, ks.t.lo2, ks.t.len2);
+            held &= ks.row2 >= 0 && ks.row2 + ks.t.len2 <= p.Lcap;
         }
         if (!held) {  // cannot happen for positions in the horizon; read nothing
             if (tid == 0 && split == 0) atomicExch(p.err, 7);
@@ -156,11 +164,21 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
     const int ntiles = t_end - t_begin;
 
     // tile index -> (first key, valid keys)
-    auto tile_at = [&](int t, int &k0, int &nk) {
-        int a = 0;
-        while (a < 2 && t >= ks.tiles[a]) { t -= ks.tiles[a]; ++a; }
-        k0 = ks.row[a] + t * BN;  // cache row of the tile's first key
-        nk = min(BN, ks.len[a] - t * BN);
+    auto tile_at = [&](int t, int &k0, int &nk) {  // cache row of the tile's first key, keys in it
+        if (t < ks.tiles0) {
+            k0 = ks.row0 + t * BN;
+            nk = min(BN, ks.t.len0 - t * BN);
+            return;
+        }
+        t -= ks.tiles0;
+        if (t < ks.tiles1) {
+            k0 = ks.row1 + t * BN;
+            nk = min(BN, ks.t.len1 - t * BN);
+            return;
+        }
+        t -= ks.tiles1;
+        k0 = ks.row2 + t * BN;
+        nk = min(BN, ks.t.len2 - t * BN);
     };
 
     const __nv_bfloat16 *kg = reinterpret_cast<const __nv_bfloat16 *>(p.kc) + b * p.ks[0] + hl * p.ks[2];
@@ -352,8 +370,7 @@ __global__ void __launch_bounds__(128) wcache_build_kernel(const WCacheParams p)
     int j = -1;
     if (o >= 0 && o < p.Lsrc) {
         const WindowStore ws = window_store(o, p.horizon, make_win(p.S, p.N, p.G, p.W, (long long)h + p.kv_head_offset));
-        for (int a = 0; a < ws.n; ++a)
-            if (i >= ws.off[a] && i < ws.off[a] + ws.len[a]) j = ws.lo[a] + (i - ws.off[a]);
+        j = window_key(ws, i);
         if (j > o) j = -1;  // a future key: appended later
     } else if (i == 0 && c == 0 && h == 0) {
         atomicExch(p.err, 7);
