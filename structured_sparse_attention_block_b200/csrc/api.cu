@@ -359,7 +359,7 @@ cowa_quad_t cowa_default_quad(int64_t Lk, int64_t Hkv, int32_t S, int32_t N)
 size_t cowa_fwd_workspace_size(const cowa_shape_t *s, cowa_quad_t q)
 {
     if (check_shape(s, q, false)) return 0;
-    return sched_bytes(s->Hkv, cdiv(s->Lq, cowa::kFwdBM)) + 256;
+    return sched_bytes(s->Hkv, cdiv(s->Lq, cowa::kFwd5BM)) + 256;
 }
 
 size_t cowa_bwd_workspace_size(const cowa_shape_t *s, cowa_quad_t q)
@@ -402,22 +402,17 @@ int cowa_fwd(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const
     p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
     p.B = (int)s->B; p.Lq = (int)s->Lq; p.Lk = (int)s->Lk;
     p.lse_ld = s->Lq;
-    // tensor-core path (TMA + tcgen05); with no keys at all there is nothing
-    // to map, and the warp-level kernel writes the empty rows
-    const bool tc = s->Lk > 0;
-    const int BN = tc ? cowa::fwd5_bn((int)s->d) : cowa::kFwdBN;
-    p.nqt = (int)cdiv(s->Lq, cowa::kFwdBM);
-    p.nkt = (int)cdiv(s->Lk, BN);
-    cudaError_t e;
-    if (!tc) {  // the warp-level kernel reads a schedule; the tcgen05 one forms its own ranges
-        int *sched = (int *)ws;
-        p.sched = sched;
-        e = cowa::launch_schedule(sched, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W, cowa::kFwdBM,
-                                  BN, 0, st);
-        if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+    if (s->Lk == 0) {
+        // no keys at all: every row sees nothing (O = 0, LSE = -inf)
+        cudaError_t e = cowa::launch_zero_rows(o, p.os, p.B, p.Lq, p.Hq, (int)s->d, st);
+        if (e == cudaSuccess) e = cowa::launch_fill_f32(lse, s->B * s->Hq * s->Lq, -INFINITY, st);
+        return e == cudaSuccess ? COWA_OK : cuda_fail(e, "constant output launch");
     }
-    e = tc ? cowa::launch_fwd_sm100(p, (int)s->d, st) : cowa::launch_fwd_mma(p, (int)s->d, st);
-    if (e == cudaErrorInvalidValue && tc) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
+    const int BN = cowa::fwd5_bn((int)s->d);
+    p.nqt = (int)cdiv(s->Lq, cowa::kFwd5BM);
+    p.nkt = (int)cdiv(s->Lk, BN);
+    cudaError_t e = cowa::launch_fwd_sm100(p, (int)s->d, st);
+    if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
     if (e != cudaSuccess) return cuda_fail(e, "forward launch");
     return COWA_OK;
 }
@@ -446,39 +441,23 @@ int cowa_bwd(const cowa_shape_t *s, cowa_quad_t quad, float softmax_scale, const
     p.dq = dq; p.dk = dk; p.dv = dv;
     p.B = (int)s->B; p.Lq = (int)s->Lq; p.Lk = (int)s->Lk;
     p.lse_ld = s->Lq;
-    char *w = (char *)ws;
-    char *rows_ws = w;
-    w += align256((size_t)(s->B * s->Hq * cowa::bwd5_lq_pad(s->Lq)) * sizeof(float2));
-    int *sched_q = (int *)w;
-    w += sched_bytes(s->Hkv, cdiv(s->Lq, 64));
-    int *sched_t = (int *)w;
+    char *rows_ws = (char *)ws;
     const int D = (int)s->d;
     cudaError_t e;
     if (s->Lq > 0 && s->Lk > 0) {
         // tensor-core path: dK/dV over key tiles of 128, dQ over query tiles of 128
         // (the tcgen05 kernels form their tile ranges themselves: no schedule)
         const int nqt = (int)cdiv(s->Lq, cowa::kBwd5QTile), nkt = (int)cdiv(s->Lk, cowa::kBwd5KeyTile);
-        e = cowa::launch_bwd_sm100(p, D, (float2 *)rows_ws, (int)cowa::bwd5_lq_pad(s->Lq), sched_q, nqt, sched_t,
-                                   nkt, st);
+        e = cowa::launch_bwd_sm100(p, D, (float2 *)rows_ws, (int)cowa::bwd5_lq_pad(s->Lq), nqt, nkt, st);
         if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
         if (e != cudaSuccess) return cuda_fail(e, "backward launch");
         return COWA_OK;
     }
-    // no queries or no keys: the warp-level kernels write the zero gradients
-    const int QB = cowa::bwd_kv_qtile(D);
-    p.nqt = (int)cdiv(s->Lq, cowa::kBwdBM);
-    p.nkt = (int)cdiv(s->Lk, cowa::kBwdBN);
-    p.delta = (float *)rows_ws;
-    p.sched = sched_q;
-    p.sched_t = sched_t;
-    e = cowa::launch_schedule(sched_q, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W, cowa::kBwdBM,
-                              cowa::kBwdBN, 0, st);
-    if (e == cudaSuccess)
-        e = cowa::launch_schedule(sched_t, p.Hkv, p.kv_head_offset, p.Lq, p.Lk, p.S, p.N, p.G, p.W, QB,
-                                  cowa::kBwdBN, 1, st);
-    if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
-    e = cowa::launch_bwd_mma(p, D, st);
-    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    // no queries or no keys: every gradient is zero
+    e = qrows ? cowa::launch_zero_rows(dq, p.qs, p.B, p.Lq, p.Hq, D, st) : cudaSuccess;
+    if (e == cudaSuccess && krows) e = cowa::launch_zero_rows(dk, p.ks, p.B, p.Lk, p.Hkv, D, st);
+    if (e == cudaSuccess && krows) e = cowa::launch_zero_rows(dv, p.vs, p.B, p.Lk, p.Hkv, D, st);
+    if (e != cudaSuccess) return cuda_fail(e, "constant gradient launch");
     return COWA_OK;
 }
 
@@ -762,7 +741,7 @@ int cowa_bwd_varlen(const cowa_varlen_shape_t *s, cowa_quad_t quad, float softma
     const long long lq_pad = cowa::bwd5_lq_pad(s->max_q);
     const int D = (int)s->d;
     const int nqt = (int)cdiv(s->max_q, cowa::kBwd5QTile), nkt = (int)cdiv(s->max_k, cowa::kBwd5KeyTile);
-    cudaError_t e = cowa::launch_bwd_sm100(p, D, (float2 *)rows_ws, (int)lq_pad, nullptr, nqt, nullptr, nkt, st);
+    cudaError_t e = cowa::launch_bwd_sm100(p, D, (float2 *)rows_ws, (int)lq_pad, nqt, nkt, st);
     if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return COWA_OK;

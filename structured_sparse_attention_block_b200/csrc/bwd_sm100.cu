@@ -740,8 +740,8 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
 
 // ----------------------------------------------------------------- host ----
 template <int D>
-static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, const int *sched_dq, int nqt_dq,
-                                 const int *sched_kv, int nkt_kv, cudaStream_t st)
+static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, int nqt_dq, int nkt_kv,
+                                 cudaStream_t st)
 {
     using K = KvCfg<D>;
     using Q = DqCfg<D>;
@@ -779,7 +779,6 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, c
         !make_bshd_map(&a.tk, p.k, D, Lk_map, p.Hkv, B_map, p.ks, K::BN) ||
         !make_bshd_map(&a.tv, p.v, D, Lk_map, p.Hkv, B_map, p.vs, K::BN))
         return cudaErrorInvalidValue;
-    a.p.sched_t = sched_kv;
     a.p.nkt = nkt_kv;
     if (nkt_kv > 0) {
         const unsigned g1 = tile_grid_blocks(nkt_kv, p.Hkv, p.B);
@@ -796,7 +795,6 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, c
         !make_bshd_map(&a.tk, p.k, D, Lk_map, p.Hkv, B_map, p.ks, Q::BN) ||
         !make_bshd_map(&a.tv, p.v, D, Lk_map, p.Hkv, B_map, p.vs, Q::BN))
         return cudaErrorInvalidValue;
-    a.p.sched = sched_dq;
     a.p.nqt = nqt_dq;
     a.npair = (p.g + Q::NSLOT - 1) / Q::NSLOT;
     if (nqt_dq > 0) {
@@ -810,12 +808,12 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, c
     return e;
 }
 
-cudaError_t launch_bwd_sm100(const AttnParams &p, int D, float2 *lsd, int lq_pad, const int *sched_dq, int nqt_dq,
-                             const int *sched_kv, int nkt_kv, cudaStream_t st)
+cudaError_t launch_bwd_sm100(const AttnParams &p, int D, float2 *lsd, int lq_pad, int nqt_dq, int nkt_kv,
+                             cudaStream_t st)
 {
     if (p.B == 0 || p.Hq == 0) return cudaSuccess;
-    return D == 128 ? launch_bwd5_d<128>(p, lsd, lq_pad, sched_dq, nqt_dq, sched_kv, nkt_kv, st)
-                    : launch_bwd5_d<64>(p, lsd, lq_pad, sched_dq, nqt_dq, sched_kv, nkt_kv, st);
+    return D == 128 ? launch_bwd5_d<128>(p, lsd, lq_pad, nqt_dq, nkt_kv, st)
+                    : launch_bwd5_d<64>(p, lsd, lq_pad, nqt_dq, nkt_kv, st);
 }
 
 }  // namespace cowa

@@ -15,14 +15,11 @@ struct AttnParams {
     const void *dout;
     const float *lse_in;
     void *dq, *dk, *dv;
-    float *delta;
-    const int *sched;       // query-tile-major schedule [Hkv][nqt][8]
-    const int *sched_t;     // key-tile-major schedule [Hkv][nkt][8]
     long long qs[3], ks[3], vs[3], os[3];
     int B, Lq, Lk, Hq, Hkv, g;
     int S, N, G, W;
     int kv_head_offset;
-    int nqt, nkt;           // tiles of the schedule in use
+    int nqt, nkt;           // query / key tiles of the launch
     float scale, scale_log2;
     int *err;               // device error word (status code of a failed device check)
     // Packed (variable-length) batch: sequence b owns query rows
@@ -111,9 +108,6 @@ cudaError_t launch_tile_classes(const int *sched, uint8_t *out, int kv_head, int
                                 int S, int N, int G, int W, int BM, int BN, int transposed,
                                 cudaStream_t st);
 
-// fwd_mma.cu (warp-level MMA forward; used when there are no keys to map)
-cudaError_t launch_fwd_mma(const AttnParams &p, int D, cudaStream_t st);
-constexpr int kFwdBM = 128, kFwdBN = 64;
 
 // fwd_sm100.cu (tcgen05 forward)
 cudaError_t launch_fwd_sm100(const AttnParams &p, int D, cudaStream_t st);
@@ -125,14 +119,15 @@ __host__ __device__ constexpr int fwd5_bn(int D) { return D == 128 ? 64 : 96; }
 bool make_bshd_map(CUtensorMap *m, const void *base, int d, long long L, long long H, long long B,
                    const long long st[3], int rows);
 
-// bwd_mma.cu
-cudaError_t launch_bwd_mma(const AttnParams &p, int D, cudaStream_t st);
-constexpr int kBwdBM = 64, kBwdBN = 64;
-inline int bwd_kv_qtile(int D) { return D == 128 ? 32 : 64; }
+// fill.cu: constant outputs of the shapes the tcgen05 kernels do not take
+// (zero rows of a strided [B, L, H, D] bf16 tensor; a constant fp32 array)
+cudaError_t launch_zero_rows(void *t, const long long st[3], int B, int L, int H, int D, cudaStream_t s);
+cudaError_t launch_fill_f32(float *p, long long n, float v, cudaStream_t s);
+
 
 // bwd_sm100.cu (tcgen05 backward: preprocess, dK/dV pass, dQ pass)
-cudaError_t launch_bwd_sm100(const AttnParams &p, int D, float2 *lsd, int lq_pad, const int *sched_dq,
-                             int nqt_dq, const int *sched_kv, int nkt_kv, cudaStream_t st);
+cudaError_t launch_bwd_sm100(const AttnParams &p, int D, float2 *lsd, int lq_pad, int nqt_dq, int nkt_kv,
+                             cudaStream_t st);
 constexpr int kBwd5KeyTile = 128;   // keys per dK/dV CTA (tensor-memory lanes)
 constexpr int kBwd5QTile = 128;     // queries per dQ CTA
 __host__ __device__ constexpr int bwd5_kv_bm(int D) { return D == 128 ? 32 : 64; }    // queries per dK/dV task

@@ -97,3 +97,20 @@ def test_bwd_workloads_sampled(oracle_mod, name, per_head, ncols):
     # rounding of dK leaves a residue far below 1% of sum_j |dK_j|
     dkf = dk.float()
     assert (dkf.sum(dim=1).abs() <= 1e-2 * dkf.abs().sum(dim=1) + 1e-6).all()
+
+
+@pytest.mark.parametrize("Lq,Lk", [(0, 200), (150, 0)])
+def test_no_queries_or_no_keys_gives_zero_gradients(Lq, Lk):
+    import structured_sparse_attention_block_b200 as cowa
+    B, Hq, Hkv, d = 2, 4, 2, 128
+    q = torch.randn(B, Lq, Hq, d, device="cuda").to(torch.bfloat16)
+    k = torch.randn(B, Lk, Hkv, d, device="cuda").to(torch.bfloat16)
+    v = torch.randn(B, Lk, Hkv, d, device="cuda").to(torch.bfloat16)
+    o = torch.randn(B, Lq, Hq, d, device="cuda").to(torch.bfloat16)
+    do = torch.randn(B, Lq, Hq, d, device="cuda").to(torch.bfloat16)
+    lse = torch.full((B, Hq, Lq), float("-inf"), device="cuda")
+    dq = torch.full_like(q, 3.0)
+    dk, dv = torch.full_like(k, 3.0), torch.full_like(v, 3.0)
+    cowa.cowa_bwd(q, k, v, o, lse, do, (4, 16, 0, 8), dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    assert torch.all(dq == 0) and torch.all(dk == 0) and torch.all(dv == 0)

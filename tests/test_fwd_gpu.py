@@ -94,3 +94,15 @@ def test_fwd_workloads_sampled_rows(oracle_mod, name, per_head):
     lse_got = lse[b, hq, i]
     assert_o(o_got, o_ref)
     assert_lse(lse_got, lse_ref)
+
+
+def test_no_keys_gives_empty_rows():
+    # a sequence with no keys at all: every row sees nothing (O = 0, LSE = -inf)
+    import structured_sparse_attention_block_b200 as cowa
+    from structured_sparse_attention_block_b200.inputs import training_inputs
+    q, _, _, _ = training_inputs(2, 130, 1, 4, 2, 64, seed=2)
+    k = torch.empty((2, 0, 2, 64), dtype=torch.bfloat16, device="cuda")
+    o, lse = cowa.cowa_fwd(q, k, k, (4, 16, 0, 8), out=torch.full_like(q, 7.0))
+    torch.cuda.synchronize()
+    assert torch.all(o == 0)
+    assert torch.all(torch.isneginf(lse))
