@@ -228,7 +228,7 @@ size_t sched_bytes(long long heads, long long tiles) { return align256((size_t)(
 // bound and its CTAs all do about the same work, so the time is set by the
 // number of full waves of resident CTAs: pick the smallest split count whose
 // waves-per-unit-of-work is within 3 % of the best, over 1 .. 64 splits and
-// at most one split per key tile.
+// at least four key tiles per split.
 int decode_splits(const cowa_shape_t *s, cowa_quad_t q, int sms)
 {
     const long long pairs = s->B * s->Hkv;
@@ -237,7 +237,9 @@ int decode_splits(const cowa_shape_t *s, cowa_quad_t q, int sms)
     if (keys > s->Lk) keys = s->Lk;
     const long long tiles = cdiv(keys, cowa::kDecBN) + 3;
     const long long resident = (long long)sms * cowa::decode_ctas_per_sm((int)s->d);
-    const long long max_sp = tiles < 64 ? tiles : 64;
+    // at most 64 splits (the merge's limit) and at least four key tiles each
+    long long max_sp = tiles / 4 < 64 ? tiles / 4 : 64;
+    if (max_sp < 1) max_sp = 1;
     double best = 1e30;
     for (long long sp = 1; sp <= max_sp; ++sp) {
         const double v = (double)cdiv(pairs * sp, resident) / (double)sp;

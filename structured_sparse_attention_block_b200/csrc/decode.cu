@@ -335,25 +335,40 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
 }
 
 template <int D>
-__global__ void decode_combine_kernel(const DecodeParams p)
+__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p)
 {
+    // thread s < splits holds split s: the max and the weights are block
+    // reductions, then every thread merges columns with the weights from
+    // shared memory (splits <= 64)
+    __shared__ float red[4], wsum[4], wt[64];
     const int row = blockIdx.x;  // b * Hq + hq
     const int b = row / p.Hq, hq = row % p.Hq;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float *pl = p.part_lse + (long long)row * p.splits;
     const float *po = p.part_o + (long long)row * p.splits * D;
-    float m = -CUDART_INF_F;
-    for (int s = 0; s < p.splits; ++s) m = fmaxf(m, pl[s]);
+    const float lv = tid < p.splits ? pl[tid] : -CUDART_INF_F;
+    float m = lv;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
     const float ms = m == -CUDART_INF_F ? 0.f : m;
-    float lsum = 0.f;
-    for (int s = 0; s < p.splits; ++s) lsum += ex2d(pl[s] - ms);
+    const float wv = tid < p.splits ? ex2d(lv - ms) : 0.f;
+    if (tid < 64) wt[tid] = wv;
+    float l = wv;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    if (lane == 0) wsum[warp] = l;
+    __syncthreads();
+    const float lsum = (wsum[0] + wsum[1]) + (wsum[2] + wsum[3]);
     __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + b * p.os[0] + hq * p.os[2];
-    for (int col = threadIdx.x; col < D; col += blockDim.x) {
+    for (int col = tid; col < D; col += blockDim.x) {
         float acc = 0.f;
-        for (int s = 0; s < p.splits; ++s) acc += ex2d(pl[s] - ms) * po[(long long)s * D + col];
+        for (int sp = 0; sp < p.splits; ++sp) acc += wt[sp] * po[(long long)sp * D + col];
         o[col] = __float2bfloat16_rn(lsum > 0.f ? acc / lsum : 0.f);
     }
-    if (threadIdx.x == 0)
-        p.lse[row] = lsum > 0.f ? (m + __log2f(lsum)) * 0.69314718055994531f : -CUDART_INF_F;
+    if (tid == 0) p.lse[row] = lsum > 0.f ? (m + __log2f(lsum)) * 0.69314718055994531f : -CUDART_INF_F;
 }
 
 // One thread per 16-byte piece of a row: row i of the windowed cache of
