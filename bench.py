@@ -12,13 +12,18 @@ Metric: effective TFLOP/s counted on visible pairs only -- 4*d flops per
 pair forward, 10*d backward, 4*d per visible key and query head in decode --
 over the step time; decode GB/s on visible K+V bytes is reported beside it.
 Timing: CUDA events on the launching stream, L2 flushed (a 512 MiB write)
-before every timed step, max over ranks.  Multi-GPU: every rank runs its own
-batch (data-parallel replicas, no collective on the data path; weak scaling).
+before every timed step, max over ranks.  Multi-GPU, no collective on the
+data path in either mode: by default every rank runs its own batch
+(data-parallel replicas, weak scaling); with ``--parallel heads`` rank r
+takes KV heads [r*Hkv/N, (r+1)*Hkv/N) of the one workload with their query
+heads and passes the first one's global index as kv_head_offset (KV-head
+tensor parallelism, strong scaling).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--parallel dp|heads]
   python bench.py --impl reference ...   # the fp64 CPU oracle, timed on host cores
 """
 import argparse
+import dataclasses
 import datetime
 import json
 import math
@@ -97,6 +102,34 @@ def max_over_ranks(values, world, device):
         import torch.distributed as dist
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return [float(x) for x in t.cpu()]
+
+
+def sum_over_ranks(values, world, device):
+    """Element-wise sum of a list of numbers over all ranks (whole-job work)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.cpu()]
+
+
+def h0_mode(args, world):
+    """True when the run shards KV heads over more than one GPU."""
+    return args.parallel == "heads" and world > 1
+
+
+def head_shard(wl, rank, world, parallel):
+    """The rank's part of a workload and its first global KV head.  Replicas
+    ("dp") run all of it; KV-head sharding ("heads") gives rank r the KV heads
+    [r*Hkv/R, (r+1)*Hkv/R) and their g query heads each (contiguous GQA
+    groups), so its windows stay those of its global heads."""
+    if parallel == "dp" or world == 1:
+        return wl, 0
+    if wl.Hkv % world:
+        raise SystemExit("--parallel heads: %s has %d KV heads, not divisible by %d GPUs"
+                         % (wl.name, wl.Hkv, world))
+    per = wl.Hkv // world
+    return dataclasses.replace(wl, Hq=wl.Hq // world, Hkv=per), rank * per
 
 
 # ----------------------------------------------------------------- clocks ----
@@ -242,9 +275,10 @@ def run_cowa(args, rank, world, local_rank):
     import structured_sparse_attention_block_b200 as cowa
     from structured_sparse_attention_block_b200.inputs import WORKLOADS, training_inputs
 
-    wl = WORKLOADS[args.workload]
-    if wl.kind != "train":
+    wl_job = WORKLOADS[args.workload]
+    if wl_job.kind != "train":
         raise SystemExit("the step workload must be a training workload")
+    wl, h0 = head_shard(wl_job, rank, world, args.parallel)
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
@@ -259,21 +293,21 @@ def run_cowa(args, rank, world, local_rank):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     od = torch.empty_like(qd)
     lsed = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device=dev)
-    ws_f = torch.empty(cowa.cowa_fwd_workspace_size(q, k, quad), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(cowa.cowa_bwd_workspace_size(q, k, quad), dtype=torch.uint8, device=dev)
-    ws_d = torch.empty(cowa.cowa_decode_workspace_size(qd, k, quad), dtype=torch.uint8, device=dev)
+    ws_f = torch.empty(cowa.cowa_fwd_workspace_size(q, k, quad, h0), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(cowa.cowa_bwd_workspace_size(q, k, quad, h0), dtype=torch.uint8, device=dev)
+    ws_d = torch.empty(cowa.cowa_decode_workspace_size(qd, k, quad, h0), dtype=torch.uint8, device=dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        cowa.cowa_fwd(q, k, v, quad, out=o, lse=lse, workspace=ws_f)
+        cowa.cowa_fwd(q, k, v, quad, kv_head_offset=h0, out=o, lse=lse, workspace=ws_f)
         if ev is not None:
             ev[1].record(stream)
-        cowa.cowa_bwd(q, k, v, o, lse, do, quad, dq=dq, dk=dk, dv=dv, workspace=ws_b)
+        cowa.cowa_bwd(q, k, v, o, lse, do, quad, kv_head_offset=h0, dq=dq, dk=dk, dv=dv, workspace=ws_b)
         if ev is not None:
             ev[2].record(stream)
-        cowa.cowa_decode(qd, k, v, seqlens, quad, out=od, lse=lsed, workspace=ws_d)
+        cowa.cowa_decode(qd, k, v, seqlens, quad, kv_head_offset=h0, out=od, lse=lsed, workspace=ws_d)
         if ev is not None:
             ev[3].record(stream)
 
@@ -296,8 +330,8 @@ def run_cowa(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    pairs = visible_pairs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, quad)
-    dec_keys = decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, quad)
+    pairs = visible_pairs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, quad, kv_head_offset=h0)
+    dec_keys = decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, quad, kv_head_offset=h0)
     work = kernel_work(wl, pairs, dec_keys)
     warm = {}
     for name, ms in warm_trace:
@@ -333,18 +367,21 @@ def run_cowa(args, rank, world, local_rank):
     t_step, t_fwd, t_bwd, t_dec = max_over_ranks([t_step, t_fwd, t_bwd, t_dec], world, dev)
 
     g = wl.Hq // wl.Hkv
-    flops_step = pairs * 14 * wl.d + dec_keys * g * 4 * wl.d
-    dec_bytes = dec_keys * 2 * wl.d * 2
-    value = flops_step * world / (t_step * 1e-3) / 1e12
+    # whole-job work: every rank's pairs and decode keys
+    pairs_job, dec_keys_job = (int(x) for x in sum_over_ranks([pairs, dec_keys], world, dev))
+    flops_job = pairs_job * 14 * wl.d + dec_keys_job * g * 4 * wl.d
+    dec_bytes = dec_keys_job * 2 * wl.d * 2
+    value = flops_job / (t_step * 1e-3) / 1e12
 
     # end to end through the public API from pinned host buffers
-    e2e = run_e2e(args, cowa, wl, q, k, v, do, qd, seqlens, quad, dev, stream, flush, world)
-    e2e["value"] = flops_step * world / (e2e.pop("ms") * 1e-3) / 1e12
+    e2e = run_e2e(args, cowa, wl, q, k, v, do, qd, seqlens, quad, h0, dev, stream, flush, world)
+    e2e["value"] = flops_job / (e2e.pop("ms") * 1e-3) / 1e12
     e2e["unit"] = "TFLOP/s"
 
+    # whole-job rates; the fractions are per GPU (job rate / N / peak)
     peaks, peak_src = load_peaks()
-    bwd_tflops = pairs * 10 * wl.d / (t_bwd * 1e-3) / 1e12
-    fwd_tflops = pairs * 4 * wl.d / (t_fwd * 1e-3) / 1e12
+    bwd_tflops = pairs_job * 10 * wl.d / (t_bwd * 1e-3) / 1e12
+    fwd_tflops = pairs_job * 4 * wl.d / (t_fwd * 1e-3) / 1e12
     dec_gbs = dec_bytes / (t_dec * 1e-3) / 1e9
 
     # per-kernel shares from the traced warm-up steps; the roofline kernel's
@@ -356,20 +393,24 @@ def run_cowa(args, rank, world, local_rank):
     for n, a in zip(names, avg):
         kernels[n] = {"launches": warm[n][0], "avg_ms": round(a, 5),
                       "share": round(warm[n][1] / total, 4)}
-        if n in work:
+        if n in work:  # per GPU: rank 0's work over the slowest rank's time
             bound, amount, unit, _ = work[n]
             if bound == "tensor":
                 kernels[n]["tflops"] = round(amount / (a * 1e-3) / 1e12, 2)
             else:
                 kernels[n]["gbs"] = round(amount / (a * 1e-3) / 1e9, 1)
     bound, amount, unit, how = work[top]
-    a_ms = max_over_ranks([sum(ms for _, ms in trace) / len(trace)], world, dev)[0]
+    # per GPU: each rank's own work over its own average launch; the slowest
+    # rank's rate is reported
+    a_local = sum(ms for _, ms in trace) / len(trace)
+    rate = amount / (a_local * 1e-3) / (1e12 if bound == "tensor" else 1e9)
+    a_ms, neg_rate = max_over_ranks([a_local, -rate], world, dev)
     if bound == "tensor":
-        achieved, peak, runit = amount / (a_ms * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        achieved, peak, runit = -neg_rate, peaks["bf16_tflops"], "TFLOP/s"
         psrc = "%s bf16_tflops (burst: the kernel runs %.2f ms inside a %.2f ms step)" % (
             peak_src, a_ms, t_step)
     else:
-        achieved, peak, runit = amount / (a_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        achieved, peak, runit = -neg_rate, peaks["hbm_gbs"], "GB/s"
         psrc = "%s hbm_gbs" % peak_src
     roofline = {
         "kernel": top, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
@@ -383,20 +424,23 @@ def run_cowa(args, rank, world, local_rank):
         "metric": "effective TFLOP/s on visible pairs (fwd/bwd) & decode GB/s, % of B200 roofline",
         "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(t_step, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic N(0,1), seeded",
-        "config": {"workload": wl.name, "B": wl.B, "Lq": wl.Lq, "Lk": wl.Lk, "Hq": wl.Hq,
-                   "Hkv": wl.Hkv, "d": wl.d, "quad": list(quad),
+        "scaling": "strong" if h0_mode(args, world) else "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic N(0,1), seeded",
+        "config": {"workload": wl_job.name, "B": wl_job.B, "Lq": wl_job.Lq, "Lk": wl_job.Lk,
+                   "Hq": wl_job.Hq, "Hkv": wl_job.Hkv, "d": wl_job.d, "quad": list(quad),
                    "step": "cowa_fwd + cowa_bwd + cowa_decode(last token, full K/V as cache)",
                    "l2": "512 MiB write before every timed step",
-                   "parallelism": "dp%d (independent replicas)" % world},
+                   "parallelism": ("kv-heads%d (rank r: KV heads [r*%d, (r+1)*%d), kv_head_offset = r*%d)"
+                                   % (world, wl.Hkv, wl.Hkv, wl.Hkv)) if h0_mode(args, world)
+                   else "dp%d (independent replicas)" % world},
         "breakdown": {
             "fwd_ms": round(t_fwd, 4), "fwd_tflops": round(fwd_tflops, 2),
-            "fwd_frac": round(fwd_tflops / peaks["bf16_tflops"], 4),
+            "fwd_frac": round(fwd_tflops / world / peaks["bf16_tflops"], 4),
             "bwd_ms": round(t_bwd, 4), "bwd_tflops": round(bwd_tflops, 2),
-            "bwd_frac": round(bwd_tflops / peaks["bf16_tflops"], 4),
+            "bwd_frac": round(bwd_tflops / world / peaks["bf16_tflops"], 4),
             "decode_ms": round(t_dec, 4), "decode_gbs": round(dec_gbs, 1),
-            "decode_frac": round(dec_gbs / peaks["hbm_gbs"], 4),
-            "visible_pairs": pairs, "decode_visible_keys": dec_keys,
+            "decode_frac": round(dec_gbs / world / peaks["hbm_gbs"], 4),
+            "visible_pairs": pairs_job, "decode_visible_keys": dec_keys_job,
             "kernels": kernels,
             "kernels_from": "CUDA events around every library launch of the traced warm-up steps",
         },
@@ -406,18 +450,19 @@ def run_cowa(args, rank, world, local_rank):
         "gpu_launches": int(launches),
     }
     if args.packed:
-        result["packed_workload"] = run_packed_workload(args, cowa, wl, dev, stream, flush, world, peaks)
+        result["packed_workload"] = run_packed_workload(args, cowa, wl, h0, dev, stream, flush, world, peaks)
     if args.full_mask:
-        result["full_mask_control"] = run_full_mask(args, cowa, wl, q, k, v, do, qd, seqlens, dev, stream,
+        result["full_mask_control"] = run_full_mask(args, cowa, wl, q, k, v, do, qd, seqlens, h0, dev, stream,
                                                     flush, world, (t_fwd, t_bwd, t_dec))
     if args.decode_workload:
-        result["decode_workload"] = run_decode_workload(args, cowa, dev, stream, flush, world, peaks, peak_src)
+        result["decode_workload"] = run_decode_workload(args, cowa, rank, dev, stream, flush, world, peaks,
+                                                        peak_src)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = run_cpu_baseline(wl, q, k, v, do, quad, args.cpu_rows)
     return result
 
 
-def run_e2e(args, cowa, wl, q, k, v, do, qd, seqlens, quad, dev, stream, flush, world):
+def run_e2e(args, cowa, wl, q, k, v, do, qd, seqlens, quad, h0, dev, stream, flush, world):
     import torch.distributed as dist
     hq, hk, hv, hdo, hqd = (t.cpu().pin_memory() for t in (q, k, v, do, qd))
     hsl = seqlens.cpu().pin_memory()
@@ -432,9 +477,9 @@ def run_e2e(args, cowa, wl, q, k, v, do, qd, seqlens, quad, dev, stream, flush, 
     def e2e_step():
         dq_, dk_, dv_, ddo, dqd = (t.to(dev, non_blocking=True) for t in (hq, hk, hv, hdo, hqd))
         dsl = hsl.to(dev, non_blocking=True)
-        o, lse = cowa.cowa_fwd(dq_, dk_, dv_, quad)
-        g1, g2, g3 = cowa.cowa_bwd(dq_, dk_, dv_, o, lse, ddo, quad)
-        od, _ = cowa.cowa_decode(dqd, dk_, dv_, dsl, quad)
+        o, lse = cowa.cowa_fwd(dq_, dk_, dv_, quad, kv_head_offset=h0)
+        g1, g2, g3 = cowa.cowa_bwd(dq_, dk_, dv_, o, lse, ddo, quad, kv_head_offset=h0)
+        od, _ = cowa.cowa_decode(dqd, dk_, dv_, dsl, quad, kv_head_offset=h0)
         for name, t in (("o", o), ("dq", g1), ("dk", g2), ("dv", g3), ("od", od)):
             outs[name].copy_(t, non_blocking=True)
 
@@ -457,7 +502,7 @@ def run_e2e(args, cowa, wl, q, k, v, do, qd, seqlens, quad, dev, stream, flush, 
             "path": "pinned host -> device copies, cowa_fwd/bwd/decode, device -> pinned host"}
 
 
-def run_full_mask(args, cowa, wl, q, k, v, do, qd, seqlens, dev, stream, flush, world, t_cowa):
+def run_full_mask(args, cowa, wl, q, k, v, do, qd, seqlens, h0, dev, stream, flush, world, t_cowa):
     """The same step with the full-causal quadruple (0, Lk, 0, 0): every key
     at distance 0 .. p is visible to every head.  The ratio of the two times
     is the speedup over a full causal mask, bounded by the ratio of visible
@@ -501,10 +546,14 @@ def run_full_mask(args, cowa, wl, q, k, v, do, qd, seqlens, dev, stream, flush, 
     cowa.cowa_get_device_error(dev)
     t = [sum(e[a].elapsed_time(e[a + 1]) for e in evs) / steps for a in range(3)]
     t = max_over_ranks(t, world, dev)
-    full_pairs = visible_pairs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, quad)
-    cowa_pairs = visible_pairs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, wl.quad)
-    full_keys = decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, quad)
-    cowa_keys = decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, wl.quad)
+    # whole-job work ratios; with KV-head sharding the slowest rank (the
+    # lowest heads, whose long windows lie nearest and are seen by the most
+    # query rows) bounds the speedup instead
+    full_pairs, cowa_pairs, full_keys, cowa_keys = sum_over_ranks([
+        visible_pairs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, quad),
+        visible_pairs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, wl.quad, kv_head_offset=h0),
+        decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, quad),
+        decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, wl.quad, kv_head_offset=h0)], world, dev)
     return {"quad": list(quad), "steps": steps,
             "fwd_ms": round(t[0], 4), "bwd_ms": round(t[1], 4), "decode_ms": round(t[2], 4),
             "speedup_fwd": round(t[0] / t_cowa[0], 3), "speedup_bwd": round(t[1] / t_cowa[1], 3),
@@ -523,7 +572,7 @@ def packed_lengths(total, lo, hi, seed):
     return out
 
 
-def run_packed_workload(args, cowa, wl, dev, stream, flush, world, peaks):
+def run_packed_workload(args, cowa, wl, h0, dev, stream, flush, world, peaks):
     """A packed (variable-length) batch with the workload's heads and window
     quadruple: as many tokens as the workload's batch, in sequences of
     log-uniform lengths between 1/16 and 1x the workload's length."""
@@ -534,16 +583,17 @@ def run_packed_workload(args, cowa, wl, dev, stream, flush, world, peaks):
     q, k, v, do = (t[0] for t in training_inputs(1, T, T, wl.Hq, wl.Hkv, wl.d, device=dev, seed=23))
     cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), device=dev)
     mx = max(lens)
-    pairs = sum(visible_pairs(1, n, n, wl.Hq, wl.Hkv, wl.quad) for n in lens)
+    pairs = int(sum_over_ranks([sum(visible_pairs(1, n, n, wl.Hq, wl.Hkv, wl.quad, kv_head_offset=h0)
+                                    for n in lens)], world, dev)[0])
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(max(3, args.steps))]
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        o, lse = cowa.cowa_fwd_varlen(q, k, v, cu, cu, mx, mx, wl.quad)
+        o, lse = cowa.cowa_fwd_varlen(q, k, v, cu, cu, mx, mx, wl.quad, kv_head_offset=h0)
         if ev is not None:
             ev[1].record(stream)
-        cowa.cowa_bwd_varlen(q, k, v, o, lse, do, cu, cu, mx, mx, wl.quad)
+        cowa.cowa_bwd_varlen(q, k, v, o, lse, do, cu, cu, mx, mx, wl.quad, kv_head_offset=h0)
         if ev is not None:
             ev[2].record(stream)
 
@@ -565,31 +615,37 @@ def run_packed_workload(args, cowa, wl, dev, stream, flush, world, peaks):
     return {"sequences": len(lens), "tokens": T, "min_len": min(lens), "max_len": mx,
             "visible_pairs": pairs, "fwd_ms": round(t_f, 4), "bwd_ms": round(t_b, 4),
             "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": round(bwd_tf, 2),
-            "fwd_frac": round(fwd_tf / peaks["bf16_tflops"], 4), "bwd_frac": round(bwd_tf / peaks["bf16_tflops"], 4),
+            "fwd_frac": round(fwd_tf / world / peaks["bf16_tflops"], 4),
+            "bwd_frac": round(bwd_tf / world / peaks["bf16_tflops"], 4),
             "lengths": "log-uniform in [L/16, L], seed 17"}
 
 
-def run_decode_workload(args, cowa, dev, stream, flush, world, peaks, peak_src):
-    """The 128K decode workload (B=16, Hq=32, Hkv=8, d=128), timed on its own."""
+def run_decode_workload(args, cowa, rank, dev, stream, flush, world, peaks, peak_src):
+    """The 128K decode workload (B=16, Hq=32, Hkv=8, d=128), timed on its own
+    (whole-job bytes over the slowest rank's time; fractions per GPU)."""
+    import torch.distributed as dist
     from structured_sparse_attention_block_b200.inputs import WORKLOADS, workload_inputs
-    wl = WORKLOADS["decode128k"]
-    q, kc, vc, sl = workload_inputs(wl, device=dev, seed=7)
+    wl, h0 = head_shard(WORKLOADS["decode128k"], rank, world, args.parallel)
+    q, kc, vc, sl = workload_inputs(wl, device=dev, seed=7 + 1000 * rank)
     out = torch.empty_like(q)
     lse = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device=dev)
-    ws = torch.empty(cowa.cowa_decode_workspace_size(q, kc, wl.quad), dtype=torch.uint8, device=dev)
+    ws = torch.empty(cowa.cowa_decode_workspace_size(q, kc, wl.quad, h0), dtype=torch.uint8, device=dev)
     for _ in range(max(3, args.warmup)):
-        cowa.cowa_decode(q, kc, vc, sl, wl.quad, out=out, lse=lse, workspace=ws)
+        cowa.cowa_decode(q, kc, vc, sl, wl.quad, kv_head_offset=h0, out=out, lse=lse, workspace=ws)
     torch.cuda.synchronize()
     n = max(args.steps, 10)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    if world > 1:
+        dist.barrier()
     for i in range(n):
         flush.zero_()
         evs[i][0].record(stream)
-        cowa.cowa_decode(q, kc, vc, sl, wl.quad, out=out, lse=lse, workspace=ws)
+        cowa.cowa_decode(q, kc, vc, sl, wl.quad, kv_head_offset=h0, out=out, lse=lse, workspace=ws)
         evs[i][1].record(stream)
     torch.cuda.synchronize()
-    ms = sum(a.elapsed_time(b) for a, b in evs) / n
-    keys = decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, wl.quad)
+    ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in evs) / n], world, dev)[0]
+    keys = int(sum_over_ranks([decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, wl.quad, kv_head_offset=h0)],
+                              world, dev)[0])
     nbytes = keys * 2 * wl.d * 2
     gbs = nbytes / (ms * 1e-3) / 1e9
 
@@ -597,26 +653,30 @@ def run_decode_workload(args, cowa, dev, stream, flush, world, peaks, peak_src):
     # each KV head holds only the keys those steps see
     horizon = 64
     origin = sl - 1
-    kw, vw = cowa.cowa_wcache_build(kc, vc, origin, wl.quad, horizon)
+    kw, vw = cowa.cowa_wcache_build(kc, vc, origin, wl.quad, horizon, kv_head_offset=h0)
     del kc, vc
     torch.cuda.empty_cache()
     for _ in range(max(3, args.warmup)):
-        cowa.cowa_decode_windowed(q, kw, vw, sl, origin, wl.quad, horizon, out=out, lse=lse, workspace=ws)
+        cowa.cowa_decode_windowed(q, kw, vw, sl, origin, wl.quad, horizon, kv_head_offset=h0,
+                                  out=out, lse=lse, workspace=ws)
     torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
     for i in range(n):
         flush.zero_()
         evs[i][0].record(stream)
-        cowa.cowa_decode_windowed(q, kw, vw, sl, origin, wl.quad, horizon, out=out, lse=lse, workspace=ws)
+        cowa.cowa_decode_windowed(q, kw, vw, sl, origin, wl.quad, horizon, kv_head_offset=h0,
+                                  out=out, lse=lse, workspace=ws)
         evs[i][1].record(stream)
     torch.cuda.synchronize()
     cowa.cowa_get_device_error(dev)
-    ms_w = sum(a.elapsed_time(b) for a, b in evs) / n
-    full_bytes = wl.B * wl.Lk * wl.Hkv * wl.d * 2 * 2
-    win_bytes = kw.numel() * kw.element_size() * 2
+    ms_w = max_over_ranks([sum(a.elapsed_time(b) for a, b in evs) / n], world, dev)[0]
+    full_bytes, win_bytes = (int(x) for x in sum_over_ranks(
+        [wl.B * wl.Lk * wl.Hkv * wl.d * 2 * 2, kw.numel() * kw.element_size() * 2], world, dev))
     del q, kw, vw
     torch.cuda.empty_cache()
     return {"workload": wl.name, "ms": round(ms, 4), "visible_kv_bytes": nbytes,
-            "GB/s": round(gbs, 1), "peak": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4),
+            "GB/s": round(gbs, 1), "peak": peaks["hbm_gbs"], "frac": round(gbs / world / peaks["hbm_gbs"], 4),
             "peak_source": "%s hbm_gbs" % peak_src,
             "full_cache_bytes": full_bytes,
             "windowed": {"horizon": horizon, "cache_bytes": win_bytes,
@@ -695,6 +755,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["cowa", "reference"], default="cowa")
     ap.add_argument("--workload", default="recall8k")
+    ap.add_argument("--parallel", choices=["dp", "heads"], default="dp",
+                    help="dp: one replica per GPU (weak scaling); heads: KV heads sharded over the GPUs "
+                         "with kv_head_offset (strong scaling)")
     ap.add_argument("--cpu-rows", type=int, default=4096, help="query rows in the CPU-baseline sample")
     ap.add_argument("--ref-rows", type=int, default=512, help="query rows per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -53,8 +53,10 @@ def _worker(rank, world, port, q, k, v, quad, result):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         from oracle import oracle
-        # the slowest rank sets the step time
+        # the slowest rank sets the step time; whole-job work adds up
         t = bench.max_over_ranks([1.0 + rank, 5.0 - rank], world, "cpu")
+        tot = bench.sum_over_ranks([1.0 + rank, 10.0 * rank], world, "cpu")
+        assert tot == [3.0, 10.0]
         # KV-head sharding: rank r owns KV heads [r*H/R, (r+1)*H/R) and their
         # query heads, and passes its first global head as kv_head_offset
         Hkv = k.shape[2]
@@ -93,3 +95,34 @@ def test_two_rank_reduction_and_head_sharding(oracle_mod):
     assert t == [2.0, 5.0]
     o_full, _ = oracle_mod.fwd(q, k, v, quad)
     np.testing.assert_allclose(o_sharded, o_full, rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("name", ["recall8k", "llm14b_32k", "op128k", "decode128k"])
+def test_head_shard_covers_every_head_once(name):
+    """KV-head sharding: the ranks' head ranges tile [0, Hkv), query heads
+    follow their KV heads, and the ranks' visible work adds up to the whole
+    workload's (the windows are those of the global heads)."""
+    from structured_sparse_attention_block_b200.inputs import WORKLOADS
+    wl = WORKLOADS[name]
+    for world in (1, 2, 4, 8):
+        if wl.Hkv % world:
+            with pytest.raises(SystemExit):
+                bench.head_shard(wl, 0, world, "heads")
+            continue
+        seen, pairs = [], 0
+        for r in range(world):
+            w, h0 = bench.head_shard(wl, r, world, "heads")
+            assert w.Hq * world == wl.Hq and w.Hkv * world == wl.Hkv
+            assert (w.B, w.Lq, w.Lk, w.d, w.quad) == (wl.B, wl.Lq, wl.Lk, wl.d, wl.quad)
+            seen += list(range(h0, h0 + w.Hkv))
+            if wl.kind == "train" and wl.Lq <= 8192:
+                pairs += bench.visible_pairs(w.B, w.Lq, w.Lk, w.Hq, w.Hkv, w.quad, kv_head_offset=h0)
+            else:
+                pairs += bench.decode_visible_keys([w.Lk] * w.B, w.Hkv, w.quad, kv_head_offset=h0)
+        assert seen == list(range(wl.Hkv))
+        if wl.kind == "train" and wl.Lq <= 8192:
+            assert pairs == bench.visible_pairs(wl.B, wl.Lq, wl.Lk, wl.Hq, wl.Hkv, wl.quad)
+        else:
+            assert pairs == bench.decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, wl.quad)
+        # replicas keep the whole workload on every rank
+        assert bench.head_shard(wl, world - 1, world, "dp") == (wl, 0)
