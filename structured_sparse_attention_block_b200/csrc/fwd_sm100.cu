@@ -3,19 +3,24 @@
 // One CTA per (query tile of 128 rows, pair of query heads of one GQA group,
 // batch).  Two query heads of a group have the same KV head, hence the same
 // window mask and the same visible key tiles, so the CTA streams each K/V
-// tile once for both and neither head wastes work.  Ten warps:
+// tile once for both and neither head wastes work.  Eleven warps:
 //   warp 8     TMA producer: both Q tiles once, then the K and V tiles the
 //              schedule lists (sink, near and long bands only) into a ring of
 //              shared-memory stages;
-//   warp 9     MMA issuer (one thread) and tensor-memory owner.  For head slot
-//              x in {0, 1}: S_x(t) = Q_x K_t^T into S_x, and O_x += P_x(t) V_t
+//   warps 9,10 MMA issuers, one thread each, warp 9 + x serving head slot x
+//              (warp 9 also owns the tensor memory): S_x(t) = Q_x K_t^T into
+//              S_x, and O_x += P_x(t) V_t
 //              with P_x(t) read from its own tensor-memory region (a later MMA
 //              writing S_x is not ordered after an earlier MMA's read of P from
 //              the same columns, so P never shares columns with S).  S_x(t+1)
 //              is issued as soon as softmax x has pulled S_x(t) into registers
 //              (S_FREE), so the next score tile is computed while the softmax
 //              of the current one runs; PV_x(t) follows when P_x(t) is written
-//              (P_FULL).  Order per tile: S_0(t+1) S_1(t+1) PV_0(t) PV_1(t);
+//              (P_FULL).  Order per tile and slot: S_x(t+1) PV_x(t).  The two
+//              slots touch disjoint tensor-memory columns, so their issuers
+//              need no ordering between them, and neither slot's waits hold up
+//              the other's MMAs; K_t and V_t are released once both issuers
+//              have committed their tile-t MMAs;
 //   warps 0-3  softmax of slot 0, warps 4-7 softmax of slot 1: thread r of a
 //              warpgroup owns query row r.  Pass 1 reads the row of S in
 //              32-column chunks and takes the max (edge tiles only apply the
@@ -34,6 +39,12 @@
 // d = 128: S_x at 64x, P_x at 128 + 32x, O_x at 192 + 160x.
 // Softmax x rewrites P_x and rescales O_x for tile t only after O_DONE_x says
 // PV_x(t-1) is complete.
+// The exponential loops of the two slots alternate per lane quadrant (the two
+// warps on one SM sub-partition): slot 1 runs tile t's after slot 0 has run
+// its own, and slot 0 runs tile t+1's after slot 1's tile t.  Without this the
+// two warps reach the exponentials together, share the MUFU and issue slots
+// there, and leave them idle while both wait on tensor-memory loads; with it
+// one warp's exponentials overlap the other's loads, max and stores.
 // Every mbarrier wait is bounded; a wait that runs out records a timeout in
 // the device error word and the CTA winds down.
 #include <cudaTypedefs.h>
@@ -70,14 +81,14 @@ struct FwdCfg {
     static constexpr int KV_BYTES = BN * D * 2;       // one of K or V
     static constexpr int ONES_BYTES = BN * 128;       // bf16 1.0, one 128-byte row per key
     static constexpr int STAGE_BYTES = 2 * KV_BYTES + ONES_BYTES;
-    static constexpr int NBAR = 12 + 2 * STAGES;
+    static constexpr int NBAR = 20 + 2 * STAGES;
     static constexpr int SMEM = 1024 + 2 * Q_BYTES + STAGES * STAGE_BYTES + 8 * NBAR + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
     static constexpr uint32_t IDESC_O = idesc_bf16(128, OW, 0, 1);
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant__ FwdArgs a)
+__global__ void __launch_bounds__(352, 1) fwd_sm100_kernel(const __grid_constant__ FwdArgs a)
 {
     using C = FwdCfg<D>;
     constexpr int BM = C::BM, BN = C::BN, ST = C::STAGES, KB = C::KB;
@@ -99,7 +110,9 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
     auto P_FULL = [&](int x) { return bar0 + 8u * (3 + 2 * ST + x); };
     auto O_DONE = [&](int x) { return bar0 + 8u * (5 + 2 * ST + x); };
     auto S_FREE = [&](int x) { return bar0 + 8u * (7 + 2 * ST + x); };
-    const uint32_t FIN = bar0 + 8u * (9 + 2 * ST);
+    auto FIN = [&](int x) { return bar0 + 8u * (9 + 2 * ST + x); };
+    // exponential-loop turn of slot x in lane quadrant qd
+    auto TURN = [&](int x, int qd) { return bar0 + 8u * (12 + 2 * ST + 4 * x + qd); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const TilePos pos = tile_pos(p.Hkv * a.npair, p.B);
@@ -134,15 +147,17 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         mbar_init(BAR_Q, 1);
         for (int s = 0; s < ST; ++s) {
             mbar_init(KV_FULL(s), 1);
-            mbar_init(KV_EMPTY(s), 1);
+            mbar_init(KV_EMPTY(s), nslot);  // one commit per MMA issuer
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(S_FULL(x), 1);
             mbar_init(P_FULL(x), 128);
             mbar_init(O_DONE(x), 1);
             mbar_init(S_FREE(x), 4);  // one arrival per softmax warp
+            for (int qd = 0; qd < 4; ++qd) mbar_init(TURN(x, qd), 1);
         }
-        mbar_init(FIN, 1);
+        mbar_init(FIN(0), 1);
+        mbar_init(FIN(1), 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -194,17 +209,18 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             for (int t = issued > ST ? issued - ST : 0; t < issued; ++t)
                 mbar_wait(KV_FULL(t % ST), (t / ST) & 1, p.err, abort_flag);
         }
-    } else if (warp == 9) {
+    } else if (warp == 9 || warp == 10) {
         // ------------------------------------------------------------ MMA
         // the whole warp runs the loop; one elected lane issues
         const uint32_t FULL = 0xffffffffu;
-        bool ok = __all_sync(FULL, mbar_wait(BAR_Q, 0, p.err, abort_flag));
+        const int x = warp - 9;  // head slot served
+        bool ok = x < nslot && __all_sync(FULL, mbar_wait(BAR_Q, 0, p.err, abort_flag));
         // descriptor bases: Q of slot 0, K and V of stage 0 (the others are
         // fixed byte offsets from these)
         const uint64_t dq0 = sdesc(sQ, 16, 1024);
         const uint64_t dk0 = sdesc(sStage, 16, 1024);
         const uint64_t dv0 = sdesc(sStage + C::KV_BYTES, BN * 128, 1024);
-        auto qk = [&](int x, int t) {  // S_x(t) = Q_x K_t^T
+        auto qk = [&](int t) {  // S_x(t) = Q_x K_t^T
             const uint32_t so = (uint32_t)(t % ST) * C::STAGE_BYTES;
             if (elect_one()) {
 #pragma unroll
@@ -218,7 +234,7 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             }
             __syncwarp();
         };
-        auto pv = [&](int x, int t) -> bool {  // O_x += P_x(t) V_t
+        auto pv = [&](int t) -> bool {  // O_x += P_x(t) V_t
             if (!__all_sync(FULL, mbar_wait(P_FULL(x), t & 1, p.err, abort_flag))) return false;
             tc_fence_after();
             const uint32_t so = (uint32_t)(t % ST) * C::STAGE_BYTES;
@@ -234,26 +250,26 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         };
         if (ntiles > 0 && (ok = ok && __all_sync(FULL, mbar_wait(KV_FULL(0), 0, p.err, abort_flag)))) {
             tc_fence_after();
-            for (int x = 0; x < nslot; ++x) qk(x, 0);
+            qk(0);
         }
         for (int t = 0; ok && t < ntiles; ++t) {
             const int tn = t + 1;
             if (tn < ntiles) {
                 if (!(ok = __all_sync(FULL, mbar_wait(KV_FULL(tn % ST), (tn / ST) & 1, p.err, abort_flag)))) break;
-                for (int x = 0; x < nslot && ok; ++x) {
-                    // softmax x holds S_x(t) in registers: S_x may be rewritten
-                    if (!(ok = __all_sync(FULL, mbar_wait(S_FREE(x), t & 1, p.err, abort_flag)))) break;
-                    tc_fence_after();
-                    qk(x, tn);
-                }
+                // softmax x holds S_x(t) in registers: S_x may be rewritten
+                if (!(ok = __all_sync(FULL, mbar_wait(S_FREE(x), t & 1, p.err, abort_flag)))) break;
+                tc_fence_after();
+                qk(tn);
             }
-            for (int x = 0; x < nslot && ok; ++x) ok = pv(x, t);
-            if (elect_one()) mma_commit(KV_EMPTY(t % ST));  // both heads are done with K_t and V_t
+            ok = pv(t);
+            if (elect_one()) mma_commit(KV_EMPTY(t % ST));  // this head is done with K_t and V_t
             __syncwarp();
         }
-        if (elect_one()) mma_commit(FIN);
-        __syncwarp();
-        mbar_wait(FIN, 0, p.err, abort_flag);
+        if (x < nslot) {
+            if (elect_one()) mma_commit(FIN(x));
+            __syncwarp();
+            mbar_wait(FIN(x), 0, p.err, abort_flag);
+        }
     } else {
         // -------------------------------------------------------- softmax
         const int x = warp >> 2;  // head slot of this warpgroup
@@ -263,6 +279,8 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
         const uint32_t tOx = tmem + C::t_o(x) + lane_off;
         const int prow = pa + r;
         const bool active = x < nslot;
+        const bool turns = nslot == 2;  // a lone head slot takes every turn
+        const uint32_t my_turn = TURN(x, warp & 3), their_turn = TURN(x ^ 1, warp & 3);
         float m_run = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         for (int t = 0; active && t < ntiles; ++t) {
@@ -340,6 +358,14 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
             // sr[e], already consumed
             const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(nms, nms);
             float2 la = make_float2(0.f, 0.f), lc = make_float2(0.f, 0.f);
+            // slot 1's turn for tile t is phase t of its barrier (slot 0 done
+            // with tile t); slot 0's for tile t > 0 is phase t-1 of its own
+            // (slot 1 done with tile t-1).  Neither can run two phases ahead
+            // of the other, so the parity is unambiguous.
+            if (turns && (x == 1 || t > 0)) {
+                ok = __all_sync(0xffffffffu, mbar_wait(my_turn, (x == 1 ? t : t - 1) & 1, p.err, abort_flag));
+                if (!ok) break;
+            }
 #pragma unroll
             for (int e = 0; e < BN / 2; ++e) {
                 const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
@@ -358,6 +384,10 @@ __global__ void __launch_bounds__(320, 1) fwd_sm100_kernel(const __grid_constant
                 else
                     la = __fadd2_rn(la, make_float2(p0, p1));
                 sr[e] = pack2(p0, p1);
+            }
+            if (turns) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(their_turn);
             }
             l += (la.x + la.y) + (lc.x + lc.y);
             // P_x and O_x are rewritten from here on: PV_x(t-1) must be complete
@@ -506,7 +536,7 @@ static cudaError_t launch_fwd5_d(const AttnParams &p, cudaStream_t st)
     const unsigned blocks = tile_grid_blocks(p.nqt, (long long)p.Hkv * a.npair, p.B);
     if (!blocks) return cudaErrorInvalidConfiguration;
     launch_begin("fwd_sm100", st);
-    fwd_sm100_kernel<D><<<blocks, 320, C::SMEM, st>>>(a);
+    fwd_sm100_kernel<D><<<blocks, 352, C::SMEM, st>>>(a);
     launch_end(st);
     return cudaGetLastError();
 }
