@@ -27,7 +27,10 @@
 // 3. dq_sm100_kernel, query-tile major like the forward: per visible key tile
 //        S = Q K^T,  dP = dO V^T,  dS = P (dP - delta),  dQ += dS K.
 //    For d = 64 a CTA takes two query heads of a GQA group (same mask, same
-//    K/V tiles) with one warpgroup each.  As in the dK/dV pass, S and dP of
+//    K/V tiles) with one warpgroup and one MMA-issuing warp each (their
+//    tensor-memory columns are disjoint, so the issuers need no ordering
+//    between them; a K/V stage is released once both have committed).  As in
+//    the dK/dV pass, S and dP of
 //    tile t+1 are issued once the warpgroup has read those of tile t
 //    (S_FREE), ahead of dQ += dS(t) K_t; dS(t+1) is written after that dQ
 //    MMA completes (DONE).
@@ -452,7 +455,7 @@ struct DqCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant__ BwdArgs a)
+__global__ void __launch_bounds__(352, 1) dq_sm100_kernel(const __grid_constant__ BwdArgs a)
 {
     using C = DqCfg<D>;
     constexpr int BM = C::BM, BN = C::BN, ST = C::ST, KB = C::KB, NSLOT = C::NSLOT;
@@ -474,7 +477,7 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
     auto S_FULL = [&](int x) { return bar0 + 8u * (1 + 2 * ST + x); };
     auto DS_FULL = [&](int x) { return bar0 + 8u * (3 + 2 * ST + x); };
     auto DONE = [&](int x) { return bar0 + 8u * (5 + 2 * ST + x); };
-    const uint32_t FIN = bar0 + 8u * (7 + 2 * ST);
+    auto FIN = [&](int x) { return bar0 + 8u * (x == 0 ? 7 + 2 * ST : 10 + 2 * ST); };
     auto S_FREE = [&](int x) { return bar0 + 8u * (8 + 2 * ST + x); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -510,15 +513,15 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
         mbar_init(BAR_Q, 1);
         for (int s = 0; s < ST; ++s) {
             mbar_init(KV_FULL(s), 1);
-            mbar_init(KV_EMPTY(s), 1);
+            mbar_init(KV_EMPTY(s), nslot);  // one commit per MMA issuer
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(S_FULL(x), 1);
             mbar_init(DS_FULL(x), 128);
             mbar_init(DONE(x), 1);
             mbar_init(S_FREE(x), 4);  // one arrival per warp
+            mbar_init(FIN(x), 1);
         }
-        mbar_init(FIN, 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -563,15 +566,16 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
             for (int t = issued > ST ? issued - ST : 0; t < issued; ++t)
                 mbar_wait(KV_FULL(t % ST), (t / ST) & 1, p.err, abort_flag);
         }
-    } else if (warp == 9) {
+    } else if (warp == 9 || warp == 10) {
         // ------------------------------------------------------------ MMA
         // the whole warp runs the loop; one elected lane issues
         const uint32_t FULL = 0xffffffffu;
-        bool ok = __all_sync(FULL, mbar_wait(BAR_Q, 0, p.err, abort_flag));
+        const int x = warp - 9;  // head slot served
+        bool ok = x < nslot && __all_sync(FULL, mbar_wait(BAR_Q, 0, p.err, abort_flag));
         const uint64_t dq0 = sdesc(sQ(0), 16, 1024), ddo0 = sdesc(sDO(0), 16, 1024);
         const uint64_t dk0 = sdesc(sStage, 16, 1024), dv0 = sdesc(sStage + C::KV_BYTES, 16, 1024);
         const uint64_t dkm0 = sdesc(sStage, BN * 128, 1024);
-        auto sdp = [&](int x, int t) {  // S_x = Q_x K_t^T, dP_x = dO_x V_t^T
+        auto sdp = [&](int t) {  // S_x = Q_x K_t^T, dP_x = dO_x V_t^T
             const uint32_t so = (uint32_t)(t % ST) * C::STAGE_BYTES;
             const uint32_t ts = tmem + x * C::SLOT;
             if (elect_one()) {
@@ -586,7 +590,7 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
             }
             __syncwarp();
         };
-        auto dq = [&](int x, int t) -> bool {  // dQ_x += dS_x K_t
+        auto dq = [&](int t) -> bool {  // dQ_x += dS_x K_t
             if (!__all_sync(FULL, mbar_wait(DS_FULL(x), t & 1, p.err, abort_flag))) return false;
             tc_fence_after();
             const uint32_t so = (uint32_t)(t % ST) * C::STAGE_BYTES;
@@ -605,27 +609,27 @@ __global__ void __launch_bounds__(320, 1) dq_sm100_kernel(const __grid_constant_
             ok = __all_sync(FULL, mbar_wait(KV_FULL(0), 0, p.err, abort_flag));
             if (ok) {
                 tc_fence_after();
-                for (int x = 0; x < nslot; ++x) sdp(x, 0);
+                sdp(0);
             }
         }
         for (int t = 0; ok && t < ntiles; ++t) {
             if (t + 1 < ntiles) {
                 if (!(ok = __all_sync(FULL, mbar_wait(KV_FULL((t + 1) % ST), ((t + 1) / ST) & 1, p.err, abort_flag))))
                     break;
-                for (int x = 0; x < nslot && ok; ++x) {
-                    // warpgroup x holds S_x(t) and dP_x(t) in registers
-                    if (!(ok = __all_sync(FULL, mbar_wait(S_FREE(x), t & 1, p.err, abort_flag)))) break;
-                    tc_fence_after();
-                    sdp(x, t + 1);
-                }
+                // warpgroup x holds S_x(t) and dP_x(t) in registers
+                if (!(ok = __all_sync(FULL, mbar_wait(S_FREE(x), t & 1, p.err, abort_flag)))) break;
+                tc_fence_after();
+                sdp(t + 1);
             }
-            for (int x = 0; x < nslot && ok; ++x) ok = dq(x, t);
-            if (elect_one()) mma_commit(KV_EMPTY(t % ST));
+            ok = dq(t);
+            if (elect_one()) mma_commit(KV_EMPTY(t % ST));  // this head is done with K_t and V_t
             __syncwarp();
         }
-        if (elect_one()) mma_commit(FIN);
-        __syncwarp();
-        mbar_wait(FIN, 0, p.err, abort_flag);
+        if (x < nslot) {
+            if (elect_one()) mma_commit(FIN(x));
+            __syncwarp();
+            mbar_wait(FIN(x), 0, p.err, abort_flag);
+        }
     } else {
         // ------------------------------------------------- dS per query row
         const int x = warp >> 2;
@@ -801,7 +805,7 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, i
         const unsigned g2 = tile_grid_blocks(nqt_dq, (long long)p.Hkv * a.npair, p.B);
         if (!g2) return cudaErrorInvalidConfiguration;
         launch_begin("dq_sm100", st);
-        dq_sm100_kernel<D><<<g2, 320, Q::SMEM, st>>>(a);
+        dq_sm100_kernel<D><<<g2, 352, Q::SMEM, st>>>(a);
         launch_end(st);
         e = cudaGetLastError();
     }
