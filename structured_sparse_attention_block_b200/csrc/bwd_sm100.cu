@@ -17,11 +17,16 @@
 //        dV += P^T dO,  dK += dS^T Q                   (MMA, P^T and dS^T from
 //                                                       tensor memory)
 //    Two warpgroups take alternate tasks so one computes while the MMAs of
-//    the other run.  Warpgroup x releases S^T/dP^T of task u as soon as it
-//    has read them (S_FREE) and the MMA thread issues S^T/dP^T of task u+2
-//    into the same buffer before the gradient MMAs of task u, so the next
+//    the other run.  Two MMA-issuing warps split the MMAs by role: one
+//    issues S^T/dP^T (writing only the task buffers), the other the gradient
+//    MMAs (the only writer of dK and dV), so each issues half the
+//    instructions and neither waits on the other's barriers.  Warpgroup x
+//    releases S^T/dP^T of task u as soon as it has read them (S_FREE) and
+//    S^T/dP^T of task u+2 go into the same buffer at once, so the next
 //    task's scores are ready when the warpgroup finishes; P^T/dS^T of task
-//    u+2 are written only after those gradient MMAs complete (G_DONE).
+//    u+2 are written only after the gradient MMAs of task u complete
+//    (G_DONE).  A Q/dO stage is released by the gradient issuer: the score
+//    MMAs of its task completed before P^T of the task existed.
 //    dK is scaled by softmax_scale in the epilogue.
 //
 // 3. dq_sm100_kernel, query-tile major like the forward: per visible key tile
@@ -114,14 +119,14 @@ struct KvCfg {
     static constexpr int STAGE_BYTES = (2 * QT_BYTES + LSD_BYTES + 1023) / 1024 * 1024;
     // tensor memory: dK, dV, then two buffers of S^T, dP^T, P^T (bf16), dS^T (bf16)
     static constexpr int T_DK = 0, T_DV = D, T_BUF = 2 * D, BUF = 3 * BM;
-    static constexpr int NBAR = 11 + 2 * ST;
+    static constexpr int NBAR = 12 + 2 * ST;
     static constexpr int SMEM = 1024 + 2 * KV_BYTES + ST * STAGE_BYTES + 8 * NBAR + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BM, 0, 0);
     static constexpr uint32_t IDESC_G = idesc_bf16(128, D, 0, 1);
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constant__ BwdArgs a)
+__global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constant__ BwdArgs a)
 {
     using C = KvCfg<D>;
     constexpr int BN = C::BN, BM = C::BM, ST = C::ST, KB = C::KB;
@@ -146,7 +151,7 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
     auto S_FULL = [&](int x) { return bar0 + 8u * (1 + 2 * ST + x); };
     auto P_FULL = [&](int x) { return bar0 + 8u * (3 + 2 * ST + x); };
     const uint32_t DONE = bar0 + 8u * (5 + 2 * ST);
-    const uint32_t FIN = bar0 + 8u * (6 + 2 * ST);
+    auto FIN = [&](int r) { return bar0 + 8u * (r == 0 ? 6 + 2 * ST : 11 + 2 * ST); };  // per issuer
     auto S_FREE = [&](int x) { return bar0 + 8u * (7 + 2 * ST + x); };
     auto G_DONE = [&](int x) { return bar0 + 8u * (9 + 2 * ST + x); };
 
@@ -189,7 +194,8 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
             mbar_init(G_DONE(x), 1);
         }
         mbar_init(DONE, 1);
-        mbar_init(FIN, 1);
+        mbar_init(FIN(0), 1);
+        mbar_init(FIN(1), 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -236,10 +242,12 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
             for (int u = issued > ST ? issued - ST : 0; u < issued; ++u)
                 mbar_wait(Q_FULL(u % ST), (u / ST) & 1, p.err, abort_flag);
         }
-    } else if (warp == 9) {
+    } else if (warp == 9 || warp == 10) {
         // ------------------------------------------------------------ MMA
-        // the whole warp runs the loop; one elected lane issues
+        // the whole warp runs the loop; one elected lane issues.  Warp 9
+        // issues the score MMAs, warp 10 the gradient MMAs.
         const uint32_t FULL = 0xffffffffu;
+        const int role = warp - 9;
         bool ok = __all_sync(FULL, mbar_wait(KV_LOADED, 0, p.err, abort_flag));
         const uint64_t dk0 = sdesc(sK, 16, 1024), dv0 = sdesc(sV, 16, 1024);
         const uint64_t dq0 = sdesc(stage_q(0), 16, 1024), ddo0 = sdesc(stage_do(0), 16, 1024);
@@ -283,23 +291,24 @@ __global__ void __launch_bounds__(320, 1) dkdv_sm100_kernel(const __grid_constan
             __syncwarp();
             return true;
         };
-        if (ok && ntask > 0) ok = sdp(0);
-        if (ok && ntask > 1) ok = sdp(1);
-        for (int u = 0; ok && u < ntask; ++u) {
-            if (u + 2 < ntask) {
-                // warpgroup u % 2 holds S^T and dP^T of task u in registers
-                if (!(ok = __all_sync(FULL, mbar_wait(S_FREE(u & 1), (u >> 1) & 1, p.err, abort_flag)))) break;
-                tc_fence_after();
-                if (!(ok = sdp(u + 2))) break;
+        if (role == 0) {
+            for (int u = 0; ok && u < ntask; ++u) {
+                if (u >= 2) {
+                    // warpgroup u % 2 has read S^T and dP^T of task u-2
+                    if (!(ok = __all_sync(FULL, mbar_wait(S_FREE(u & 1), ((u - 2) >> 1) & 1, p.err, abort_flag))))
+                        break;
+                    tc_fence_after();
+                }
+                ok = sdp(u);
             }
-            ok = grad(u);
+        } else {
+            for (int u = 0; ok && u < ntask; ++u) ok = grad(u);
+            if (elect_one()) mma_commit(DONE);  // every gradient MMA; the score MMAs completed before them
+            __syncwarp();
         }
-        if (elect_one()) {
-            mma_commit(DONE);
-            mma_commit(FIN);
-        }
+        if (elect_one()) mma_commit(FIN(role));
         __syncwarp();
-        mbar_wait(FIN, 0, p.err, abort_flag);
+        mbar_wait(FIN(role), 0, p.err, abort_flag);
     } else {
         // ---------------------------------------------- P^T and dS^T per key
         const int x = warp >> 2;
@@ -788,7 +797,7 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, i
         const unsigned g1 = tile_grid_blocks(nkt_kv, p.Hkv, p.B);
         if (!g1) return cudaErrorInvalidConfiguration;
         launch_begin("dkdv_sm100", st);
-        dkdv_sm100_kernel<D><<<g1, 320, K::SMEM, st>>>(a);
+        dkdv_sm100_kernel<D><<<g1, 352, K::SMEM, st>>>(a);
         launch_end(st);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
