@@ -91,13 +91,6 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const AttnParams p, float
 }
 
 // bitmask of bit positions [lo, hi] within 0..31 (empty when lo > hi)
-__device__ __forceinline__ uint32_t span_bits(int lo, int hi)
-{
-    lo = max(lo, 0);
-    hi = min(hi, 31);
-    return lo > hi ? 0u : ((0xFFFFFFFFu >> (31 - (hi - lo))) << lo);
-}
-
 // ------------------------------------------------------------------ dK/dV --
 struct BwdArgs {
     CUtensorMap tq, tk, tv, tdo;
@@ -317,14 +310,9 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tb = tmem + C::T_BUF + x * C::BUF + lane_off;
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-        // aligned positions p that see key jg: sink [jg, Lk-1], near
-        // [jg, jg+N-1], long [jg+c, jg+e-1], as 32-bit bounds (an empty
-        // interval has hi < lo; every position is below 2^30)
-        const long long pmax = (long long)sg.Lk - 1;
-        const int snk_hi = jg < w.S ? (int)pmax : -1;
-        const int nr_hi = w.N > 0 ? (int)min((long long)jg + w.N - 1, pmax) : -1;
-        const int lg_lo = (int)min((long long)jg + w.c, pmax + 1);
-        const int lg_hi = w.e > w.c ? (int)min((long long)jg + w.e - 1, pmax) : -1;
+        // the aligned positions that see key jg (sink, near, long), as runs
+        // formed once: a task's columns need no mask when one run holds them
+        const Runs3 kr = key_pos_runs(jg, w, sg.Lk - 1);
         // this warpgroup's tasks u = x, x+2, ...: query head gi of the group
         // and position t in the key tile's query-tile list, advanced without
         // division
@@ -343,18 +331,14 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
             }
             const int q0 = qt * BM;
             const int nrows = min(BM, sg.Lq - q0);
-            const int pa = q0 + delta_pos;
-            const bool full = tile_full(pa, pa + nrows - 1, c0, BN, sg.Lk, w);
+            const int pa = q0 + delta_pos, pb = pa + nrows - 1;
+            // no mask when every key of the warp sees every in-range column
+            const bool full = __all_sync(0xffffffffu, runs_cover(kr, pa, pb));
             uint32_t vis[BM / 32];
+            if (!full) {
 #pragma unroll
-            for (int c = 0; c < BM / 32; ++c) {
-                // query columns of chunk c: p = pa + c*32 + bit, rows < nrows
-                const int pc = pa + c * 32, rmax = pa + nrows - 1;
-                auto span = [&](int lo, int hi) -> uint32_t {
-                    hi = min(hi, rmax);
-                    return hi < lo ? 0u : span_bits(lo - pc, hi - pc);
-                };
-                vis[c] = full ? 0xFFFFFFFFu : (span(jg, snk_hi) | span(jg, nr_hi) | span(lg_lo, lg_hi));
+                for (int c = 0; c < BM / 32; ++c)  // columns p = pa + c*32 + bit, in range up to pb
+                    vis[c] = runs_bits(kr, pa + c * 32) & span_bits(0, pb - pa - c * 32);
             }
             const float2 *lsd = stage_lsd(u % ST);
             ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), k & 1, p.err, abort_flag));
@@ -656,19 +640,18 @@ __global__ void __launch_bounds__(352, 1) dq_sm100_kernel(const __grid_constant_
         }
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nl2 = make_float2(nl, nl),
                      nd2 = make_float2(nd, nd);
+        // the keys row prow sees, as runs formed once: a tile needs no mask
+        // when one run holds it for every row of the warp
+        const Runs3 rr = row_key_runs(prow, w);
         bool ok = true;
         for (int t = 0; active && t < ntiles; ++t) {
             // tile set-up, independent of the scores: done while they land
-            const int kt = tile_of(t);
-            const bool full = tile_full(pa, pb, kt * BN, BN, sg.Lk, w);
+            const int j0 = tile_of(t) * BN;
+            const bool full = __all_sync(0xffffffffu, runs_cover(rr, j0, j0 + BN - 1));
             uint32_t vis[BN / 32];
+            if (!full) {
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
-                const int j0 = kt * BN + c * 32;
-                uint32_t m = span_bits(-j0, min(w.S - 1, prow) - j0);
-                if (w.N > 0) m |= span_bits(prow - w.N + 1 - j0, prow - j0);
-                if (w.e > w.c) m |= span_bits(prow - w.e + 1 - j0, prow - w.c - j0);
-                vis[c] = full ? 0xFFFFFFFFu : m;
+                for (int c = 0; c < BN / 32; ++c) vis[c] = runs_bits(rr, j0 + c * 32);
             }
             ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), t & 1, p.err, abort_flag));
             if (!ok) break;

@@ -42,6 +42,91 @@ __host__ __device__ __forceinline__ bool visible(int p, int j, const Win &w)
     return d >= 0 && (j < w.S || d < w.N || (d >= w.c && d < w.e));
 }
 
+// Bits lo..hi of a 32-bit word (clipped to 0..31; none when lo > hi).
+__host__ __device__ __forceinline__ uint32_t span_bits(int lo, int hi)
+{
+    lo = lo > 0 ? lo : 0;
+    hi = hi < 31 ? hi : 31;
+    return lo > hi ? 0u : ((0xFFFFFFFFu >> (31 - (hi - lo))) << lo);
+}
+
+// The visible set of one query row (keys) or one key (query positions) as at
+// most three runs [a, b], ascending, disjoint and not touching; an absent run
+// has a > b.  A thread of the tcgen05 kernels owns one row or one key for the
+// whole CTA, so it forms its runs once; a tile is then fully visible to it
+// when one run covers the tile's span, and its edge bitmask is the union of
+// the runs' bits.
+struct Runs3 {
+    int a0, b0, a1, b1, a2, b2;
+};
+
+// Adds run [a, b] (a not below any earlier run's start) to the runs formed
+// so far, merging it with the open run when they overlap or touch.
+struct RunBuilder {
+    Runs3 r{1, 0, 1, 0, 1, 0};
+    int n = 0, ca = 1, cb = 0;  // runs closed so far; the open run
+    __host__ __device__ void close()
+    {
+        if (ca > cb) return;
+        if (n == 0) { r.a0 = ca; r.b0 = cb; }
+        else if (n == 1) { r.a1 = ca; r.b1 = cb; }
+        else { r.a2 = ca; r.b2 = cb; }
+        ++n;
+    }
+    __host__ __device__ void add(int a, int b)
+    {
+        if (a > b) return;
+        if (ca <= cb && a <= cb + 1) {
+            cb = b > cb ? b : cb;
+            return;
+        }
+        close();
+        ca = a;
+        cb = b;
+    }
+    __host__ __device__ Runs3 done()
+    {
+        close();
+        return r;
+    }
+};
+
+// Keys seen by the query at aligned position p: sink [0, min(S-1, p)], long
+// [p-e+1, p-c] and near [p-N+1, p], clipped at key 0 (in this order their
+// starts do not decrease, since e >= N).
+__host__ __device__ inline Runs3 row_key_runs(int p, const Win &w)
+{
+    RunBuilder rb;
+    rb.add(0, w.S - 1 < p ? w.S - 1 : p);
+    if (w.e > w.c) rb.add(p - w.e + 1 > 0 ? p - w.e + 1 : 0, p - w.c);
+    if (w.N > 0) rb.add(p - w.N + 1 > 0 ? p - w.N + 1 : 0, p);
+    return rb.done();
+}
+
+// Aligned query positions (at most pmax) that see key j: sink [j, pmax] for
+// j < S, near [j, j+N-1] and long [j+c, j+e-1].
+__host__ __device__ inline Runs3 key_pos_runs(int j, const Win &w, int pmax)
+{
+    RunBuilder rb;
+    const int near_hi = w.N > 0 ? (j + (w.N - 1) < pmax ? j + (w.N - 1) : pmax) : j - 1;
+    const int first_hi = j < w.S ? pmax : near_hi;  // the sink reaches every later position
+    rb.add(j, first_hi);
+    if (w.e > w.c) rb.add(j + w.c, j + (w.e - 1) < pmax ? j + (w.e - 1) : pmax);
+    return rb.done();
+}
+
+// Whether one run holds all of [lo, hi].
+__host__ __device__ __forceinline__ bool runs_cover(const Runs3 &r, int lo, int hi)
+{
+    return (r.a0 <= lo && hi <= r.b0) || (r.a1 <= lo && hi <= r.b1) || (r.a2 <= lo && hi <= r.b2);
+}
+
+// Bit k set when index j0 + k lies in a run.
+__host__ __device__ __forceinline__ uint32_t runs_bits(const Runs3 &r, int j0)
+{
+    return span_bits(r.a0 - j0, r.b0 - j0) | span_bits(r.a1 - j0, r.b1 - j0) | span_bits(r.a2 - j0, r.b2 - j0);
+}
+
 // Key tiles visited by a query tile whose in-range rows have aligned
 // positions pa..pb: the union over rows of the sink, near and long key
 // intervals, each contiguous, so every listed tile holds a visible pair.

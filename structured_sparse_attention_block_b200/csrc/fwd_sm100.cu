@@ -281,37 +281,24 @@ __global__ void __launch_bounds__(352, 1) fwd_sm100_kernel(const __grid_constant
         const bool active = x < nslot;
         const bool turns = nslot == 2;  // a lone head slot takes every turn
         const uint32_t my_turn = TURN(x, warp & 3), their_turn = TURN(x ^ 1, warp & 3);
+        // the keys row prow sees (sink, long, near), as runs formed once:
+        // a tile needs no mask when one run holds it for every row of the
+        // warp (a valid row's runs end at its own position, so a tile
+        // reaching past the sequence's last key is never held)
+        const Runs3 rr = row_key_runs(prow, w);
         float m_run = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         for (int t = 0; active && t < ntiles; ++t) {
             // tile set-up, independent of the scores: done while they land.
             // Edge tiles build, per 32-key chunk, the bitmask of keys the row
-            // sees: the union of its sink, near and long key intervals.
-            const int kt = tile_of(t);
-            // (the longest key length serves for the sequence's own: no
-            // covering interval ends past pa <= Lk_b - 1, so a tile reaching
-            // past the sequence's last key is never full)
-            const bool full = tile_full(pa, pb, kt * BN, BN, p.Lk, w);
+            // sees.
+            const int j0 = tile_of(t) * BN;
+            const bool full = __all_sync(0xffffffffu, runs_cover(rr, j0, j0 + BN - 1));
             constexpr int NC = BN / 32;  // 32-column chunks of the row
             uint32_t vis[NC];
             if (!full) {
 #pragma unroll
-                for (int c = 0; c < NC; ++c) {
-                    const int j0 = kt * BN + c * 32;
-                    // key intervals [lo, hi] of the row, relative to j0
-                    const int sh = min(w.S - 1, prow) - j0;                    // sink [0, min(S-1, p)]
-                    const int nl = prow - w.N + 1 - j0, nh = prow - j0;        // near [p-N+1, p]
-                    const int ll = prow - w.e + 1 - j0, lh = prow - w.c - j0;  // long [p-e+1, p-c]
-                    auto bits = [](int lo, int hi) -> uint32_t {
-                        lo = max(lo, 0);
-                        hi = min(hi, 31);
-                        return lo > hi ? 0u : ((0xFFFFFFFFu >> (31 - (hi - lo))) << lo);
-                    };
-                    uint32_t m = bits(-j0, sh);
-                    if (w.N > 0) m |= bits(nl, nh);
-                    if (w.e > w.c) m |= bits(ll, lh);
-                    vis[c] = m;
-                }
+                for (int c = 0; c < NC; ++c) vis[c] = runs_bits(rr, j0 + c * 32);
             }
             ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), t & 1, p.err, abort_flag));
             if (!ok) break;
@@ -371,7 +358,8 @@ __global__ void __launch_bounds__(352, 1) fwd_sm100_kernel(const __grid_constant
                 const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
                                              sc2, nm2);
                 float p0, p1;
-                if (C::POLY_EVERY && e % C::POLY_EVERY == C::POLY_EVERY - 1) {  // FMA pipe, the rest on the MUFU
+                constexpr int PE = C::POLY_EVERY > 0 ? C::POLY_EVERY : 1;
+                if (C::POLY_EVERY && e % PE == PE - 1) {  // FMA pipe, the rest on the MUFU
                     const float2 pp = exp2_poly2(xa);
                     p0 = pp.x;
                     p1 = pp.y;
