@@ -73,9 +73,10 @@ struct FwdCfg {
     static constexpr __host__ __device__ int t_p(int x) { return D == 128 ? 128 + 32 * x : 192 + 64 * x; }
     static constexpr __host__ __device__ int t_o(int x) { return D == 128 ? 192 + 160 * x : 320 + 96 * x; }
     static constexpr int OW = D + 16;                 // O columns, then the bf16 row sums
-    // exponentials on the FMA pipe: one pair in three for d = 64, where the
-    // softmax paces the kernel; none for d = 128, where it measured slower
-    static constexpr int POLY_EVERY = D == 64 ? 3 : 0;
+    // exponentials on the FMA pipe: one pair in four for d = 64, where the
+    // softmax paces the kernel (measured against none, one in two and one in
+    // three); none for d = 128, where it measured slower
+    static constexpr int POLY_EVERY = D == 64 ? 4 : 0;
     static constexpr int KB = D / 64;                 // 128-byte blocks along d
     static constexpr int Q_BYTES = BM * D * 2;        // one head's query tile
     static constexpr int KV_BYTES = BN * D * 2;       // one of K or V
