@@ -216,14 +216,42 @@ KERNEL_SOURCES = {
 SHARED_SOURCES = ["common.cuh", "kernels.cuh", "sm100.cuh"]
 
 
+def strip_comments(src):
+    """C/C++ source without its comments and blank lines, trailing spaces
+    removed: what the compiler sees of it, so that editing a comment does not
+    mark a kernel as changed.  String and character literals are kept whole."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).splitlines())
+    return "\n".join(ln for ln in lines if ln) + "\n"
+
+
 def kernel_source_sha(kernel):
-    """First 16 hex digits of sha256 over the kernel's source files."""
+    """First 16 hex digits of sha256 over the code (comments stripped) of the
+    kernel's source files."""
     import hashlib
     csrc = os.path.join(ROOT, "structured_sparse_attention_block_b200", "csrc")
     h = hashlib.sha256()
     for name in sorted(KERNEL_SOURCES.get(kernel, []) + SHARED_SOURCES):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + b"\0" + strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

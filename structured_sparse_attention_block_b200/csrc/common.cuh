@@ -247,8 +247,10 @@ __host__ __device__ inline TileRanges key_tile_ranges(int c0, int c1, int Lq, in
 // j >= S the rows that see it form j + D with D = [0,N) u [c,e); a row
 // range fits one connected part [a,b] of D iff j lies in [pb-b, pa-a].  Sink
 // columns j < S need j <= pa.  The tile is full iff its columns are covered
-// by the union of those (at most three) column intervals.  Scalars only, so
-// the per-tile test stays in registers.
+// by the union of those (at most three) column intervals.  Scalars only.
+// Labels the tiles of cowa_tile_classes; the tcgen05 kernels test coverage
+// per thread instead (runs_cover on the thread's visible runs, then a warp
+// vote).
 __host__ __device__ inline bool tile_full(int pa, int pb, int c0, int BN, int Lk, const Win &w)
 {
     const int c1 = c0 + BN - 1;

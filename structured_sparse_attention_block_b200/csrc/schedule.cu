@@ -7,11 +7,13 @@
 // (KV head, query tile) this kernel writes the sink / near / long key-tile
 // ranges, merged into at most three disjoint sorted ranges; the key-tile
 // major form (for dK/dV) lists, for every key tile, the query tiles that see
-// it.  Whether a visited tile needs the element mask is decided per tile by
-// tile_full() in the consumers.  The tcgen05 kernels evaluate the same closed
-// form per CTA (query_tile_ranges / key_tile_ranges) instead of reading this
-// table; it serves the warp-level kernels of the degenerate shapes and
-// cowa_tile_classes, the schedule as the kernels see it.
+// it.  The tcgen05 kernels evaluate the same closed form per CTA
+// (query_tile_ranges / key_tile_ranges) instead of reading this table; it
+// serves cowa_tile_classes, the schedule as a table that tests compare with
+// brute force, with each visited tile labelled full or partial by
+// tile_full().  (The kernels decide per warp instead: a warp skips the mask
+// when each of its threads' visible runs covers the tile, which holds for
+// every warp of a full tile and for no warp whose rows see only part of it.)
 #include "common.cuh"
 #include "kernels.cuh"
 

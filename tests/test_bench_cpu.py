@@ -126,3 +126,15 @@ def test_head_shard_covers_every_head_once(name):
             assert pairs == bench.decode_visible_keys([wl.Lk] * wl.B, wl.Hkv, wl.quad)
         # replicas keep the whole workload on every rank
         assert bench.head_shard(wl, world - 1, world, "dp") == (wl, 0)
+
+
+def test_source_hash_ignores_comments_only():
+    """The staleness check of the committed DRAM counters: comments and blank
+    lines do not count as a kernel change, code (string literals included)
+    does."""
+    code = 'int f() { return 1; }  // one\n/* block\n comment */\nconst char *s = "// kept /* */";\n'
+    assert bench.strip_comments(code) == 'int f() { return 1; }\nconst char *s = "// kept /* */";\n'
+    assert bench.strip_comments(code) == bench.strip_comments(code.replace("// one", "// other\n\n"))
+    assert bench.strip_comments(code) != bench.strip_comments(code.replace("return 1", "return 2"))
+    assert bench.strip_comments(code) != bench.strip_comments(code.replace("// kept", "// kept!"))
+    assert bench.strip_comments("char c = '\\'';  // q\n") == "char c = '\\'';\n"
