@@ -300,6 +300,17 @@ COWA_API int cowa_tile_classes(int64_t Lq, int64_t Lk, int64_t kv_head, cowa_qua
  */
 COWA_API int cowa_get_device_error(void *stream);
 
+/*
+ * Self-test of the timeout path: launches one 32-thread block whose only
+ * work is the kernels' bounded mbarrier wait on a barrier that nothing
+ * completes.  After the wait limit (2 s) the block records COWA_ERR_TIMEOUT in
+ * the device error word and returns, so the context stays usable, and
+ * cowa_get_device_error(stream) then returns COWA_ERR_TIMEOUT.  Touches no
+ * caller memory.  Returns launch-time errors only: COWA_ERR_UNSUPPORTED on a
+ * device other than sm_100, COWA_ERR_CUDA if the launch fails.
+ */
+COWA_API int cowa_selftest_wait_timeout(void *stream);
+
 #ifdef __cplusplus
 }
 #endif

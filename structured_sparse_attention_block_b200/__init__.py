@@ -30,7 +30,7 @@ __all__ = ["CowaError", "cowa_fwd", "cowa_bwd", "cowa_decode", "cowa_default_qua
            "cowa_decode_workspace_size", "cowa_get_device_error", "cowa_launch_count",
            "cowa_decode_noalloc", "cowa_trace_start", "cowa_trace_stop", "cowa_trace_entries",
            "cowa_wcache_rows", "cowa_wcache_build", "cowa_wcache_append", "cowa_decode_windowed",
-           "cowa_fwd_varlen", "cowa_bwd_varlen",
+           "cowa_fwd_varlen", "cowa_bwd_varlen", "cowa_selftest_wait_timeout",
            "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -112,6 +112,8 @@ def lib():
         L.cowa_tile_classes.argtypes = [i64, i64, i64, Quad, i32, i32, ctypes.c_int, vp, vp, sz, vp]
         L.cowa_get_device_error.restype = ctypes.c_int
         L.cowa_get_device_error.argtypes = [vp]
+        L.cowa_selftest_wait_timeout.restype = ctypes.c_int
+        L.cowa_selftest_wait_timeout.argtypes = [vp]
         VP = ctypes.POINTER(VarlenShape)
         for name in ("cowa_fwd_varlen_workspace_size", "cowa_bwd_varlen_workspace_size"):
             f = getattr(L, name)
@@ -514,6 +516,14 @@ def cowa_trace_entries():
         _check(L.cowa_trace_entry(i, ctypes.byref(name), ctypes.byref(ms)))
         out.append((name.value.decode(), float(ms.value)))
     return out, int(L.cowa_trace_dropped())
+
+
+def cowa_selftest_wait_timeout(device=None):
+    """Launch the timeout self-test: a block whose bounded wait on a barrier
+    that nothing completes runs out after 2 s and records COWA_ERR_TIMEOUT,
+    which the next cowa_get_device_error raises."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    _check(lib().cowa_selftest_wait_timeout(_stream(dev)))
 
 
 def cowa_get_device_error(device=None):

@@ -16,6 +16,9 @@
 namespace cowa {
 __device__ int g_cowa_device_error = 0;
 
+// The timeout self-test kernel's launcher (selftest.cu).
+cudaError_t launch_wait_selftest(int *err, cudaStream_t st);
+
 // Records a status and its detail for cowa_last_error_detail() from code
 // outside this file.
 int set_error_detail(int status, const char *detail);
@@ -778,6 +781,15 @@ int cowa_tile_classes(int64_t Lq, int64_t Lk, int64_t kv_head, cowa_quad_t quad,
         e = cowa::launch_tile_classes((const int *)ws, out, (int)kv_head, (int)Lq, (int)Lk, quad.S, quad.N, quad.G,
                                       quad.W, BM, BN, transposed ? 1 : 0, st);
     if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+    return COWA_OK;
+}
+
+int cowa_selftest_wait_timeout(void *stream)
+{
+    const int rc = check_device(nullptr);
+    if (rc != COWA_OK) return rc;
+    const cudaError_t e = cowa::launch_wait_selftest(device_error_word(), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wait self-test launch");
     return COWA_OK;
 }
 
