@@ -147,3 +147,12 @@ def test_varlen_argument_errors(cowa):
     assert call(vshape(tk=0, mk=0)) == 2      # no keys at all
     assert lib.cowa_fwd_varlen(ctypes.byref(vshape()), cowa.Quad(1, 2, 0, 3), 0.0, None, p, p, p, p, p, p, p,
                                1 << 20, None) == 1  # cu_q is NULL
+
+
+def test_selftest_refused_without_a_device(cowa):
+    """With no sm_100 device the timeout self-test launches nothing and
+    returns a status (the GPU test covers the launch itself)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present: tests/test_timeout_gpu.py runs the self-test")
+    assert cowa.lib().cowa_selftest_wait_timeout(None) in (2, 5)  # UNSUPPORTED or CUDA
