@@ -262,10 +262,15 @@ COWA_API int cowa_decode(const cowa_shape_t *shape, cowa_quad_t quad, float soft
  *   COWA_DECODE_NOALLOC_SCRATCH_BYTES bytes inside the library, which every
  *   GPU that loads the library holds until the process exits.  Shapes whose
  *   partials (cowa_decode_workspace_size) exceed it are refused with
- *   COWA_ERR_WORKSPACE and a detail message; nothing is launched then.
- *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.  Every call on a device shares the one array:
+ *   COWA_ERR_WORKSPACE and a detail message; nothing is launched then.  The
+ *   split count, hence the size, depends on the device's SM count: a caller
+ *   can check cowa_decode_workspace_size(shape, quad) <=
+ *   COWA_DECODE_NOALLOC_SCRATCH_BYTES on the target device ahead of time.
+ *   The first call in a CUDA context (the device's primary context, another
+ *   context a host runtime makes current, or a new primary context after a
+ *   device reset) looks up the array's device address in that context
+ *   (cudaGetSymbolAddress) and keeps it under the context's ID; make that
+ *   first call before any stream capture.  Every call on a device shares the one array:
  *   calls whose kernels overlap on the GPU (different streams, no ordering
  *   between them) race on it and must not be issued.  The array keeps the
  *   last call's partials; each call overwrites every partial it reads.
@@ -280,8 +285,10 @@ COWA_API int cowa_decode_noalloc(const cowa_shape_t *shape, cowa_quad_t quad, fl
  * Visible-tile classes of one KV head, as the training kernels see them, for
  * checking the schedule: writes out[qt * nkt + kt] (device, uint8) for the
  * tiling BM x BN, BM in {32, 64, 128} and BN in {64, 96, 128} (the forward
- * uses 128 x 96 for d = 64 and 128 x 64 for d = 128, the backward 64 x 64
- * and, key-tile major, 32 or 64 x 64),
+ * uses query tiles of 128 with key tiles of 96 for d = 64 and 64 for
+ * d = 128; the dQ pass query tiles of 128 with key tiles of 64; the dK/dV
+ * pass, key-tile major, key tiles of 128 with query tiles of 64 for d = 64
+ * and 32 for d = 128),
  * nqt = ceil(Lq/BM), nkt = ceil(Lk/BN):
  *   0 = tile skipped, 1 = visited with the element mask applied,
  *   2 = visited without a mask (every in-range pair visible).

@@ -182,6 +182,94 @@ def bwd_dkv_cols(q, k, v, dout, quad, cols, scale=None, kv_head_offset=0, widx=N
     return dk, dv
 
 
+def _visible_np(p, j, w, quad):
+    """The mask rule of ``cowa_ref_visible`` on numpy arrays (broadcasting):
+    key j visible from aligned position p under window index w iff
+    d = p - j >= 0 and (j < S or d < N or N+G+w*W <= d < N+G+(w+1)*W)."""
+    S, N, G, W = (int(x) for x in quad)
+    d = p - j
+    c = N + G + w * W
+    return (d >= 0) & (j >= 0) & ((j < S) | (d < N) | ((d >= c) & (d < c + W)))
+
+
+def bwd_dkv_cols_fast(q, k, v, dout, quad, cols, scale=None, kv_head_offset=0, chunk=256):
+    """dK, dV of selected key columns [(b, hkv, j), ...] -> ([n, d], [n, d]),
+    the same definitions as ``bwd_dkv_cols`` with numpy matrix products for
+    the scores and the PV sums of whole chunks of rows (every row's softmax is
+    still taken over exactly its visible keys, in fp64).  For the full-size
+    workloads, where a sink column is seen by every query row: each of those
+    rows needs its own LSE and O, which the per-row C loops cannot afford.
+
+    Per KV head h of a column, over the rows i (of the g query heads of the
+    group) that see column j: s_il = scale <q_i, k_l> on the row's visible
+    keys l, LSE_i = log sum_l exp(s_il), P_il = exp(s_il - LSE_i),
+    O_i = sum_l P_il v_l, delta_i = <dO_i, O_i>, dP_ij = <dO_i, v_j>,
+    dS_ij = P_ij (dP_ij - delta_i); dK_j = scale sum_i dS_ij q_i,
+    dV_j = sum_i P_ij dO_i."""
+    def widen(x):  # slices are widened when taken: a full-size fp64 copy would not fit
+        x = np.asarray(x)
+        return (lambda *i: bits_to_f64(x[i])) if x.dtype == np.uint16 else (lambda *i: np.asarray(x[i], np.float64))
+
+    qf, kf, vf, df = (widen(x) for x in (q, k, v, dout))
+    B, Lq, Hq, D = np.shape(q)
+    Lk, Hkv = np.shape(k)[1], np.shape(k)[2]
+    g = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    S, N, G, W = (int(x) for x in quad)
+    cols = [tuple(int(a) for a in c) for c in cols]
+    dk = np.zeros((len(cols), D))
+    dv = np.zeros((len(cols), D))
+    by_head = {}
+    for n, (b, h, j) in enumerate(cols):
+        by_head.setdefault((b, h), []).append((n, j))
+    shift = Lk - Lq
+    for (b, h), members in by_head.items():
+        w = h + int(kv_head_offset)
+        p_all = np.arange(Lq, dtype=np.int64) + shift
+        js = np.array([j for _, j in members], dtype=np.int64)
+        sees = _visible_np(p_all[:, None], js[None, :], w, quad)  # [Lq, ncols]
+        rows = np.nonzero(sees.any(axis=1))[0]
+        for r0 in range(0, len(rows), chunk):
+            ri = rows[r0:r0 + chunk]
+            pr = ri + shift
+            # candidate keys: the union over the chunk's rows of the sink
+            # [0, S), near [p-N+1, p] and long [p-e+1, p-c] ranges (c =
+            # N+G+w*W, e = c+W), a superset of every row's visible keys; each
+            # row's own mask is then the rule itself
+            lo, hi = int(pr.min()), int(pr.max())
+            c = N + G + w * W
+            parts = [np.arange(0, min(S, hi + 1, Lk)),
+                     np.arange(max(0, lo - N + 1), min(hi + 1, Lk)),
+                     np.arange(max(0, lo - (c + W) + 1), min(hi - c + 1, Lk))]
+            kidx = np.unique(np.concatenate([x for x in parts if x.size] or [np.zeros(0, np.int64)]))
+            m = _visible_np(pr[:, None], kidx[None, :], w, quad)
+            kk, vv = kf(b, kidx, h), vf(b, kidx, h)
+            kcol = {j: (kf(b, j, h), vf(b, j, h)) for _, j in members}
+            for hq in range(h * g, (h + 1) * g):
+                qi, di = qf(b, ri, hq), df(b, ri, hq)
+                s = scale * (qi @ kk.T)
+                s[~m] = -np.inf
+                mx = s.max(axis=1, keepdims=True)
+                np.subtract(s, mx, out=s)
+                np.exp(s, out=s)  # exp(s - max): 0 off the mask
+                tot = s.sum(axis=1)
+                lse = mx[:, 0] + np.log(tot)
+                o = (s @ vv) / tot[:, None]  # sum_l P_il v_l with P = exp(s - LSE)
+                delta = (di * o).sum(axis=1)
+                for n, j in members:
+                    sel = _visible_np(pr, j, w, quad)
+                    if not sel.any():
+                        continue
+                    kj, vj = kcol[j]
+                    pij = np.exp(scale * (qi[sel] @ kj) - lse[sel])
+                    dpij = di[sel] @ vj
+                    dsij = pij * (dpij - delta[sel])
+                    dk[n] += scale * (dsij @ qi[sel])
+                    dv[n] += pij @ di[sel]
+    return dk, dv
+
+
 def decode(q, k_cache, v_cache, seqlens, quad, scale=None, kv_head_offset=0,
            widx=None):
     """Single-token decode: q [B,Hq,d], caches [B,Lcap,Hkv,d], seqlens [B].
@@ -240,4 +328,4 @@ def bits_to_f64(bits) -> np.ndarray:
 
 
 __all__ = ["threads", "default_quad", "visible", "mask", "tile_counts", "fwd", "fwd_rows", "bwd",
-           "bwd_dq_rows", "bwd_dkv_cols", "decode", "window_keys", "bf16_bits", "bits_to_f64"]
+           "bwd_dq_rows", "bwd_dkv_cols", "bwd_dkv_cols_fast", "decode", "window_keys", "bf16_bits", "bits_to_f64"]

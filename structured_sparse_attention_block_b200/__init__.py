@@ -34,7 +34,9 @@ __all__ = ["CowaError", "cowa_fwd", "cowa_bwd", "cowa_decode", "cowa_default_qua
            "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "libcowa.so")
+# COWA_DEBUG=1 selects the checking build (index checks in the kernels,
+# failed checks reported as COWA_ERR_DEVICE); see build.py
+_LIB_PATH = os.path.join(_HERE, "libcowa_debug.so" if os.environ.get("COWA_DEBUG") == "1" else "libcowa.so")
 _lib = None
 
 COWA_OK = 0
@@ -76,13 +78,14 @@ def library_path() -> str:
 
 
 def lib():
-    """The loaded ``libcowa.so``; raises if it has not been built."""
+    """The loaded ``libcowa.so`` (``libcowa_debug.so`` under COWA_DEBUG=1);
+    raises if it has not been built."""
     global _lib
     if _lib is None:
         if not os.path.exists(_LIB_PATH):
             raise RuntimeError(
-                "libcowa.so is missing at %s: build it with "
-                "`python -m structured_sparse_attention_block_b200.build`" % _LIB_PATH)
+                "%s is missing: build it with `python -m structured_sparse_attention_block_b200.build%s`"
+                % (_LIB_PATH, " --debug" if _LIB_PATH.endswith("_debug.so") else ""))
         L = ctypes.CDLL(_LIB_PATH)
         vp, sz, i32, i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64
         SP = ctypes.POINTER(Shape)

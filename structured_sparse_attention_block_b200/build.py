@@ -4,6 +4,13 @@ Each ``csrc/*.cu`` is compiled by nvcc for ``arch=compute_100a,code=sm_100a``
 into ``_build/`` and linked into a shared library next to this file, so the
 binary travels with the source tree.  Run ``python -m
 structured_sparse_attention_block_b200.build`` or call ``build()``.
+
+``build(debug=True)`` (``--debug``) builds the checking variant
+``libcowa_debug.so`` from the same sources with ``-DCOWA_DEBUG`` (objects in
+``_build_debug/``): its kernels check tile, row and workspace indices against
+the extents they must stay within and report a failed check as
+COWA_ERR_DEVICE instead of making the access.  The binding loads it instead
+of ``libcowa.so`` when the environment sets ``COWA_DEBUG=1``.
 """
 import concurrent.futures
 import os
@@ -14,6 +21,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libcowa.so")
+OUT_DEBUG = os.path.join(HERE, "_build_debug")
+LIB_DEBUG = os.path.join(HERE, "libcowa_debug.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 NVCC_FLAGS = [
@@ -42,8 +51,8 @@ def _deps():
     return files
 
 
-def _compile(src, extra, verbose):
-    obj = os.path.join(OUT, os.path.basename(src)[:-3] + ".o")
+def _compile(src, extra, verbose, out=OUT):
+    obj = os.path.join(out, os.path.basename(src)[:-3] + ".o")
     cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
@@ -53,25 +62,28 @@ def _compile(src, extra, verbose):
     return obj, res.stderr
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    """Compile every kernel source and link ``libcowa.so``; return its path."""
-    if not force and os.path.exists(LIB):
+def build(force: bool = False, verbose: bool = False, extra=(), debug: bool = False) -> str:
+    """Compile every kernel source and link ``libcowa.so`` (``debug``: the
+    checking variant ``libcowa_debug.so``); return its path."""
+    lib, out = (LIB_DEBUG, OUT_DEBUG) if debug else (LIB, OUT)
+    extra = list(extra) + (["-DCOWA_DEBUG"] if debug else [])
+    if not force and os.path.exists(lib):
         newest = max(os.path.getmtime(f) for f in _deps())
-        if os.path.getmtime(LIB) >= newest:
-            return LIB
-    os.makedirs(OUT, exist_ok=True)
+        if os.path.getmtime(lib) >= newest:
+            return lib
+    os.makedirs(out, exist_ok=True)
     with concurrent.futures.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
-        results = list(ex.map(lambda s: _compile(s, list(extra), verbose), sources()))
+        results = list(ex.map(lambda s: _compile(s, extra, verbose, out), sources()))
     if verbose:
         for _, log in results:
             sys.stderr.write(log)
-    tmp = LIB + ".tmp.%d" % os.getpid()
+    tmp = lib + ".tmp.%d" % os.getpid()
     cmd = [_nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
            "-o", tmp, *[o for o, _ in results], "-lcudart"]
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

@@ -90,7 +90,6 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const AttnParams p, float
     if (live && piece == 0) lsd[row] = make_float2(nl, nl == -CUDART_INF_F ? 0.f : -s);
 }
 
-// bitmask of bit positions [lo, hi] within 0..31 (empty when lo > hi)
 // ------------------------------------------------------------------ dK/dV --
 struct BwdArgs {
     CUtensorMap tq, tk, tv, tdo;
@@ -100,19 +99,31 @@ struct BwdArgs {
     int npair;
 };
 
+// Tensor-memory plan of a dK/dV CTA (512 columns, 128 lanes = its keys):
+//   [0, D)            dK accumulator (fp32)
+//   [D, 2D)           dV accumulator (fp32)
+//   [2D, 2D + D/2)    K of the CTA's keys, bf16 pairs: the A operand of S^T
+//   [2D + D/2, 3D)    V, the A operand of dP^T
+//   [3D, 3D + BM)     S^T of the current task (fp32)
+//   [3D + BM, 3D+2BM) dP^T of the current task
+//   3D + 2BM + x*BM   P^T (BM/2 columns of bf16 pairs), then dS^T, of the
+//                     tasks of warpgroup x
+// D = 128: BM = 32 ends at 512; D = 64: BM = 64 ends at 448.
 template <int D>
 struct KvCfg {
     static constexpr int BN = kBwd5KeyTile;  // keys per CTA
     static constexpr int BM = bwd5_kv_bm(D);  // queries per task
-    static constexpr int ST = D == 64 ? 8 : 4;  // Q/dO stages (d = 64: 8 measured 2 % faster than 6, 4 % than 4)
+    static constexpr int ST = 8;              // Q/dO stages
     static constexpr int KB = D / 64;
     static constexpr int KV_BYTES = BN * D * 2;
     static constexpr int QT_BYTES = BM * D * 2;
     static constexpr int LSD_BYTES = BM * 8;
     static constexpr int STAGE_BYTES = (2 * QT_BYTES + LSD_BYTES + 1023) / 1024 * 1024;
-    // tensor memory: dK, dV, then two buffers of S^T, dP^T, P^T (bf16), dS^T (bf16)
-    static constexpr int T_DK = 0, T_DV = D, T_BUF = 2 * D, BUF = 3 * BM;
-    static constexpr int NBAR = 12 + 2 * ST;
+    static constexpr int T_DK = 0, T_DV = D, T_K = 2 * D, T_V = 2 * D + D / 2;
+    static constexpr int T_S = 3 * D, T_DP = 3 * D + BM;
+    static constexpr __host__ __device__ int t_pd(int x) { return 3 * D + 2 * BM + x * BM; }
+    static_assert(3 * D + 4 * BM <= 512, "tensor-memory plan exceeds 512 columns");
+    static constexpr int NBAR = 13 + 2 * ST;
     static constexpr int SMEM = 1024 + 2 * KV_BYTES + ST * STAGE_BYTES + 8 * NBAR + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BM, 0, 0);
     static constexpr uint32_t IDESC_G = idesc_bf16(128, D, 0, 1);
@@ -147,6 +158,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
     auto FIN = [&](int r) { return bar0 + 8u * (r == 0 ? 6 + 2 * ST : 11 + 2 * ST); };  // per issuer
     auto S_FREE = [&](int x) { return bar0 + 8u * (7 + 2 * ST + x); };
     auto G_DONE = [&](int x) { return bar0 + 8u * (9 + 2 * ST + x); };
+    const uint32_t KV_TM = bar0 + 8u * (12 + 2 * ST);  // K and V are in tensor memory
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const TilePos pos = tile_pos(p.Hkv, p.B);
@@ -189,6 +201,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
         mbar_init(DONE, 1);
         mbar_init(FIN(0), 1);
         mbar_init(FIN(1), 1);
+        mbar_init(KV_TM, 8);  // one arrival per elementwise warp
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -221,6 +234,13 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
                 if (u >= ST && !mbar_wait(Q_EMPTY(s), ((u / ST) - 1) & 1, p.err, abort_flag)) break;
                 int hq, qt;
                 task(u, hq, qt);
+                // a listed query tile holds rows; its row pairs lie in the workspace
+                if (!dcheck(qt >= 0 && qt * BM < sg.Lq && (qt + 1) * BM <= a.lq_pad && hq >= hl * p.g &&
+                                hq < (hl + 1) * p.g,
+                            p.err)) {
+                    *abort_flag = 1;
+                    break;
+                }
                 mbar_expect_tx(Q_FULL(s), 2 * C::QT_BYTES + C::LSD_BYTES);
                 for (int kb = 0; kb < KB; ++kb) {
                     tma_load_4d(stage_q(s) + kb * BM * 128, &a.tq, Q_FULL(s), kb * 64, sg.qoff + qt * BM, hq, sg.tb);
@@ -238,28 +258,28 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
     } else if (warp == 9 || warp == 10) {
         // ------------------------------------------------------------ MMA
         // the whole warp runs the loop; one elected lane issues.  Warp 9
-        // issues the score MMAs, warp 10 the gradient MMAs.
+        // issues the score MMAs, warp 10 the gradient MMAs.  Every A operand
+        // comes from tensor memory (K, V, P^T, dS^T): only Q and dO are read
+        // from shared memory.
         const uint32_t FULL = 0xffffffffu;
         const int role = warp - 9;
-        bool ok = __all_sync(FULL, mbar_wait(KV_LOADED, 0, p.err, abort_flag));
-        const uint64_t dk0 = sdesc(sK, 16, 1024), dv0 = sdesc(sV, 16, 1024);
+        bool ok = __all_sync(FULL, mbar_wait(KV_TM, 0, p.err, abort_flag));
+        tc_fence_after();
         const uint64_t dq0 = sdesc(stage_q(0), 16, 1024), ddo0 = sdesc(stage_do(0), 16, 1024);
         const uint64_t dqm0 = sdesc(stage_q(0), BM * 128, 1024), ddom0 = sdesc(stage_do(0), BM * 128, 1024);
-        auto sdp = [&](int u) -> bool {  // S^T, dP^T of task u into buffer u % 2
-            const int s = u % ST, x = u & 1;
+        auto sdp = [&](int u) -> bool {  // S^T, dP^T of task u
+            const int s = u % ST;
             if (!__all_sync(FULL, mbar_wait(Q_FULL(s), (u / ST) & 1, p.err, abort_flag))) return false;
             tc_fence_after();
-            const uint32_t tb = tmem + C::T_BUF + x * C::BUF;
             const uint32_t so = (uint32_t)s * C::STAGE_BYTES;
             if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t ko = (kk >> 2) * BN * 128 + (kk & 3) * 32;
                     const uint32_t qo = so + (kk >> 2) * BM * 128 + (kk & 3) * 32;
-                    mma_ss(tb, sdesc_add(dk0, ko), sdesc_add(dq0, qo), C::IDESC_S, kk > 0);
-                    mma_ss(tb + BM, sdesc_add(dv0, ko), sdesc_add(ddo0, qo), C::IDESC_S, kk > 0);
+                    mma_ts(tmem + C::T_S, tmem + C::T_K + kk * 8, sdesc_add(dq0, qo), C::IDESC_S, kk > 0);
+                    mma_ts(tmem + C::T_DP, tmem + C::T_V + kk * 8, sdesc_add(ddo0, qo), C::IDESC_S, kk > 0);
                 }
-                mma_commit(S_FULL(x));
+                mma_commit(S_FULL(u & 1));
             }
             __syncwarp();
             return true;
@@ -268,15 +288,14 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
             const int s = u % ST, x = u & 1;
             if (!__all_sync(FULL, mbar_wait(P_FULL(x), (u >> 1) & 1, p.err, abort_flag))) return false;
             tc_fence_after();
-            const uint32_t tb = tmem + C::T_BUF + x * C::BUF;
+            const uint32_t tb = tmem + C::t_pd(x);
             const uint32_t so = (uint32_t)s * C::STAGE_BYTES;
             if (elect_one()) {
 #pragma unroll
                 for (int k2 = 0; k2 < BM / 16; ++k2) {
                     const uint32_t acc = (u > 0 || k2 > 0) ? 1u : 0u;
-                    mma_ts(tmem + C::T_DV, tb + 2 * BM + k2 * 8, sdesc_add(ddom0, so + k2 * 2048), C::IDESC_G, acc);
-                    mma_ts(tmem + C::T_DK, tb + 2 * BM + BM / 2 + k2 * 8, sdesc_add(dqm0, so + k2 * 2048), C::IDESC_G,
-                           acc);
+                    mma_ts(tmem + C::T_DV, tb + k2 * 8, sdesc_add(ddom0, so + k2 * 2048), C::IDESC_G, acc);
+                    mma_ts(tmem + C::T_DK, tb + BM / 2 + k2 * 8, sdesc_add(dqm0, so + k2 * 2048), C::IDESC_G, acc);
                 }
                 mma_commit(Q_EMPTY(s));
                 mma_commit(G_DONE(x));
@@ -286,9 +305,11 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
         };
         if (role == 0) {
             for (int u = 0; ok && u < ntask; ++u) {
-                if (u >= 2) {
-                    // warpgroup u % 2 has read S^T and dP^T of task u-2
-                    if (!(ok = __all_sync(FULL, mbar_wait(S_FREE(u & 1), ((u - 2) >> 1) & 1, p.err, abort_flag))))
+                if (u >= 1) {
+                    // S^T and dP^T have one region: the warpgroup of task u-1
+                    // has read those of task u-1
+                    const int xp = (u - 1) & 1;
+                    if (!(ok = __all_sync(FULL, mbar_wait(S_FREE(xp), ((u - 1) >> 1) & 1, p.err, abort_flag))))
                         break;
                     tc_fence_after();
                 }
@@ -308,7 +329,32 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
         const int jl = (warp & 3) * 32 + lane;  // key row within the tile
         const int jg = c0 + jl;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tb = tmem + C::T_BUF + x * C::BUF + lane_off;
+        // K (warpgroup 0) or V (warpgroup 1) of this key into tensor memory:
+        // row jl of the 128-byte-swizzled tile, 16-byte chunk c of each
+        // 64-element block stored at chunk c ^ (jl % 8)
+        bool ok = __all_sync(0xffffffffu, mbar_wait(KV_LOADED, 0, p.err, abort_flag));
+        {
+            const unsigned char *src = sm + (x == 0 ? 0 : C::KV_BYTES) + jl * 128;
+            const uint32_t dst = tmem + (x == 0 ? C::T_K : C::T_V) + lane_off;
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb) {
+                uint32_t r[32];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v4 = *reinterpret_cast<const uint4 *>(src + kb * BN * 128 + ((c ^ (jl & 7)) * 16));
+                    r[4 * c] = v4.x;
+                    r[4 * c + 1] = v4.y;
+                    r[4 * c + 2] = v4.z;
+                    r[4 * c + 3] = v4.w;
+                }
+                tmem_st32(dst + kb * 32, r);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(KV_TM);
+        }
+        const uint32_t tS = tmem + C::T_S + lane_off, tPD = tmem + C::t_pd(x) + lane_off;
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
         // the aligned positions that see key jg (sink, near, long), as runs
         // formed once: a task's columns need no mask when one run holds them
@@ -317,8 +363,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
         // and position t in the key tile's query-tile list, advanced without
         // division
         int gi = nq > 0 ? x / nq : 0, tq = nq > 0 ? x % nq : 0;
-        bool ok = true;
-        for (int k = 0;; ++k) {
+        for (int k = 0; ok; ++k) {
             const int u = 2 * k + x;
             if (u >= ntask) break;
             // task set-up, independent of the scores: done while they land
@@ -344,14 +389,16 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
             ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), k & 1, p.err, abort_flag));
             if (!ok) break;
             tc_fence_after();
+            // S^T and dP^T in 32-column chunks; once the last chunk is in
+            // registers the region is released for the next task's scores
+            // (d = 128: the whole task is one chunk)
 #pragma unroll
             for (int c = 0; c < BM / 32; ++c) {
                 uint32_t sr[32], dr[32];
-                tmem_ld32(tb + c * 32, sr);
-                tmem_ld32(tb + BM + c * 32, dr);
+                tmem_ld32(tS + c * 32, sr);
+                tmem_ld32(tS + BM + c * 32, dr);
                 tmem_wait_ld();
                 if (c == BM / 32 - 1) {
-                    // all of S^T and dP^T read: S^T/dP^T of task u+2 may land
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(S_FREE(x));
@@ -361,6 +408,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
                     for (int e = 0; e < 32; ++e)
                         if (!((vis[c] >> e) & 1u)) sr[e] = __float_as_uint(-CUDART_INF_F);
                 }
+                // P^T and dS^T as bf16 pairs: entry e holds columns 2e, 2e+1
                 uint32_t pk[16], dk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -375,14 +423,15 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
                     dk[e] = pack2(ds.x, ds.y);
                 }
                 if (c == 0 && k > 0) {
-                    // the gradient MMAs of task u-2 read P^T/dS^T of this buffer
-                    // (G_DONE(x) has completed k-1 or k phases)
+                    // the gradient MMAs of this warpgroup's previous task read
+                    // its P^T/dS^T columns (G_DONE(x) has completed k-1 or k
+                    // phases)
                     ok = __all_sync(0xffffffffu, mbar_wait(G_DONE(x), (k - 1) & 1, p.err, abort_flag));
                     if (!ok) break;
                     tc_fence_after();
                 }
-                tmem_st16(tb + 2 * BM + c * 16, pk);
-                tmem_st16(tb + 2 * BM + BM / 2 + c * 16, dk);
+                tmem_st16(tPD + c * 16, pk);
+                tmem_st16(tPD + BM / 2 + c * 16, dk);
             }
             if (!ok) break;
             tmem_wait_st();
@@ -413,7 +462,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
             uint32_t pk[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) pk[e] = pack2(__uint_as_float(g[2 * e]) * f, __uint_as_float(g[2 * e + 1]) * f);
-            if (jg < sg.Lk) {
+            if (jg < sg.Lk && dcheck(sg.koff + jg < (p.cu_q ? p.total_k : p.Lk), p.err)) {
                 uint4 *dst = reinterpret_cast<uint4 *>(grow_ + c * 16);
                 dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
@@ -547,6 +596,10 @@ __global__ void __launch_bounds__(352, 1) dq_sm100_kernel(const __grid_constant_
                 const int s = t % ST;
                 if (t >= ST && !mbar_wait(KV_EMPTY(s), ((t / ST) - 1) & 1, p.err, abort_flag)) break;
                 const int kt = tile_of(t);
+                if (!dcheck(kt >= 0 && kt * BN < sg.Lk, p.err)) {  // a listed tile holds keys
+                    *abort_flag = 1;
+                    break;
+                }
                 mbar_expect_tx(KV_FULL(s), C::STAGE_BYTES);
                 const uint32_t sk = sStage + s * C::STAGE_BYTES, sv = sk + C::KV_BYTES;
                 for (int kb = 0; kb < KB; ++kb) {
@@ -633,7 +686,7 @@ __global__ void __launch_bounds__(352, 1) dq_sm100_kernel(const __grid_constant_
         const bool active = x < nslot;
         const int hq = hq0 + x;
         float nl = -CUDART_INF_F, nd = 0.f;
-        if (active && i0 + r < sg.Lq) {
+        if (active && i0 + r < sg.Lq && dcheck(i0 + r < a.lq_pad, p.err)) {
             const float2 v = a.lsd[((long long)b * p.Hq + hq) * a.lq_pad + i0 + r];
             nl = v.x;
             nd = v.y;
@@ -722,11 +775,320 @@ __global__ void __launch_bounds__(352, 1) dq_sm100_kernel(const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
                     pk[e] = pack2(__uint_as_float(g[2 * e]) * p.scale, __uint_as_float(g[2 * e + 1]) * p.scale);
-                if (r < nrows) {
+                if (r < nrows && dcheck(sg.qoff + i0 + r < (p.cu_q ? p.total_q : p.Lq), p.err)) {
                     uint4 *dst = reinterpret_cast<uint4 *>(drow + c * 16);
                     dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------ dQ, d = 128 --
+// Query-tile major with Q and dO resident in tensor memory: S = Q K^T and
+// dP = dO V^T take their A operands from there, dQ += dS K takes dS from
+// there, so every MMA reads only K or V from shared memory.  One query head
+// per CTA, key tiles of 64.  Both elementwise warpgroups work on every tile,
+// warpgroup x on key columns [32x, 32x + 32): a row's dS needs no statistic
+// of the other columns, so the split costs no exchange and halves the time
+// from scores to dS.  Tensor memory (512 columns, lanes = query rows):
+//   [0, 128) dQ (fp32), [128, 192) Q, [192, 256) dO (bf16 pairs),
+//   [256, 320) S, [320, 384) dP, 384 + 32y dS of the tiles t with t % 2 = y.
+// Order per tile t: S(t), dP(t) once both warpgroups hold S(t-1) and dP(t-1)
+// in registers (S_FREE); dQ += dS(t) K_t once dS(t) is written (DS_FULL);
+// dS(t+2) is written after dQ(t) completes (DONE).
+struct DqTmCfg {
+    static constexpr int D = 128, BM = kBwd5QTile, BN = 64;
+    static constexpr int ST = 4;
+    static constexpr int KB = D / 64;
+    static constexpr int QT_BYTES = BM * D * 2;
+    static constexpr int KV_BYTES = BN * D * 2;
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+    static constexpr int T_DQ = 0, T_Q = 128, T_DO = 192, T_S = 256, T_DP = 320;
+    static constexpr __host__ __device__ int t_ds(int y) { return 384 + 32 * y; }
+    static constexpr int NBAR = 12 + 2 * ST;
+    static constexpr int SMEM = 1024 + 2 * QT_BYTES + ST * STAGE_BYTES + 8 * NBAR + 16;
+    static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
+    static constexpr uint32_t IDESC_Q = idesc_bf16(128, D, 0, 1);
+};
+
+__global__ void __launch_bounds__(352, 1) dq_tm_kernel(const __grid_constant__ BwdArgs a)
+{
+    using C = DqTmCfg;
+    constexpr int D = C::D, BM = C::BM, BN = C::BN, ST = C::ST, KB = C::KB;
+    const AttnParams &p = a.p;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char *sm = smem_raw + (base - raw);
+    const uint32_t sQ = base, sDO = base + C::QT_BYTES, sStage = base + 2 * C::QT_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 2 * C::QT_BYTES + ST * C::STAGE_BYTES);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const uint32_t bar0 = smem_addr(bars);
+    const uint32_t BAR_Q = bar0;
+    auto KV_FULL = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto KV_EMPTY = [&](int s) { return bar0 + 8u * (1 + ST + s); };
+    const uint32_t S_FULL = bar0 + 8u * (1 + 2 * ST);
+    const uint32_t S_FREE = bar0 + 8u * (2 + 2 * ST);
+    auto DS_FULL = [&](int y) { return bar0 + 8u * (3 + 2 * ST + y); };
+    auto DONE = [&](int y) { return bar0 + 8u * (5 + 2 * ST + y); };
+    auto FIN = [&](int r) { return bar0 + 8u * (7 + 2 * ST + r); };
+    const uint32_t QD_TM = bar0 + 8u * (9 + 2 * ST);  // Q and dO are in tensor memory
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const TilePos pos = tile_pos(p.Hq, p.B);
+    const int qt = p.nqt - 1 - pos.step;  // long rows first
+    const int hq = pos.slot, hl = hq / p.g;
+    const int b = pos.b;
+    const SeqGeom sg = seq_geom(p, b);
+    const int i0 = qt * BM;
+    if (i0 >= sg.Lq) return;  // past the end of this sequence of a packed batch
+    const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
+    const int delta_pos = sg.Lk - sg.Lq;
+    const int nrows = min(BM, sg.Lq - i0);
+    const int pa = i0 + delta_pos, pb = i0 + nrows - 1 + delta_pos;
+
+    // the key tiles this query tile visits, from the same closed form as the
+    // schedule builder
+    const TileRanges tr = query_tile_ranges(pa, pb, w, BN);
+    const int nr = tr.n;
+    const int lo0 = tr.lo0, lo1 = tr.lo1, lo2 = tr.lo2;
+    const int len0 = tr.len0, len1 = tr.len1, len2 = tr.len2;
+    const int ntiles = (nr > 0 ? len0 : 0) + (nr > 1 ? len1 : 0) + (nr > 2 ? len2 : 0);
+    auto tile_of = [&](int t) {
+        if (t < len0 || nr == 1) return lo0 + t;
+        t -= len0;
+        if (t < len1 || nr == 2) return lo1 + t;
+        return lo2 + t - len1;
+    };
+
+    if (tid == 0) {
+        mbar_init(BAR_Q, 1);
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(KV_FULL(s), 1);
+            mbar_init(KV_EMPTY(s), 1);
+        }
+        mbar_init(S_FULL, 1);
+        mbar_init(S_FREE, 8);  // one arrival per elementwise warp
+        for (int y = 0; y < 2; ++y) {
+            mbar_init(DS_FULL(y), 256);
+            mbar_init(DONE(y), 1);
+            mbar_init(FIN(y), 1);
+        }
+        mbar_init(QD_TM, 8);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_addr(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tmap(&a.tq);
+        prefetch_tmap(&a.tk);
+        prefetch_tmap(&a.tv);
+        prefetch_tmap(&a.tdo);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ TMA
+        if (lane == 0) {
+            mbar_expect_tx(BAR_Q, 2 * C::QT_BYTES);
+            for (int kb = 0; kb < KB; ++kb) {
+                tma_load_4d(sQ + kb * BM * 128, &a.tq, BAR_Q, kb * 64, sg.qoff + i0, hq, sg.tb);
+                tma_load_4d(sDO + kb * BM * 128, &a.tdo, BAR_Q, kb * 64, sg.qoff + i0, hq, sg.tb);
+            }
+            int issued = 0;
+            for (int t = 0; t < ntiles; ++t) {
+                const int s = t % ST;
+                if (t >= ST && !mbar_wait(KV_EMPTY(s), ((t / ST) - 1) & 1, p.err, abort_flag)) break;
+                const int kt = tile_of(t);
+                if (!dcheck(kt >= 0 && kt * BN < sg.Lk, p.err)) {  // a listed tile holds keys
+                    *abort_flag = 1;
+                    break;
+                }
+                mbar_expect_tx(KV_FULL(s), C::STAGE_BYTES);
+                const uint32_t sk = sStage + s * C::STAGE_BYTES, sv = sk + C::KV_BYTES;
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_4d(sk + kb * BN * 128, &a.tk, KV_FULL(s), kb * 64, sg.koff + kt * BN, hl, sg.tb);
+                    tma_load_4d(sv + kb * BN * 128, &a.tv, KV_FULL(s), kb * 64, sg.koff + kt * BN, hl, sg.tb);
+                }
+                issued = t + 1;
+            }
+            mbar_wait(BAR_Q, 0, p.err, abort_flag);
+            for (int t = issued > ST ? issued - ST : 0; t < issued; ++t)
+                mbar_wait(KV_FULL(t % ST), (t / ST) & 1, p.err, abort_flag);
+        }
+    } else if (warp == 9 || warp == 10) {
+        // ------------------------------------------------------------ MMA
+        // the whole warp runs the loop; one elected lane issues.  Warp 9
+        // issues S and dP, warp 10 the dQ MMAs (the accumulator's only writer).
+        const uint32_t FULL = 0xffffffffu;
+        const int role = warp - 9;
+        bool ok = __all_sync(FULL, mbar_wait(QD_TM, 0, p.err, abort_flag));
+        tc_fence_after();
+        const uint64_t dk0 = sdesc(sStage, 16, 1024), dv0 = sdesc(sStage + C::KV_BYTES, 16, 1024);
+        const uint64_t dkm0 = sdesc(sStage, BN * 128, 1024);
+        if (role == 0) {
+            for (int t = 0; ok && t < ntiles; ++t) {
+                const int s = t % ST;
+                if (!(ok = __all_sync(FULL, mbar_wait(KV_FULL(s), (t / ST) & 1, p.err, abort_flag)))) break;
+                if (t > 0 && !(ok = __all_sync(FULL, mbar_wait(S_FREE, (t - 1) & 1, p.err, abort_flag)))) break;
+                tc_fence_after();
+                const uint32_t so = (uint32_t)s * C::STAGE_BYTES;
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t ko = so + (kk >> 2) * BN * 128 + (kk & 3) * 32;
+                        mma_ts(tmem + C::T_S, tmem + C::T_Q + kk * 8, sdesc_add(dk0, ko), C::IDESC_S, kk > 0);
+                        mma_ts(tmem + C::T_DP, tmem + C::T_DO + kk * 8, sdesc_add(dv0, ko), C::IDESC_S, kk > 0);
+                    }
+                    mma_commit(S_FULL);
+                }
+                __syncwarp();
+            }
+        } else {
+            for (int t = 0; ok && t < ntiles; ++t) {
+                const int y = t & 1;
+                if (!(ok = __all_sync(FULL, mbar_wait(DS_FULL(y), (t >> 1) & 1, p.err, abort_flag)))) break;
+                tc_fence_after();
+                const uint32_t so = (uint32_t)(t % ST) * C::STAGE_BYTES;
+                if (elect_one()) {
+#pragma unroll
+                    for (int k2 = 0; k2 < BN / 16; ++k2)
+                        mma_ts(tmem + C::T_DQ, tmem + C::t_ds(y) + k2 * 8, sdesc_add(dkm0, so + k2 * 2048), C::IDESC_Q,
+                               (t > 0 || k2 > 0) ? 1u : 0u);
+                    mma_commit(DONE(y));
+                    mma_commit(KV_EMPTY(t % ST));  // S(t), dP(t) completed before dS(t) existed
+                }
+                __syncwarp();
+            }
+        }
+        if (elect_one()) mma_commit(FIN(role));
+        __syncwarp();
+        mbar_wait(FIN(role), 0, p.err, abort_flag);
+    } else {
+        // ------------------------------- dS of 32 key columns per query row
+        const int x = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        // Q (warpgroup 0) or dO (warpgroup 1) of this row into tensor memory
+        bool ok = __all_sync(0xffffffffu, mbar_wait(BAR_Q, 0, p.err, abort_flag));
+        {
+            const unsigned char *src = sm + (x == 0 ? 0 : C::QT_BYTES) + r * 128;
+            const uint32_t dst = tmem + (x == 0 ? C::T_Q : C::T_DO) + lane_off;
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb) {
+                uint32_t v[32];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v4 = *reinterpret_cast<const uint4 *>(src + kb * BM * 128 + ((c ^ (r & 7)) * 16));
+                    v[4 * c] = v4.x;
+                    v[4 * c + 1] = v4.y;
+                    v[4 * c + 2] = v4.z;
+                    v[4 * c + 3] = v4.w;
+                }
+                tmem_st32(dst + kb * 32, v);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(QD_TM);
+        }
+        const int prow = pa + r;
+        float nl = -CUDART_INF_F, nd = 0.f;
+        if (i0 + r < sg.Lq && dcheck(i0 + r < a.lq_pad, p.err)) {
+            const float2 v = a.lsd[((long long)b * p.Hq + hq) * a.lq_pad + i0 + r];
+            nl = v.x;
+            nd = v.y;
+        }
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nl2 = make_float2(nl, nl),
+                     nd2 = make_float2(nd, nd);
+        const uint32_t tS = tmem + C::T_S + x * 32 + lane_off, tDP = tmem + C::T_DP + x * 32 + lane_off;
+        // the keys row prow sees, as runs formed once: a half tile needs no
+        // mask when one run holds it for every row of the warp
+        const Runs3 rr = row_key_runs(prow, w);
+        for (int t = 0; ok && t < ntiles; ++t) {
+            // tile set-up, independent of the scores: done while they land
+            const int j0 = tile_of(t) * BN + x * 32;
+            const bool full = __all_sync(0xffffffffu, runs_cover(rr, j0, j0 + 31));
+            const uint32_t vis = full ? 0xffffffffu : runs_bits(rr, j0);
+            ok = __all_sync(0xffffffffu, mbar_wait(S_FULL, t & 1, p.err, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sr[32], dr[32];
+            tmem_ld32(tS, sr);
+            tmem_ld32(tDP, dr);
+            tmem_wait_ld();
+            // S and dP of tile t are in registers: those of tile t+1 may land
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(S_FREE);
+            if (!full) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if (!((vis >> e) & 1u)) sr[e] = __float_as_uint(-CUDART_INF_F);
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
+                                             sc2, nl2);
+                const float2 pr = make_float2(fast_ex2(xa.x), fast_ex2(xa.y));
+                const float2 tt = __fadd2_rn(make_float2(__uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1])),
+                                             nd2);
+                const float2 ds = __fmul2_rn(pr, tt);
+                pk[e] = pack2(ds.x, ds.y);
+            }
+            const int y = t & 1;
+            if (t >= 2) {
+                // dQ += dS(t-2) K reads these columns (DONE(y) has completed
+                // phase (t >> 1) - 1 or is about to; never phase t >> 1)
+                ok = __all_sync(0xffffffffu, mbar_wait(DONE(y), ((t >> 1) - 1) & 1, p.err, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+            }
+            tmem_st16(tmem + C::t_ds(y) + x * 16 + lane_off, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(DS_FULL(y));
+        }
+        // the last dQ MMA: DONE of the last tile's parity
+        if (ok && ntiles > 0)
+            ok = __all_sync(0xffffffffu, mbar_wait(DONE((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1, p.err, abort_flag));
+        tc_fence_after();
+        const bool have = ok && ntiles > 0;
+        __nv_bfloat16 *drow = reinterpret_cast<__nv_bfloat16 *>(p.dq) + sg.tb * p.qs[0] +
+                              (long long)(sg.qoff + i0 + r) * p.qs[1] + hq * p.qs[2] + x * (D / 2);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {  // warpgroup x writes columns [64x, 64x + 64)
+            uint32_t g[16];
+            if (have) {
+                tmem_ld16(tmem + C::T_DQ + x * (D / 2) + c * 16 + lane_off, g);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) g[e] = 0u;
+            }
+            uint32_t pk[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                pk[e] = pack2(__uint_as_float(g[2 * e]) * p.scale, __uint_as_float(g[2 * e + 1]) * p.scale);
+            if (r < nrows && dcheck(sg.qoff + i0 + r < (p.cu_q ? p.total_q : p.Lq), p.err)) {
+                uint4 *dst = reinterpret_cast<uint4 *>(drow + c * 16);
+                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
         }
     }
@@ -744,16 +1106,14 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, i
 {
     using K = KvCfg<D>;
     using Q = DqCfg<D>;
-    static bool configured[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (!configured[dev & 63]) {
-        cudaError_t e = cudaFuncSetAttribute(dkdv_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(dq_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Q::SMEM);
-        if (e != cudaSuccess) return e;
-        configured[dev & 63] = true;
-    }
+    static std::atomic<bool> configured[64];
+    cudaError_t e = once_per_device(configured, [] {
+        cudaError_t r = cudaFuncSetAttribute(dkdv_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
+        if (r != cudaSuccess) return r;
+        return D == 128 ? cudaFuncSetAttribute(dq_tm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DqTmCfg::SMEM)
+                        : cudaFuncSetAttribute(dq_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Q::SMEM);
+    });
+    if (e != cudaSuccess) return e;
     const long long rows = (long long)p.B * p.Hq * lq_pad;
     constexpr int PREP_ROWS = 8 * (32 / (D / 8));  // rows per 256-thread block
     if (rows > 0) {
@@ -761,7 +1121,7 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, i
         bwd_prep_kernel<D><<<(unsigned)((rows + PREP_ROWS - 1) / PREP_ROWS), 256, 0, st>>>(p, lsd, lq_pad);
         launch_end(st);
     }
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
     BwdArgs a;
@@ -789,12 +1149,25 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, i
         if (e != cudaSuccess) return e;
     }
     // dQ: query tiles of 128 rows, key tiles of BN
+    const int dq_bn = D == 128 ? DqTmCfg::BN : Q::BN;
     if (!make_bshd_map(&a.tq, p.q, D, Lq_map, p.Hq, B_map, p.qs, Q::BM) ||
         !make_bshd_map(&a.tdo, p.dout, D, Lq_map, p.Hq, B_map, p.os, Q::BM) ||
-        !make_bshd_map(&a.tk, p.k, D, Lk_map, p.Hkv, B_map, p.ks, Q::BN) ||
-        !make_bshd_map(&a.tv, p.v, D, Lk_map, p.Hkv, B_map, p.vs, Q::BN))
+        !make_bshd_map(&a.tk, p.k, D, Lk_map, p.Hkv, B_map, p.ks, dq_bn) ||
+        !make_bshd_map(&a.tv, p.v, D, Lk_map, p.Hkv, B_map, p.vs, dq_bn))
         return cudaErrorInvalidValue;
     a.p.nqt = nqt_dq;
+    if (D == 128) {
+        // one query head per CTA, Q and dO resident in tensor memory
+        if (nqt_dq > 0) {
+            const unsigned g2 = tile_grid_blocks(nqt_dq, p.Hq, p.B);
+            if (!g2) return cudaErrorInvalidConfiguration;
+            launch_begin("dq_sm100", st);
+            dq_tm_kernel<<<g2, 352, DqTmCfg::SMEM, st>>>(a);
+            launch_end(st);
+            e = cudaGetLastError();
+        }
+        return e;
+    }
     a.npair = (p.g + Q::NSLOT - 1) / Q::NSLOT;
     if (nqt_dq > 0) {
         const unsigned g2 = tile_grid_blocks(nqt_dq, (long long)p.Hkv * a.npair, p.B);

@@ -123,6 +123,9 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
     // after the key loop the K/V stages are reused as the warp-merge scratch
     float *sRed = reinterpret_cast<float *>(smem_raw);
 
+    // the merge kernel may be scheduled now; it waits for this grid to
+    // complete before it reads any partial
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int split = blockIdx.x, hl = blockIdx.y, b = blockIdx.z;
     const int g = p.g;
@@ -186,6 +189,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
     auto load_kv = [&](int t, int stage) {
         int k0, nk;
         tile_at(t, k0, nk);
+        if (!dcheck(k0 >= 0 && nk >= 0 && k0 + nk <= p.Lcap, p.err)) nk = 0;  // rows of the cache only
         load_tile<D, BN, NT>(sK + stage * BN * D, kg + (long long)k0 * p.ks[1], p.ks[1], nk, tid);
         load_tile<D, BN, NT>(sV + stage * BN * D, vg + (long long)k0 * p.vs[1], p.vs[1], nk, tid);
     };
@@ -328,6 +332,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
             o += f * wo[(u * 16 + row) * D + col];
         }
         const long long pi = pbase + (long long)row * p.splits;
+        if (!dcheck(pi < (long long)p.B * p.Hq * p.splits, p.err)) break;
         p.part_o[pi * D + col] = lsum > 0.f ? o / lsum : 0.f;
         if (col == 0)  // log2-domain LSE of this split
             p.part_lse[pi] = lsum > 0.f ? m + __log2f(lsum) : -CUDART_INF_F;
@@ -341,6 +346,10 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     // reductions, then every thread merges columns with the weights from
     // shared memory (splits <= 64)
     __shared__ float red[4], wsum[4], wt[64];
+    // every partial of the split grid (the launch's programmatic
+    // predecessor, or any earlier work when launched plainly) is complete
+    // and visible past this point
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row = blockIdx.x;  // b * Hq + hq
     const int b = row / p.Hq, hq = row % p.Hq;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -466,24 +475,35 @@ static cudaError_t launch_decode_d(const DecodeParams &p, cudaStream_t st)
 {
     constexpr int smem = decode_smem_bytes(D);
     static_assert((128 + 64 * D) * 4 <= 6 * kDecBN * D * 2, "merge scratch must fit the K/V stages");
-    static bool configured[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (!configured[dev & 63]) {
-        cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured[dev & 63] = true;
-    }
+    static std::atomic<bool> configured[64];
+    cudaError_t e = once_per_device(configured, [] {
+        return cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (e != cudaSuccess) return e;
     dim3 grid(p.splits, p.Hkv, p.B);
     launch_begin("decode_split", st);
     decode_split_kernel<D><<<grid, 128, smem, st>>>(p);
     launch_end(st);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    // the merge is launched as a programmatic dependent of the split kernel:
+    // its blocks are scheduled while the splits still run (the split kernel
+    // allows it at its start) and wait on the device for the split grid to
+    // complete, so the second launch adds no gap of its own
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.B * p.Hq));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     launch_begin("decode_combine", st);
-    decode_combine_kernel<D><<<p.B * p.Hq, 128, 0, st>>>(p);
+    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, p);
     launch_end(st);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

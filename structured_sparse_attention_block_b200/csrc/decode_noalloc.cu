@@ -7,8 +7,10 @@
 // which cudaMalloc (which may synchronise the whole device) is not allowed.
 // They still pass q, the caches, seqlens, o and lse; the partial outputs of
 // the KV splits go to the static array below.
-#include <mutex>
+#include <cuda.h>
 #include <stdio.h>
+
+#include <mutex>
 
 #include "../../include/cowa.h"
 #include "kernels.cuh"
@@ -26,28 +28,71 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
 // In host code g_decode_scratch names a host-side stand-in, not the device
 // array, so the kernels get the device address that cudaGetSymbolAddress
-// reports, looked up once per device with that device current.
+// reports.  That address belongs to the CUDA context the library's module is
+// loaded in, so it is looked up once per context, with the context current,
+// and cached under the context's ID: the primary context of each device, a
+// driver-API context that a host runtime makes current instead, or the new
+// primary context after a device reset (context IDs are never reused within
+// a process, so a stale address is never handed out).
 std::mutex g_scratch_mu;
-void *g_scratch_addr[64] = {};
+struct ScratchEntry {
+    unsigned long long ctx_id;
+    void *addr;
+};
+ScratchEntry g_scratch_addr[64];
+int g_scratch_used = 0;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// ID of the current context (0 when the driver entry points are unavailable,
+// in which case the address is looked up on every call).
+unsigned long long current_context_id()
+{
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *a = nullptr, *b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+            qa == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+            qb == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+            get_id = reinterpret_cast<CtxGetIdFn>(b);
+        }
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 int scratch_address(void **out)
 {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cowa::set_error_detail(COWA_ERR_CUDA, cudaGetErrorString(e));
-    if (dev < 0 || dev >= 64) return cowa::set_error_detail(COWA_ERR_UNSUPPORTED, "device index above 63");
+    unsigned long long id = current_context_id();
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void *ptr = nullptr;
-        e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
-        if (e != cudaSuccess) {
-            char msg[256];
-            snprintf(msg, sizeof msg, "cudaGetSymbolAddress(decode scratch): %s", cudaGetErrorString(e));
-            return cowa::set_error_detail(COWA_ERR_CUDA, msg);
+    for (int i = 0; id && i < g_scratch_used; ++i)
+        if (g_scratch_addr[i].ctx_id == id) {
+            *out = g_scratch_addr[i].addr;
+            return COWA_OK;
         }
-        g_scratch_addr[dev] = ptr;
+    // (with no context current yet, the runtime makes the device's primary
+    // context current here; its ID is read again below)
+    void *ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    if (e != cudaSuccess) {
+        char msg[256];
+        snprintf(msg, sizeof msg, "cudaGetSymbolAddress(decode scratch): %s", cudaGetErrorString(e));
+        return cowa::set_error_detail(COWA_ERR_CUDA, msg);
     }
-    *out = g_scratch_addr[dev];
+    if (!id) id = current_context_id();
+    if (id) {
+        // a full table (64 contexts seen) recycles its oldest slot
+        g_scratch_addr[g_scratch_used < 64 ? g_scratch_used++ : (int)(id % 64)] = {id, ptr};
+    }
+    *out = ptr;
     return COWA_OK;
 }
 

@@ -197,6 +197,10 @@ __global__ void __launch_bounds__(352, 1) fwd_sm100_kernel(const __grid_constant
                 const int s = t % ST;
                 if (t >= ST && !mbar_wait(KV_EMPTY(s), ((t / ST) - 1) & 1, p.err, abort_flag)) break;
                 const int kt = tile_of(t);
+                if (!dcheck(kt >= 0 && kt * BN < sp.Lk, p.err)) {  // a listed tile holds keys
+                    *abort_flag = 1;
+                    break;
+                }
                 mbar_expect_tx(KV_FULL(s), 2 * C::KV_BYTES);
                 const uint32_t sk = sStage + s * C::STAGE_BYTES, sv = sk + C::KV_BYTES;
                 for (int kb = 0; kb < KB; ++kb) {
@@ -444,13 +448,13 @@ __global__ void __launch_bounds__(352, 1) fwd_sm100_kernel(const __grid_constant
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
                     pk[e] = pack2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-                if (r < nrows) {
+                if (r < nrows && dcheck(se.qoff + i0 + r < (p.cu_q ? p.total_q : p.Lq) && hq < p.Hq, p.err)) {
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 16);
                     dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
             }
-            if (r < nrows)
+            if (r < nrows && dcheck(se.qoff + i0 + r < p.lse_ld, p.err))
                 p.lse[((long long)se.tb * p.Hq + hq) * p.lse_ld + se.qoff + i0 + r] =
                     l > 0.f ? m_run * 0.69314718055994531f + logf(l) : -CUDART_INF_F;
         }
@@ -503,14 +507,11 @@ template <int D>
 static cudaError_t launch_fwd5_d(const AttnParams &p, cudaStream_t st)
 {
     using C = FwdCfg<D>;
-    static bool configured[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (!configured[dev & 63]) {
-        cudaError_t e = cudaFuncSetAttribute(fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e != cudaSuccess) return e;
-        configured[dev & 63] = true;
-    }
+    static std::atomic<bool> configured[64];
+    cudaError_t e = once_per_device(configured, [] {
+        return cudaFuncSetAttribute(fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    });
+    if (e != cudaSuccess) return e;
     FwdArgs a;
     memset(&a, 0, sizeof a);
     a.p = p;

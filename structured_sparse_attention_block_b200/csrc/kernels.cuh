@@ -6,7 +6,44 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace cowa {
+
+// One-time set-up of a device for a group of kernels (their dynamic
+// shared-memory limits): `fn` runs on the current device until it succeeds
+// once there.  Host threads that make their first call at the same time may
+// both run it, which is harmless: it only sets idempotent attributes.
+template <class F>
+cudaError_t once_per_device(std::atomic<bool> (&done)[64], F fn)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (done[dev & 63].load(std::memory_order_acquire)) return cudaSuccess;
+    e = fn();
+    if (e == cudaSuccess) done[dev & 63].store(true, std::memory_order_release);
+    return e;
+}
+
+// Checking build (compiled with -DCOWA_DEBUG into libcowa_debug.so):
+// device-side checks of tile, row and workspace indices against the extents
+// they must stay within.  A failed check records COWA_ERR_DEVICE (7) in the
+// device error word and the caller skips the guarded access (a tcgen05 CTA
+// also raises its abort flag, so its pipeline winds down through the bounded
+// waits); nothing traps.  In the release build every check is the constant
+// true and compiles away.
+__device__ __forceinline__ bool dcheck(bool ok, int *err)
+{
+#ifdef COWA_DEBUG
+    if (!ok) atomicExch(err, 7);
+    return ok;
+#else
+    (void)ok;
+    (void)err;
+    return true;
+#endif
+}
 
 struct AttnParams {
     const void *q, *k, *v;

@@ -5,12 +5,13 @@ mean-abs 1e-3 of the fp64 oracle; dQ, dK, dV within max-abs 2e-2 * max|ref|.
 LSE has no stated bound; fp32 scores of bf16 inputs give it an absolute error
 far below 2e-3, which is the bound used here.
 
-O is returned in bf16, and rounding to bf16 alone moves a value by up to half
-a unit in the last place, 2^-9 |O| (up to 0.0156 for |O| in [4, 8)).  Rows
-that see only a handful of keys (edge cases: one-key windows, the first rows
-of a dense causal mask, sharp logits) keep |O| close to a single |v|, so
-their tests pass ``out_rounding=True`` and add that half-ulp to the max-abs
-bound.  The workload tests use the plain bound.
+O is returned in bf16, rounded to nearest (ties to even) from the kernel's
+fp32 result, so the max-abs bound is applied to that fp32 value: the bf16
+output must be the rounding of some value within 1e-2 of the oracle's O,
+i.e. lie in [rne(ref - 1e-2), rne(ref + 1e-2)] (rounding is monotone).  No
+slack is added: an output outside that interval came from an fp32 value more
+than 1e-2 away.  The mean-abs bound compares with rne(ref), the exact value
+of a bf16 output.
 """
 import numpy as np
 import torch
@@ -22,22 +23,25 @@ def to64(t):
     return t.detach().float().cpu().double().numpy()
 
 
-def bf16_half_ulp(x):
-    """Half the bf16 spacing at |x| (8 significant bits)."""
+def bf16_rne(x):
+    """fp64 values rounded to bf16 (8 significant bits), nearest with ties
+    to even, in one step (no intermediate fp32 rounding); returned as fp64."""
+    x = np.asarray(x, dtype=np.float64)
     ax = np.abs(x)
-    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
-    return np.where(ax > 0, 2.0 ** (e - 8), 0.0)
+    fin = np.isfinite(x) & (ax > 0)
+    e = np.floor(np.log2(np.where(fin, ax, 1.0)))
+    ulp = 2.0 ** (e - 7)
+    return np.where(fin, np.round(x / ulp) * ulp, x)  # np.round: half to even
 
 
-def assert_o(o_gpu, o_ref, what="O", out_rounding=False):
+def assert_o(o_gpu, o_ref, what="O"):
     got = to64(o_gpu) if isinstance(o_gpu, torch.Tensor) else o_gpu
-    diff = np.abs(got - o_ref)
     assert np.isfinite(got).all(), "%s has non-finite values" % what
-    if out_rounding:
-        excess = diff - bf16_half_ulp(o_ref)
-        assert excess.max() <= O_MAX, "%s max-abs beyond output rounding %.3g > %g" % (what, excess.max(), O_MAX)
-    else:
-        assert diff.max() <= O_MAX, "%s max-abs %.3g > %g" % (what, diff.max(), O_MAX)
+    lo, hi = bf16_rne(o_ref - O_MAX), bf16_rne(o_ref + O_MAX)
+    out = np.maximum(lo - got, got - hi)  # > 0: no value within O_MAX rounds to got
+    assert out.max() <= 0, "%s: bf16 output not the rounding of a value within %g of the oracle " \
+        "(max-abs %.3g, %d elements)" % (what, O_MAX, np.abs(got - o_ref).max(), int((out > 0).sum()))
+    diff = np.abs(got - bf16_rne(o_ref))
     assert diff.mean() <= O_MEAN, "%s mean-abs %.3g > %g" % (what, diff.mean(), O_MEAN)
 
 

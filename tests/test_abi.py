@@ -32,6 +32,18 @@ def test_every_declared_symbol_is_exported(cowa):
         assert hasattr(lib, n), "missing export %s" % n
 
 
+def test_checking_build_exports_the_same_symbols(cowa):
+    """The COWA_DEBUG variant (index checks in the kernels) is a drop-in
+    replacement: it builds from the same sources and exports every entry
+    point the header declares."""
+    from structured_sparse_attention_block_b200 import build
+    path = build.build(debug=True)
+    assert path.endswith("libcowa_debug.so") and path != cowa.library_path()
+    lib = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(lib, n), "missing export %s in the checking build" % n
+
+
 def test_status_strings_and_version(cowa):
     lib = cowa.lib()
     assert lib.cowa_abi_version() == 1

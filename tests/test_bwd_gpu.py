@@ -60,15 +60,37 @@ def test_bwd_strided_and_offset_heads(oracle_mod):
 
 
 def key_columns(wl, per_head, seed):
-    """(b, h, j): the last columns (seen by few rows), one sink column and
-    one column inside each head's long window where the oracle can afford it."""
+    """(b, h, j): the last columns of every KV head, seen by few rows."""
     rng = np.random.default_rng(seed)
-    S, N, G, W = wl.quad
     cols = []
     for h in range(wl.Hkv):
         for j in range(wl.Lk - per_head, wl.Lk):
             cols.append((int(rng.integers(0, wl.B)), h, j))
     return cols
+
+
+def heavy_columns(wl, heads, sink=True):
+    """(b, h, j): a sink column (every query row sees it: the longest dK/dV
+    CTA) and a column in the middle of the long window of the last query
+    row, for each of `heads`."""
+    S, N, G, W = wl.quad
+    cols = []
+    for n, h in enumerate(heads):
+        b = n % wl.B
+        if sink and S > 0:
+            cols.append((b, h, min(S - 1, 3 + n)))
+        c = N + G + h * W
+        j = wl.Lk - 1 - (c + W // 2)
+        if W > 0 and j >= S:
+            cols.append((b, h, j))
+    return cols
+
+
+# the heavy columns: recall8k and llm14b_32k with sink columns; at op128k a
+# sink column needs every one of the 524288 (row, query head) forwards of its
+# KV head (about two minutes of the oracle), so there the long-window columns
+# are compared element by element and the sink columns through the sums below
+HEAVY = {"recall8k": ((1, 2), True), "llm14b_32k": ((0, 5), True), "op128k": ((1, 6), False)}
 
 
 @pytest.mark.parametrize("name,per_head,ncols", [("recall8k", 32, 24), ("llm14b_32k", 6, 8),
@@ -83,20 +105,26 @@ def test_bwd_workloads_sampled(oracle_mod, name, per_head, ncols):
     rq = oracle_mod.bwd_dq_rows(qb, kb, vb, db, wl.quad, rows)
     b, hq, i = (torch.tensor([r[a] for r in rows], device=q.device) for a in range(3))
     assert_grad(dq[b, i, hq], rq, "dQ rows")
-    cols = key_columns(wl, ncols, seed=3)
-    if name == "recall8k":  # the sink column and a long-window column: every row sees j=0
-        cols += [(0, 1, 0), (1, 2, wl.Lk - 1 - wl.quad[1] - 2 * wl.quad[3] - 5)]
-    rk, rv = oracle_mod.bwd_dkv_cols(qb, kb, vb, db, wl.quad, cols)
-    cb, ch, cj = (torch.tensor([c[a] for c in cols], device=q.device) for a in range(3))
-    # the tolerance scale of a sampled set is the largest gradient of the full
-    # tensor, as for the small cases
-    assert_grad(dk[cb, cj, ch], rk, "dK cols")
-    assert_grad(dv[cb, cj, ch], rv, "dV cols")
-    # a property at any size: sum_j dK_j = 0 per (b, KV head), because the
-    # outputs do not change when one vector is added to every key; bf16
-    # rounding of dK leaves a residue far below 1% of sum_j |dK_j|
-    dkf = dk.float()
+    # few-row columns through the per-column C loops, the heavy columns
+    # through the chunked form of the same definitions
+    for cols, fn in ((key_columns(wl, ncols, seed=3), oracle_mod.bwd_dkv_cols),
+                     (heavy_columns(wl, *HEAVY[name]), oracle_mod.bwd_dkv_cols_fast)):
+        rk, rv = fn(qb, kb, vb, db, wl.quad, cols)
+        cb, ch, cj = (torch.tensor([c[a] for c in cols], device=q.device) for a in range(3))
+        # the tolerance scale is the largest |gradient| among the sampled columns
+        assert_grad(dk[cb, cj, ch], rk, "dK cols %s" % cols[:2])
+        assert_grad(dv[cb, cj, ch], rv, "dV cols %s" % cols[:2])
+    # properties at any size, over every column (the sink columns included):
+    # sum_j dK_j = 0 per (b, KV head), because the outputs do not change when
+    # one vector is added to every key; sum_j dV_j = sum over the group's rows
+    # of dO, because every row's probabilities sum to one (every row of these
+    # workloads sees at least one key).  bf16 rounding of dK, dV leaves a
+    # residue far below 1 % of the sums of magnitudes.
+    dkf, dvf = dk.float(), dv.float()
     assert (dkf.sum(dim=1).abs() <= 1e-2 * dkf.abs().sum(dim=1) + 1e-6).all()
+    g = wl.Hq // wl.Hkv
+    want = do.float().sum(dim=1).view(wl.B, wl.Hkv, g, wl.d).sum(dim=2)
+    assert ((dvf.sum(dim=1) - want).abs() <= 1e-2 * dvf.abs().sum(dim=1) + 1e-3).all()
 
 
 @pytest.mark.parametrize("Lq,Lk", [(0, 200), (150, 0)])

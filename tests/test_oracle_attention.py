@@ -302,3 +302,25 @@ def test_bf16_inputs_are_widened_exactly(oracle_mod):
     back = oracle_mod.bits_to_f64(qb)
     assert (np.abs(back - q) <= np.abs(q) * 2.0 ** -8 + 1e-38).all()
     assert np.abs(back - q).max() > 0
+
+
+def test_dkv_cols_fast_equals_per_column_loops(oracle_mod):
+    """The chunked (matrix-product) dK/dV column routine that the full-size
+    GPU tests use for the heavy columns reproduces the per-column C loops
+    (themselves pinned above) on ragged shapes, offsets, gaps and chunk
+    boundaries."""
+    rng = np.random.default_rng(1)
+
+    def bf(shape):
+        x = rng.standard_normal(shape, dtype=np.float32)
+        return (x.view(np.uint32) >> 16).astype(np.uint16)
+
+    for B, Lq, Lk, Hq, Hkv, d, quad, off in [(2, 300, 300, 4, 2, 16, (5, 30, 0, 70), 0),
+                                             (1, 200, 260, 6, 3, 8, (0, 17, 4, 50), 2),
+                                             (1, 180, 150, 2, 1, 8, (3, 20, 0, 90), 0)]:
+        q, k, v, do = bf((B, Lq, Hq, d)), bf((B, Lk, Hkv, d)), bf((B, Lk, Hkv, d)), bf((B, Lq, Hq, d))
+        cols = [(b, h, j) for b in range(B) for h in range(Hkv) for j in (0, 1, 3, Lk // 2, Lk - 1, Lk - 40)]
+        rk, rv = oracle_mod.bwd_dkv_cols(q, k, v, do, quad, cols, kv_head_offset=off)
+        fk, fv = oracle_mod.bwd_dkv_cols_fast(q, k, v, do, quad, cols, kv_head_offset=off, chunk=37)
+        assert np.abs(rk - fk).max() <= 1e-12 * max(1.0, np.abs(rk).max())
+        assert np.abs(rv - fv).max() <= 1e-12 * max(1.0, np.abs(rv).max())

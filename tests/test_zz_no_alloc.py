@@ -5,8 +5,11 @@ over only input and output buffers, or a serving loop where cudaMalloc is not
 allowed) get a decode whose split scratch is a fixed array inside the
 library.  These tests call it through the C ABI and compare it with
 cowa_decode, which takes a caller workspace, on two calls in a row (the
-second call finds the first call's partials still in the array), and check
-that a shape too large for the array is refused before anything runs.
+second call finds the first call's partials still in the array), check that
+a call leaves device memory as it found it (neither torch's allocator nor the
+driver's free-memory count moves), call it once through the Python wrapper,
+and check that a shape too large for the array is refused before anything
+runs.
 """
 import ctypes
 
@@ -42,6 +45,40 @@ def test_noalloc_matches_decode_on_two_calls_in_a_row():
         assert_o(out[:, 0], to64(o_ref[:, 0]), what="noalloc O")
         diff = (lse - lse_ref).abs().max().item()
         assert diff <= LSE_ABS
+
+
+def test_noalloc_leaves_device_memory_unchanged():
+    import structured_sparse_attention_block_b200 as cowa
+    from structured_sparse_attention_block_b200.inputs import decode_inputs
+    quad = (64, 512, 0, 896)
+    q, kc, vc, sl = decode_inputs(4, 4096, 16, 4, 128, seed=5, seqlens=[4096, 3000, 100, 1])
+    out = torch.empty((4, 1, 16, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((4, 16), dtype=torch.float32, device="cuda")
+    assert noalloc_status(cowa, q, kc, vc, sl, quad, out, lse) == 0  # first call: set-up
+    torch.cuda.synchronize()
+    alloc0 = torch.cuda.memory_allocated()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert noalloc_status(cowa, q, kc, vc, sl, quad, out, lse) == 0
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert free1 == free0
+
+
+def test_noalloc_python_wrapper():
+    import structured_sparse_attention_block_b200 as cowa
+    from structured_sparse_attention_block_b200.inputs import decode_inputs
+    quad = (16, 128, 0, 300)
+    q, kc, vc, sl = decode_inputs(3, 1000, 8, 2, 64, seed=6, seqlens=[1000, 513, 2])
+    o_ref, lse_ref = cowa.cowa_decode(q, kc, vc, sl, quad)
+    out = torch.full_like(o_ref, float("nan"))
+    lse = torch.full_like(lse_ref, float("nan"))
+    o, l2 = cowa.cowa_decode_noalloc(q, kc, vc, sl, quad, out, lse)
+    torch.cuda.synchronize()
+    assert o.data_ptr() == out.data_ptr() and l2.data_ptr() == lse.data_ptr()
+    assert_o(out[:, 0], to64(o_ref[:, 0]), what="noalloc O (wrapper)")
+    assert (lse - lse_ref).abs().max().item() <= LSE_ABS
 
 
 def test_noalloc_refuses_shapes_beyond_the_static_scratch():
