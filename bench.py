@@ -507,6 +507,9 @@ def run_cowa(args, rank, world, local_rank):
     if args.decode_workload:
         result["decode_workload"] = run_decode_workload(args, cowa, rank, dev, stream, flush, world, peaks,
                                                         peak_src)
+    if args.mala and not h0_mode(args, world):
+        result["mala_workload"] = run_mala_workload(args, cowa, rank, dev, stream, flush, world, peaks,
+                                                    tensor_peak)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = run_cpu_baseline(wl, q, k, v, do, quad, args.cpu_rows)
     return result
@@ -776,6 +779,77 @@ def run_decode_workload(args, cowa, rank, dev, stream, flush, world, peaks, peak
                          "GB/s": round(nbytes / (ms_w * 1e-3) / 1e9, 1)}}
 
 
+def mala_pair_counts(keep, Lq, Lk, bm=128, bn=64):
+    """(causal pairs, kept pairs) over all (b, hq) of a MALA decision array
+    keep [B, Hq, nqt, nkt]: a block's pairs are (i, j) with j <= i + Lk - Lq."""
+    nqt, nkt = keep.shape[2], keep.shape[3]
+    p = np.arange(Lq, dtype=np.int64) + (Lk - Lq)
+    per_block = np.zeros((nqt, nkt), dtype=np.int64)
+    for t in range(nkt):
+        j0, j1 = t * bn, min((t + 1) * bn, Lk)
+        cnt = np.clip(np.minimum(p + 1, j1) - j0, 0, None)  # keys of block t row i sees
+        per_block[:, t] = np.add.reduceat(cnt, np.arange(0, Lq, bm))
+    causal = int(per_block.sum()) * keep.shape[0] * keep.shape[1]
+    kept = int((keep.astype(np.int64) * per_block[None, None]).sum())
+    return causal, kept
+
+
+def run_mala_workload(args, cowa, rank, dev, stream, flush, world, peaks, tensor_peak):
+    """MALA (the pages' companion operator: full causal scoring, blocks of
+    128 query rows x 64 keys kept when some row gives them at least tau of
+    its softmax mass) on the 14B-like 32K shape, where the pages quote its
+    training-FLOP saving; forward and backward timed separately.  Work is
+    counted per the reading: forward 2d per causal pair (scoring) + 2d per
+    kept pair (PV); backward 6d per causal pair (S, dQ, dK) + 4d per kept
+    pair (dP, dV)."""
+    import torch.distributed as dist
+    from structured_sparse_attention_block_b200.inputs import WORKLOADS, workload_inputs
+    wl = WORKLOADS["llm14b_32k"]
+    tau = 2.0 ** -8
+    q, k, v, do = workload_inputs(wl, seed=11 + 1000 * rank)
+    o, lse, keep = cowa.cowa_mala_fwd(q, k, v, tau)
+    ws = torch.empty(cowa.lib().cowa_mala_bwd_workspace_size(
+        ctypes_shape(cowa, q, k, v, o)), dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        cowa.cowa_mala_fwd(q, k, v, tau, out=o, lse=lse, keep=keep)
+        cowa.cowa_mala_bwd(q, k, v, o, lse, keep, do, workspace=ws)
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 10))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    if world > 1:
+        dist.barrier()
+    for e in evs:
+        flush.zero_()
+        e[0].record(stream)
+        cowa.cowa_mala_fwd(q, k, v, tau, out=o, lse=lse, keep=keep)
+        e[1].record(stream)
+        cowa.cowa_mala_bwd(q, k, v, o, lse, keep, do, workspace=ws)
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    cowa.cowa_get_device_error(dev)
+    t_f, t_b = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in evs) / n,
+                               sum(e[1].elapsed_time(e[2]) for e in evs) / n], world, dev)
+    causal, kept = mala_pair_counts(keep.cpu().numpy(), wl.Lq, wl.Lk)
+    causal, kept = (int(x) for x in sum_over_ranks([causal, kept], world, dev))
+    fwd_fl = causal * 2 * wl.d + kept * 2 * wl.d
+    bwd_fl = causal * 6 * wl.d + kept * 4 * wl.d
+    del q, k, v, do, o, lse, keep, ws
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "tau": tau, "block": [128, 64],
+            "causal_pairs": causal, "kept_pairs": kept, "kept_fraction": round(kept / causal, 4),
+            "fwd_ms": round(t_f, 4), "bwd_ms": round(t_b, 4),
+            "fwd_tflops": round(fwd_fl / (t_f * 1e-3) / 1e12, 2), "bwd_tflops": round(bwd_fl / (t_b * 1e-3) / 1e12, 2),
+            "fwd_frac": round(fwd_fl / (t_f * 1e-3) / 1e12 / world / tensor_peak, 4),
+            "bwd_frac": round(bwd_fl / (t_b * 1e-3) / 1e12 / world / tensor_peak, 4),
+            "counted": "fwd 2d/causal pair + 2d/kept pair; bwd 6d/causal pair + 4d/kept pair",
+            "inputs": "synthetic N(0,1): attention is diffuse, so a block's mass falls with the row's length"}
+
+
+def ctypes_shape(cowa, q, k, v, o):
+    import ctypes
+    return ctypes.byref(cowa._shape(q, k, v, o, 0))
+
+
 # ------------------------------------------------------------ CPU oracle ----
 def oracle_sample(wl, q, k, v, do, quad, rows):
     """The oracle on a bounded sample of the step: batch element 0, the last
@@ -861,6 +935,8 @@ def main():
                     help="skip the packed variable-length batch of the workload's heads and windows")
     ap.add_argument("--no-full-mask", dest="full_mask", action="store_false",
                     help="skip the full-causal-mask control run of the same step")
+    ap.add_argument("--no-mala", dest="mala", action="store_false",
+                    help="skip the MALA forward + backward leg (14B-like 32K shape)")
     args = ap.parse_args()
     if args.cpu_rows is None:
         args.cpu_rows = CPU_ROWS.get(args.workload, 256)

@@ -236,6 +236,52 @@ COWA_API int cowa_bwd(const cowa_shape_t *shape, cowa_quad_t quad, float softmax
              void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * MassAlloc Attention (MALA), the companion operator of the same pages
+ * ("Two new attention models slash redundancy...", first section; "CoWindow
+ * Attention: Full Causal Coverage Is a Collective Property", abstract): it
+ * keeps full causal QK scoring and lets attention's own softmax statistics
+ * decide where the remaining work of a block is skipped.  The pages give no
+ * rule; this library fixes the plainest reading:
+ *   - scores on every causal pair (bottom-right alignment, p = i + Lk - Lq;
+ *     query head hq uses KV head hq / (Hq / Hkv)); LSE over all of them;
+ *   - per block of 128 query rows x 64 keys of one head, the mass each row
+ *     gives the block, M = sum_j P_ij with P = exp(s - LSE); the block is kept
+ *     when some row of it has M >= tau, skipped otherwise;
+ *   - O_i = sum over kept blocks of P_ij v_j: the dropped mass is not
+ *     redistributed (LSE stays the full statistic);
+ *   - the gradient is that of this O with the block decisions held fixed:
+ *     dV and dP only over kept pairs, dS = P (dP - delta) over every causal
+ *     pair (skipped pairs keep -P * delta through the LSE).
+ * The decision compares an fp32 sum of the kernel's fp32 probabilities with
+ * tau; a block whose mass lies within about 1e-5 (relative) of tau may be
+ * decided either way.
+ *
+ * cowa_mala_keep_bytes: bytes of the decision array keep[B][Hq][ceil(Lq/128)]
+ *   [ceil(Lk/64)] (uint8: 1 kept, 0 skipped or past the causal diagonal).
+ * cowa_mala_fwd: q, k, v as for cowa_fwd (shape->kv_head_offset must be 0:
+ *   MALA has no per-head windows); o [B, Lq, Hq, d] bf16, lse [B, Hq, Lq]
+ *   fp32 (natural log) and keep (device, cowa_mala_keep_bytes) out.  tau is
+ *   a finite value >= 0: tau = 0 keeps every causal block (dense causal
+ *   attention), tau > 1 keeps none (O = 0, LSE still the full statistic).
+ *   Needs no workspace.  Rows with no causal key give O = 0, LSE = -inf.
+ * cowa_mala_bwd: q, k, v, o, lse and keep from cowa_mala_fwd, dout (o's
+ *   strides); dq, dk, dv out as for cowa_bwd; workspace of
+ *   cowa_mala_bwd_workspace_size bytes, 256-byte aligned.
+ * Both are asynchronous on `stream`; errors as for cowa_fwd / cowa_bwd
+ * (COWA_ERR_INVALID_ARG for a NULL keep, tau < 0 or not finite, or a
+ * nonzero kv_head_offset).
+ */
+COWA_API size_t cowa_mala_keep_bytes(const cowa_shape_t *shape);
+COWA_API int cowa_mala_fwd(const cowa_shape_t *shape, float tau, float softmax_scale,
+             const void *q, const void *k, const void *v, void *o, float *lse, uint8_t *keep,
+             void *stream);
+COWA_API size_t cowa_mala_bwd_workspace_size(const cowa_shape_t *shape);
+COWA_API int cowa_mala_bwd(const cowa_shape_t *shape, float softmax_scale,
+             const void *q, const void *k, const void *v, const void *o, const float *lse,
+             const uint8_t *keep, const void *dout, void *dq, void *dk, void *dv,
+             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Single-token decode over a KV cache (paper abstract: decoding).
  *   shape->Lq must be 1 and shape->Lk is the cache capacity Lcap.
  *   q [B, 1, Hq, d]; k_cache / v_cache [B, Lcap, Hkv, d]; seqlens [B] int32

@@ -31,6 +31,7 @@ __all__ = ["CowaError", "cowa_fwd", "cowa_bwd", "cowa_decode", "cowa_default_qua
            "cowa_decode_noalloc", "cowa_trace_start", "cowa_trace_stop", "cowa_trace_entries",
            "cowa_wcache_rows", "cowa_wcache_build", "cowa_wcache_append", "cowa_decode_windowed",
            "cowa_fwd_varlen", "cowa_bwd_varlen", "cowa_selftest_wait_timeout",
+           "cowa_mala_fwd", "cowa_mala_bwd",
            "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -107,6 +108,14 @@ def lib():
         L.cowa_bwd.argtypes = [SP, Quad, ctypes.c_float] + [vp] * 9 + [vp, sz, vp]
         L.cowa_decode.restype = ctypes.c_int
         L.cowa_decode.argtypes = [SP, Quad, ctypes.c_float] + [vp] * 6 + [vp, sz, vp]
+        L.cowa_mala_keep_bytes.restype = sz
+        L.cowa_mala_keep_bytes.argtypes = [SP]
+        L.cowa_mala_fwd.restype = ctypes.c_int
+        L.cowa_mala_fwd.argtypes = [SP, ctypes.c_float, ctypes.c_float] + [vp] * 7
+        L.cowa_mala_bwd_workspace_size.restype = sz
+        L.cowa_mala_bwd_workspace_size.argtypes = [SP]
+        L.cowa_mala_bwd.restype = ctypes.c_int
+        L.cowa_mala_bwd.argtypes = [SP, ctypes.c_float] + [vp] * 10 + [vp, sz, vp]
         L.cowa_decode_noalloc.restype = ctypes.c_int
         L.cowa_decode_noalloc.argtypes = [SP, Quad, ctypes.c_float] + [vp] * 6 + [vp]
         L.cowa_schedule_workspace_size.restype = sz
@@ -238,6 +247,67 @@ def cowa_fwd(q, k, v, quad, softmax_scale=None, kv_head_offset=0, out=None, lse=
     _check(L.cowa_fwd(ctypes.byref(shape), qd, scale, _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                       _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)))
     return out, lse
+
+
+def cowa_mala_fwd(q, k, v, tau, softmax_scale=None, out=None, lse=None, keep=None):
+    """MALA forward (full causal scoring; blocks of 128 query rows x 64 keys
+    kept when some row gives them at least ``tau`` of its softmax mass).
+    Returns ``(o, lse, keep)`` with keep uint8 [B, Hq, ceil(Lq/128),
+    ceil(Lk/64)]; see ``cowa_mala_fwd`` in include/cowa.h."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bf16_cuda(t, n)
+    B, Lq, Hq, d = q.shape
+    Lk = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    kshape = (B, Hq, -(-Lq // 128), -(-Lk // 64))
+    if keep is None:
+        keep = torch.empty(kshape, dtype=torch.uint8, device=q.device)
+    _bf16_cuda(out, "out")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, Lq):
+        raise ValueError("lse must be contiguous fp32 [B, Hq, Lq]")
+    if keep.dtype != torch.uint8 or not keep.is_contiguous() or tuple(keep.shape) != kshape:
+        raise ValueError("keep must be contiguous uint8 %s" % (kshape,))
+    shape = _shape(q, k, v, out, 0)
+    scale = 0.0 if softmax_scale is None else float(softmax_scale)
+    _check(lib().cowa_mala_fwd(ctypes.byref(shape), float(tau), scale, _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                               _ptr(lse), _ptr(keep), _stream(q.device)))
+    return out, lse, keep
+
+
+def cowa_mala_bwd(q, k, v, o, lse, keep, dout, softmax_scale=None, dq=None, dk=None, dv=None,
+                  workspace=None):
+    """MALA backward with the forward's block decisions held fixed.  Returns
+    ``(dq, dk, dv)``; dO uses o's strides, each gradient its input's."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _bf16_cuda(t, n)
+    if dout.stride() != o.stride():
+        raise ValueError("dout must have the strides of o")
+    dq = torch.empty_strided(q.shape, q.stride(), dtype=q.dtype, device=q.device) if dq is None else dq
+    dk = torch.empty_strided(k.shape, k.stride(), dtype=k.dtype, device=k.device) if dk is None else dk
+    dv = torch.empty_strided(v.shape, v.stride(), dtype=v.dtype, device=v.device) if dv is None else dv
+    for t, ref, n in ((dq, q, "dq"), (dk, k, "dk"), (dv, v, "dv")):
+        _bf16_cuda(t, n)
+        if t.stride() != ref.stride() or t.shape != ref.shape:
+            raise ValueError("%s must match the shape and strides of its input" % n)
+    B, Lq, Hq, d = q.shape
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, Lq):
+        raise ValueError("lse must be contiguous fp32 [B, Hq, Lq]")
+    kshape = (B, Hq, -(-Lq // 128), -(-k.shape[1] // 64))
+    if keep.dtype != torch.uint8 or not keep.is_contiguous() or tuple(keep.shape) != kshape:
+        raise ValueError("keep must be contiguous uint8 %s" % (kshape,))
+    shape = _shape(q, k, v, o, 0)
+    L = lib()
+    need = L.cowa_mala_bwd_workspace_size(ctypes.byref(shape))
+    if need == 0:
+        _raise_size_error(L)
+    ws = _workspace(need, q.device, workspace)
+    scale = 0.0 if softmax_scale is None else float(softmax_scale)
+    _check(L.cowa_mala_bwd(ctypes.byref(shape), scale, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(keep),
+                           _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(q.device)))
+    return dq, dk, dv
 
 
 def _raise_size_error(L):

@@ -752,6 +752,107 @@ int cowa_bwd_varlen(const cowa_varlen_shape_t *s, cowa_quad_t quad, float softma
     return COWA_OK;
 }
 
+// ------------------------------------------------------------------- MALA --
+// MassAlloc Attention: full causal scoring, blocks of kMalaBM query rows x
+// kMalaBN keys kept when some row gives them at least tau of its softmax
+// mass (the reading is in include/cowa.h and csrc/mala.cu).
+
+static int check_mala(const cowa_shape_t *s, float tau)
+{
+    const cowa_quad_t full = {0, 0, 0, 0};
+    int r = check_shape(s, full, false);
+    if (r) return r;
+    if (s->kv_head_offset != 0) return fail(COWA_ERR_INVALID_ARG, "MALA has no per-head windows: kv_head_offset must be 0");
+    if (!(tau >= 0.f) || !(tau <= 1e30f)) return fail(COWA_ERR_INVALID_ARG, "tau must be a finite value >= 0");
+    return COWA_OK;
+}
+
+size_t cowa_mala_keep_bytes(const cowa_shape_t *s)
+{
+    if (check_mala(s, 0.f)) return 0;
+    return (size_t)(s->B * s->Hq * cdiv(s->Lq, cowa::kMalaBM) * cdiv(s->Lk, cowa::kMalaBN));
+}
+
+int cowa_mala_fwd(const cowa_shape_t *s, float tau, float softmax_scale, const void *q, const void *k, const void *v,
+                  void *o, float *lse, uint8_t *keep, void *stream)
+{
+    int r = check_mala(s, tau);
+    if (r) return r;
+    const bool qrows = s->B * s->Lq * s->Hq > 0, krows = s->B * s->Lk * s->Hkv > 0;
+    if ((r = check_ptr(q, qrows, "q")) || (r = check_ptr(k, qrows && krows, "k")) ||
+        (r = check_ptr(v, qrows && krows, "v")) || (r = check_ptr(o, qrows, "o")) ||
+        (r = check_ptr(lse, qrows, "lse")))
+        return r;
+    if (qrows && krows && !keep) return fail(COWA_ERR_INVALID_ARG, "keep is NULL");
+    if (!qrows) return COWA_OK;
+    if ((r = check_device(nullptr))) return r;
+    cudaStream_t st = (cudaStream_t)stream;
+    cowa::AttnParams p{};
+    fill_common(p, s, cowa_quad_t{0, 0, 0, 0}, softmax_scale);
+    p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
+    p.B = (int)s->B; p.Lq = (int)s->Lq; p.Lk = (int)s->Lk;
+    p.lse_ld = s->Lq;
+    if (s->Lk == 0) {
+        // no keys: every row sees nothing (O = 0, LSE = -inf); no blocks
+        cudaError_t e = cowa::launch_zero_rows(o, p.os, p.B, p.Lq, p.Hq, (int)s->d, st);
+        if (e == cudaSuccess) e = cowa::launch_fill_f32(lse, s->B * s->Hq * s->Lq, -INFINITY, st);
+        return e == cudaSuccess ? COWA_OK : cuda_fail(e, "constant output launch");
+    }
+    p.nqt = (int)cdiv(s->Lq, cowa::kMalaBM);
+    p.nkt = (int)cdiv(s->Lk, cowa::kMalaBN);
+    cudaError_t e = cowa::launch_mala_fwd(p, (int)s->d, keep, tau, st);
+    if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
+    if (e != cudaSuccess) return cuda_fail(e, "MALA forward launch");
+    return COWA_OK;
+}
+
+size_t cowa_mala_bwd_workspace_size(const cowa_shape_t *s)
+{
+    if (check_mala(s, 0.f)) return 0;
+    return cowa_bwd_workspace_size(s, cowa_quad_t{0, (int32_t)s->Lk, 0, 0});
+}
+
+int cowa_mala_bwd(const cowa_shape_t *s, float softmax_scale, const void *q, const void *k, const void *v,
+                  const void *o, const float *lse, const uint8_t *keep, const void *dout, void *dq, void *dk, void *dv,
+                  void *ws, size_t ws_bytes, void *stream)
+{
+    int r = check_mala(s, 0.f);
+    if (r) return r;
+    const bool qrows = s->B * s->Lq * s->Hq > 0, krows = s->B * s->Lk * s->Hkv > 0;
+    if (qrows && krows && !keep) return fail(COWA_ERR_INVALID_ARG, "keep is NULL");
+    if (!qrows || !krows) {
+        // no pair at all: the gradients are those of cowa_bwd (zero)
+        return cowa_bwd(s, cowa_quad_t{0, (int32_t)s->Lk, 0, 0}, softmax_scale, q, k, v, o, lse, dout, dq, dk, dv, ws,
+                        ws_bytes, stream);
+    }
+    if ((r = check_ptr(q, true, "q")) || (r = check_ptr(k, true, "k")) || (r = check_ptr(v, true, "v")) ||
+        (r = check_ptr(o, true, "o")) || (r = check_ptr(lse, true, "lse")) || (r = check_ptr(dout, true, "dout")) ||
+        (r = check_ptr(dq, true, "dq")) || (r = check_ptr(dk, true, "dk")) || (r = check_ptr(dv, true, "dv")))
+        return r;
+    if ((r = check_device(nullptr))) return r;
+    // the backward of every causal pair (the scores are full), with the
+    // forward's block decisions: pairs of skipped blocks keep only -P * delta
+    const cowa_quad_t full = {0, (int32_t)s->Lk, 0, 0};
+    const size_t need = cowa_bwd_workspace_size(s, full);
+    if (!ws || ws_bytes < need || (uintptr_t)ws % 256)
+        return fail(COWA_ERR_WORKSPACE, "MALA bwd workspace needs %zu bytes, 256-byte aligned (got %zu)", need, ws_bytes);
+    cudaStream_t st = (cudaStream_t)stream;
+    cowa::AttnParams p{};
+    fill_common(p, s, full, softmax_scale);
+    p.q = q; p.k = k; p.v = v; p.o = (void *)o; p.lse_in = lse; p.dout = dout;
+    p.dq = dq; p.dk = dk; p.dv = dv;
+    p.B = (int)s->B; p.Lq = (int)s->Lq; p.Lk = (int)s->Lk;
+    p.lse_ld = s->Lq;
+    p.keep = keep;
+    p.keep_nqt = (int)cdiv(s->Lq, cowa::kMalaBM);
+    p.keep_nkt = (int)cdiv(s->Lk, cowa::kMalaBN);
+    const int nqt = (int)cdiv(s->Lq, cowa::kBwd5QTile), nkt = (int)cdiv(s->Lk, cowa::kBwd5KeyTile);
+    cudaError_t e = cowa::launch_bwd_sm100(p, (int)s->d, (float2 *)ws, (int)cowa::bwd5_lq_pad(s->Lq), nqt, nkt, st);
+    if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
+    if (e != cudaSuccess) return cuda_fail(e, "MALA backward launch");
+    return COWA_OK;
+}
+
 size_t cowa_schedule_workspace_size(int64_t Lq, int64_t Lk, int32_t BM, int32_t BN)
 {
     if (Lq < 0 || Lk < 0 || BM <= 0 || BN <= 0) return 0;

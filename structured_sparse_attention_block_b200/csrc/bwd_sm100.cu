@@ -161,8 +161,26 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
     const uint32_t KV_TM = bar0 + 8u * (12 + 2 * ST);  // K and V are in tensor memory
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const TilePos pos = tile_pos(p.Hkv, p.B);
-    const int kt = pos.step, hl = pos.slot, b = pos.b;  // sink keys first
+    // order: the sink tile (key tile 0, seen by every query) of every
+    // (KV head, batch) first, then (batch, KV head) after (batch, KV head)
+    // with their key tiles ascending, so the CTAs resident together are
+    // neighbouring key tiles of one head, which read the same query rows
+    // (measured at 32K: DRAM reads 9.0 -> 1.6 GB per launch, L2 hit rate 63 ->
+    // 91 %); the long sink CTAs start in the first wave
+    int kt, hl, b;
+    {
+        const unsigned hb_n = (unsigned)p.Hkv * (unsigned)p.B, lin = blockIdx.x;
+        if (lin < hb_n) {
+            kt = 0;
+            b = (int)(lin / (unsigned)p.Hkv);
+            hl = (int)(lin % (unsigned)p.Hkv);
+        } else {
+            const unsigned per = (unsigned)(p.nkt - 1), r = lin - hb_n, hb = r / per;
+            kt = 1 + (int)(r - hb * per);
+            b = (int)(hb / (unsigned)p.Hkv);
+            hl = (int)(hb % (unsigned)p.Hkv);
+        }
+    }
     const SeqGeom sg = seq_geom(p, b);
     const int c0 = kt * BN;
     if (c0 >= sg.Lk) return;  // past the end of this sequence of a packed batch
@@ -363,12 +381,19 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
         // and position t in the key tile's query-tile list, advanced without
         // division
         int gi = nq > 0 ? x / nq : 0, tq = nq > 0 ? x % nq : 0;
+        // MALA block decisions of this key's column for the group's first
+        // query head (nullptr for CoWA)
+        const uint8_t *kbase = p.keep ? p.keep + ((long long)b * p.Hq + hl * p.g) * p.keep_nqt * p.keep_nkt +
+                                            jg / kMalaBN
+                                      : nullptr;
         for (int k = 0; ok; ++k) {
             const int u = 2 * k + x;
             if (u >= ntask) break;
             // task set-up, independent of the scores: done while they land
             const int qt = tq < len0 || nr == 1 ? lo0 + tq
                            : (tq - len0 < len1 || nr == 2 ? lo1 + tq - len0 : lo2 + tq - len0 - len1);
+            // MALA: a key of a skipped block has dP = 0 and no dV share
+            const bool skip = kbase && !kbase[(gi * p.keep_nqt + qt * BM / kMalaBM) * p.keep_nkt];
             tq += 2;
             while (tq >= nq) {
                 tq -= nq;
@@ -408,6 +433,10 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
                     for (int e = 0; e < 32; ++e)
                         if (!((vis[c] >> e) & 1u)) sr[e] = __float_as_uint(-CUDART_INF_F);
                 }
+                if (skip) {  // MALA skipped block: dP = 0
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) dr[e] = 0u;
+                }
                 // P^T and dS^T as bf16 pairs: entry e holds columns 2e, 2e+1
                 uint32_t pk[16], dk[16];
 #pragma unroll
@@ -429,6 +458,10 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
                     ok = __all_sync(0xffffffffu, mbar_wait(G_DONE(x), (k - 1) & 1, p.err, abort_flag));
                     if (!ok) break;
                     tc_fence_after();
+                }
+                if (skip) {  // and no share of dV
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
                 }
                 tmem_st16(tPD + c * 16, pk);
                 tmem_st16(tPD + BM / 2 + c * 16, dk);
@@ -700,6 +733,10 @@ __global__ void __launch_bounds__(352, 1) dq_sm100_kernel(const __grid_constant_
         for (int t = 0; active && t < ntiles; ++t) {
             // tile set-up, independent of the scores: done while they land
             const int j0 = tile_of(t) * BN;
+            // MALA: a skipped block's pairs have dP = 0 (query tiles of this
+            // pass are the blocks' rows, key tiles their keys)
+            const bool skip = p.keep && !p.keep[(((long long)b * p.Hq + hq) * p.keep_nqt + qt) * p.keep_nkt +
+                                                j0 / kMalaBN];
             const bool full = __all_sync(0xffffffffu, runs_cover(rr, j0, j0 + BN - 1));
             uint32_t vis[BN / 32];
             if (!full) {
@@ -735,8 +772,10 @@ __global__ void __launch_bounds__(352, 1) dq_sm100_kernel(const __grid_constant_
                     // measured 2 % faster here, slower in the dK/dV pass
                     constexpr int PE = D == 64 ? 4 : 0, PM = PE > 0 ? PE : 1;
                     const float2 pr = (PE && e % PM == PM - 1) ? exp2_poly2(xa) : make_float2(fast_ex2(xa.x), fast_ex2(xa.y));
-                    const float2 tt = __fadd2_rn(make_float2(__uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1])),
-                                                 nd2);
+                    const float2 tt = skip ? nd2
+                                           : __fadd2_rn(make_float2(__uint_as_float(dr[2 * e]),
+                                                                    __uint_as_float(dr[2 * e + 1])),
+                                                        nd2);
                     const float2 ds = __fmul2_rn(pr, tt);
                     pk[e] = pack2(ds.x, ds.y);
                 }
@@ -1022,6 +1061,9 @@ __global__ void __launch_bounds__(352, 1) dq_tm_kernel(const __grid_constant__ B
         for (int t = 0; ok && t < ntiles; ++t) {
             // tile set-up, independent of the scores: done while they land
             const int j0 = tile_of(t) * BN + x * 32;
+            // MALA: a skipped block's pairs have dP = 0
+            const bool skip = p.keep && !p.keep[(((long long)b * p.Hq + hq) * p.keep_nqt + qt) * p.keep_nkt +
+                                                j0 / kMalaBN];
             const bool full = __all_sync(0xffffffffu, runs_cover(rr, j0, j0 + 31));
             const uint32_t vis = full ? 0xffffffffu : runs_bits(rr, j0);
             ok = __all_sync(0xffffffffu, mbar_wait(S_FULL, t & 1, p.err, abort_flag));
@@ -1046,8 +1088,9 @@ __global__ void __launch_bounds__(352, 1) dq_tm_kernel(const __grid_constant__ B
                 const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
                                              sc2, nl2);
                 const float2 pr = make_float2(fast_ex2(xa.x), fast_ex2(xa.y));
-                const float2 tt = __fadd2_rn(make_float2(__uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1])),
-                                             nd2);
+                const float2 tt = skip ? nd2
+                                       : __fadd2_rn(make_float2(__uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1])),
+                                                    nd2);
                 const float2 ds = __fmul2_rn(pr, tt);
                 pk[e] = pack2(ds.x, ds.y);
             }

@@ -66,6 +66,11 @@ struct AttnParams {
     const int *cu_q, *cu_k;
     int total_q, total_k;
     long long lse_ld;                 // LSE row pitch: Lq, or total_q when packed
+    // MALA backward: the forward's block decisions keep[b][hq][i / kMalaBM]
+    // [j / kMalaBN] (nullptr for CoWA); a pair of a skipped block has dP = 0
+    // and contributes nothing to dV (only -P * delta remains in dS)
+    const uint8_t *keep;
+    int keep_nqt, keep_nkt;
 };
 
 // Lengths and row offsets of sequence b, and its batch coordinate (b for a
@@ -156,6 +161,11 @@ __host__ __device__ constexpr int fwd5_bn(int D) { return D == 128 ? 64 : 96; }
 bool make_bshd_map(CUtensorMap *m, const void *base, int d, long long L, long long H, long long B,
                    const long long st[3], int rows);
 
+// mala.cu (MALA forward): blocks of kMalaBM query rows x kMalaBN keys decide
+// together; keep[b][hq][qt][kt] receives the decisions
+constexpr int kMalaBM = 128, kMalaBN = 64;
+cudaError_t launch_mala_fwd(const AttnParams &p, int D, uint8_t *keep, float tau, cudaStream_t st);
+
 // fill.cu: constant outputs of the shapes the tcgen05 kernels do not take
 // (zero rows of a strided [B, L, H, D] bf16 tensor; a constant fp32 array)
 cudaError_t launch_zero_rows(void *t, const long long st[3], int B, int L, int H, int D, cudaStream_t s);
@@ -171,12 +181,12 @@ __host__ __device__ constexpr int bwd5_kv_bm(int D) { return D == 128 ? 32 : 64;
 __host__ __device__ constexpr int bwd5_dq_bn(int D) { return D == 128 ? 128 : 64; }   // keys per dQ tile
 inline long long bwd5_lq_pad(long long Lq) { return (Lq + 63) / 64 * 64; }
 
-// Launch order of the tiled tcgen05 kernels: a 1-D grid whose block index
-// runs over (head slot, batch) fastest and over the tile step slowest.  The
-// launcher maps step 0 to the heaviest tile of every head (the last query
-// tile for the query-major passes, the first key tile, which holds the sink
-// keys, for the key-major pass), so the long CTAs start in the first waves
-// and the short ones fill the tail.
+// Launch order of the query-major tcgen05 kernels (forward, dQ): a 1-D grid
+// whose block index runs over (head slot, batch) fastest and over the tile
+// step slowest.  The kernels map step 0 to the heaviest tile of every head
+// (the last query tile), so the long CTAs start in the first waves and the
+// short ones fill the tail.  (The key-major dK/dV pass orders its own grid:
+// sink tiles first, then key tiles ascending head by head.)
 struct TilePos {
     int step, slot, b;
 };

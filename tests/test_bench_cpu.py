@@ -138,3 +138,21 @@ def test_source_hash_ignores_comments_only():
     assert bench.strip_comments(code) != bench.strip_comments(code.replace("return 1", "return 2"))
     assert bench.strip_comments(code) != bench.strip_comments(code.replace("// kept", "// kept!"))
     assert bench.strip_comments("char c = '\\'';  // q\n") == "char c = '\\'';\n"
+
+
+def test_mala_pair_counts_match_brute_force():
+    """The MALA leg's causal and kept pair counts from a block decision array
+    equal a loop over every (row, key) pair."""
+    from bench import mala_pair_counts
+    rng = np.random.default_rng(0)
+    for Lq, Lk in [(300, 400), (257, 257), (130, 64), (64, 300)]:
+        nqt, nkt = -(-Lq // 128), -(-Lk // 64)
+        keep = (rng.random((2, 3, nqt, nkt)) < 0.5).astype(np.uint8)
+        causal, kept = mala_pair_counts(keep, Lq, Lk)
+        cb = kb = 0
+        for i in range(Lq):
+            for j in range(Lk):
+                if j <= i + Lk - Lq:
+                    cb += 6
+                    kb += int(keep[:, :, i // 128, j // 64].sum())
+        assert (causal, kept) == (cb, kb)
