@@ -675,16 +675,42 @@ static void fill_varlen(cowa::AttnParams &p, const cowa_varlen_shape_t *s, cowa_
     p.lse_ld = s->total_q;
 }
 
+// Work list of a packed batch for tiles of 128 rows: (sequence, tile) items,
+// at most total/128 + B of them, and the scratch of the list builder
+// (3 ints per possible tile count of one sequence).
+struct WorkList {
+    long long items, max_tiles;
+    size_t list_bytes() const { return align256((size_t)items * sizeof(int2)); }
+    size_t scratch_bytes() const { return align256((size_t)(3 * (max_tiles + 1)) * sizeof(int)); }
+    size_t bytes() const { return list_bytes() + scratch_bytes(); }
+};
+static WorkList work_list(long long total, long long max_len, long long B)
+{
+    return WorkList{total / 128 + B + 1, cdiv(max_len, 128)};
+}
+
+// Builds the list into ws (list, then scratch); returns the pointer to the list.
+static cudaError_t build_work_list(const WorkList &wl, const int32_t *cu, long long B, bool descending, char *ws,
+                                   int2 **list, cudaStream_t st)
+{
+    *list = (int2 *)ws;
+    return cowa::launch_varlen_worklist(cu, (int)B, 128, (int)wl.max_tiles, descending, *list, (int)wl.items,
+                                        (int *)(ws + wl.list_bytes()), device_error_word(), st);
+}
+
 size_t cowa_fwd_varlen_workspace_size(const cowa_varlen_shape_t *s, cowa_quad_t q)
 {
     if (check_varlen(s, q)) return 0;
-    return 256;  // the kernels form their tile ranges themselves
+    // the kernels form their tile ranges themselves; the work list of the
+    // query tiles sizes the grid to the real tiles
+    return work_list(s->total_q, s->max_q, s->B).bytes() + 256;
 }
 
 size_t cowa_bwd_varlen_workspace_size(const cowa_varlen_shape_t *s, cowa_quad_t q)
 {
     if (check_varlen(s, q)) return 0;
-    return align256((size_t)(s->B * s->Hq * cowa::bwd5_lq_pad(s->max_q)) * sizeof(float2)) + 256;
+    return align256((size_t)(s->B * s->Hq * cowa::bwd5_lq_pad(s->max_q)) * sizeof(float2)) +
+           work_list(s->total_q, s->max_q, s->B).bytes() + work_list(s->total_k, s->max_k, s->B).bytes() + 256;
 }
 
 int cowa_fwd_varlen(const cowa_varlen_shape_t *s, cowa_quad_t quad, float softmax_scale, const int32_t *cu_q,
@@ -712,7 +738,13 @@ int cowa_fwd_varlen(const cowa_varlen_shape_t *s, cowa_quad_t quad, float softma
     const int BN = cowa::fwd5_bn((int)s->d);
     p.nqt = (int)cdiv(s->max_q, cowa::kFwd5BM);
     p.nkt = (int)cdiv(s->max_k, BN);
-    cudaError_t e = cowa::launch_fwd_sm100(p, (int)s->d, st);
+    const WorkList wq = work_list(s->total_q, s->max_q, s->B);
+    int2 *list = nullptr;
+    cudaError_t e = build_work_list(wq, cu_q, s->B, true, (char *)ws, &list, st);
+    if (e != cudaSuccess) return cuda_fail(e, "work list launch");
+    p.work = list;
+    p.work_n = (int)wq.items;
+    e = cowa::launch_fwd_sm100(p, (int)s->d, st);
     if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
     if (e != cudaSuccess) return cuda_fail(e, "forward launch");
     return COWA_OK;
@@ -746,7 +778,16 @@ int cowa_bwd_varlen(const cowa_varlen_shape_t *s, cowa_quad_t quad, float softma
     const long long lq_pad = cowa::bwd5_lq_pad(s->max_q);
     const int D = (int)s->d;
     const int nqt = (int)cdiv(s->max_q, cowa::kBwd5QTile), nkt = (int)cdiv(s->max_k, cowa::kBwd5KeyTile);
-    cudaError_t e = cowa::launch_bwd_sm100(p, D, (float2 *)rows_ws, (int)lq_pad, nqt, nkt, st);
+    // work lists: query tiles (dQ, last tile first), key tiles (dK/dV, first
+    // tile first)
+    const WorkList wq = work_list(s->total_q, s->max_q, s->B), wk = work_list(s->total_k, s->max_k, s->B);
+    char *lists = rows_ws + align256((size_t)(s->B * s->Hq * lq_pad) * sizeof(float2));
+    int2 *list_q = nullptr, *list_k = nullptr;
+    cudaError_t e = build_work_list(wq, cu_q, s->B, true, lists, &list_q, st);
+    if (e == cudaSuccess) e = build_work_list(wk, cu_k, s->B, false, lists + wq.bytes(), &list_k, st);
+    if (e != cudaSuccess) return cuda_fail(e, "work list launch");
+    e = cowa::launch_bwd_sm100(p, D, (float2 *)rows_ws, (int)lq_pad, nqt, nkt, st, list_q, (int)wq.items, list_k,
+                               (int)wk.items);
     if (e == cudaErrorInvalidValue) return fail(COWA_ERR_CUDA, "TMA descriptor encoding failed");
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return COWA_OK;

@@ -7,27 +7,33 @@
 //    delta = rowsum(dO * O), rows padded to a multiple of 64 (padding and rows
 //    that see no key get (-inf, 0), so their probabilities are 0).
 //
-// 2. dkdv_sm100_kernel, key-tile major: one CTA per (128 keys, KV head,
-//    batch).  The keys are the rows of every accumulator (tensor-memory lanes).
+// 2. dK/dV pass, key-tile major: one CTA per (128 keys, KV head, batch).
+//    The keys are the rows of every accumulator (tensor-memory lanes).
 //    Tasks are (query head of the group, query tile of BM rows) from the
-//    key-tile-major schedule.  Per task u, in buffer x = u % 2:
+//    key-tile-major schedule.  Per task u:
 //        S^T = K Q^T,  dP^T = V dO^T                   (MMA, into tensor memory)
 //        P^T = 2^(S^T*scale*log2e - LSE*log2e),  dS^T = P^T (dP^T - delta)
-//                                                      (warpgroup x, thread = key)
+//                                                      (warpgroup u % 2, thread = key)
 //        dV += P^T dO,  dK += dS^T Q                   (MMA, P^T and dS^T from
 //                                                       tensor memory)
 //    Two warpgroups take alternate tasks so one computes while the MMAs of
 //    the other run.  Two MMA-issuing warps split the MMAs by role: one
-//    issues S^T/dP^T (writing only the task buffers), the other the gradient
-//    MMAs (the only writer of dK and dV), so each issues half the
-//    instructions and neither waits on the other's barriers.  Warpgroup x
-//    releases S^T/dP^T of task u as soon as it has read them (S_FREE) and
-//    S^T/dP^T of task u+2 go into the same buffer at once, so the next
-//    task's scores are ready when the warpgroup finishes; P^T/dS^T of task
-//    u+2 are written only after the gradient MMAs of task u complete
-//    (G_DONE).  A Q/dO stage is released by the gradient issuer: the score
-//    MMAs of its task completed before P^T of the task existed.
-//    dK is scaled by softmax_scale in the epilogue.
+//    issues S^T/dP^T (writing only the score region), the other the gradient
+//    MMAs (the only writer of dK and dV), so neither waits on the other's
+//    barriers.  The scores are released (S_FREE) as soon as a warpgroup
+//    holds them in registers; P^T/dS^T of a warpgroup's task are written only
+//    after the gradient MMAs of its previous task complete (G_DONE).  A Q/dO
+//    stage is released by the gradient issuer: the score MMAs of its task
+//    completed before P^T of the task existed.  dK is scaled by
+//    softmax_scale in the epilogue.  Two forms:
+//    dkdv_sm100_kernel (d = 128): K and V stay in tensor memory as the A
+//      operands of S^T and dP^T, so every MMA reads only Q or dO from shared
+//      memory (two shared-memory operands cap an MMA at 128 bytes per
+//      cycle); one score region (the 512 columns hold K, V, dK, dV, the
+//      scores and two P^T/dS^T regions), 32-query tasks;
+//    dkdv_sm100_ss_kernel (d = 64): K and V in shared memory, two full task
+//      buffers (scores of task u+2 land in buffer u % 2 while the other
+//      warpgroup works), 64-query tasks.
 //
 // 3. dq_sm100_kernel, query-tile major like the forward: per visible key tile
 //        S = Q K^T,  dP = dO V^T,  dS = P (dP - delta),  dQ += dS K.
@@ -45,6 +51,8 @@
 // tcgen05.commit tracks every earlier MMA of the issuing thread.  Every
 // mbarrier wait is bounded and reports a timeout through the error word.
 #include <math_constants.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -99,6 +107,38 @@ struct BwdArgs {
     int npair;
 };
 
+// Grid order of the key-major dK/dV pass: the sink tile (key tile 0, seen
+// by every query) of every (KV head, batch) first, then (batch, KV head)
+// after (batch, KV head) with their key tiles ascending, so the CTAs resident
+// together are neighbouring key tiles of one head, which read the same query
+// rows (measured at 32K, d = 128: DRAM reads 9.0 -> 1.6 GB per launch, L2 hit
+// rate 63 -> 91 %); the long sink CTAs start in the first wave.
+// A packed batch's CTA takes item blockIdx.x / Hkv of the key-major work
+// list instead; false when it has no item.
+__device__ __forceinline__ bool dkdv_order(const AttnParams &p, int &kt, int &hl, int &b)
+{
+    if (p.work) {
+        const int2 it = p.work[blockIdx.x / (unsigned)p.Hkv];
+        hl = (int)(blockIdx.x % (unsigned)p.Hkv);
+        b = it.x;
+        kt = it.y;
+        return it.x >= 0;
+    }
+    const unsigned hb_n = (unsigned)p.Hkv * (unsigned)p.B, lin = blockIdx.x;
+    if (lin < hb_n) {
+        kt = 0;
+        b = (int)(lin / (unsigned)p.Hkv);
+        hl = (int)(lin % (unsigned)p.Hkv);
+    } else {
+        const unsigned per = (unsigned)(p.nkt - 1), r = lin - hb_n, hb = r / per;
+        kt = 1 + (int)(r - hb * per);
+        b = (int)(hb / (unsigned)p.Hkv);
+        hl = (int)(hb % (unsigned)p.Hkv);
+    }
+    return true;
+}
+
+// dK/dV, d = 128: K and V resident in tensor memory.
 // Tensor-memory plan of a dK/dV CTA (512 columns, 128 lanes = its keys):
 //   [0, D)            dK accumulator (fp32)
 //   [D, 2D)           dV accumulator (fp32)
@@ -161,26 +201,8 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
     const uint32_t KV_TM = bar0 + 8u * (12 + 2 * ST);  // K and V are in tensor memory
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // order: the sink tile (key tile 0, seen by every query) of every
-    // (KV head, batch) first, then (batch, KV head) after (batch, KV head)
-    // with their key tiles ascending, so the CTAs resident together are
-    // neighbouring key tiles of one head, which read the same query rows
-    // (measured at 32K: DRAM reads 9.0 -> 1.6 GB per launch, L2 hit rate 63 ->
-    // 91 %); the long sink CTAs start in the first wave
     int kt, hl, b;
-    {
-        const unsigned hb_n = (unsigned)p.Hkv * (unsigned)p.B, lin = blockIdx.x;
-        if (lin < hb_n) {
-            kt = 0;
-            b = (int)(lin / (unsigned)p.Hkv);
-            hl = (int)(lin % (unsigned)p.Hkv);
-        } else {
-            const unsigned per = (unsigned)(p.nkt - 1), r = lin - hb_n, hb = r / per;
-            kt = 1 + (int)(r - hb * per);
-            b = (int)(hb / (unsigned)p.Hkv);
-            hl = (int)(hb % (unsigned)p.Hkv);
-        }
-    }
+    if (!dkdv_order(p, kt, hl, b)) return;
     const SeqGeom sg = seq_geom(p, b);
     const int c0 = kt * BN;
     if (c0 >= sg.Lk) return;  // past the end of this sequence of a packed batch
@@ -509,6 +531,363 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
     if (warp == 9) tmem_dealloc(tmem, 512);
 }
 
+// ---------------------------------------------------------- dK/dV, d = 64 --
+// At d = 64 the accumulators take 128 columns and two full task buffers
+// (S^T, dP^T, P^T, dS^T of 64 queries, 192 columns each) fit beside them, but
+// not K and V as well: this kernel reads K and V from shared memory (their
+// score MMAs are then paced by shared-memory bandwidth) and double-buffers
+// the scores instead, which measured faster at d = 64 (0.30 ms against 0.43
+// ms for the resident-K/V form with one score region, recall8k).  Task
+// pipeline as described at the top of this file.
+template <int D>
+struct KvSsCfg {
+    static constexpr int BN = kBwd5KeyTile;  // keys per CTA
+    static constexpr int BM = bwd5_kv_bm(D);  // queries per task
+    static constexpr int ST = 8;  // Q/dO stages (8 measured 2 % faster than 6, 4 % than 4)
+    static constexpr int KB = D / 64;
+    static constexpr int KV_BYTES = BN * D * 2;
+    static constexpr int QT_BYTES = BM * D * 2;
+    static constexpr int LSD_BYTES = BM * 8;
+    static constexpr int STAGE_BYTES = (2 * QT_BYTES + LSD_BYTES + 1023) / 1024 * 1024;
+    // tensor memory: dK, dV, then two buffers of S^T, dP^T, P^T (bf16), dS^T (bf16)
+    static constexpr int T_DK = 0, T_DV = D, T_BUF = 2 * D, BUF = 3 * BM;
+    static constexpr int NBAR = 12 + 2 * ST;
+    static constexpr int SMEM = 1024 + 2 * KV_BYTES + ST * STAGE_BYTES + 8 * NBAR + 16;
+    static constexpr uint32_t IDESC_S = idesc_bf16(128, BM, 0, 0);
+    static constexpr uint32_t IDESC_G = idesc_bf16(128, D, 0, 1);
+};
+
+template <int D>
+__global__ void __launch_bounds__(352, 1) dkdv_sm100_ss_kernel(const __grid_constant__ BwdArgs a)
+{
+    using C = KvSsCfg<D>;
+    constexpr int BN = C::BN, BM = C::BM, ST = C::ST, KB = C::KB;
+    const AttnParams &p = a.p;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char *sm = smem_raw + (base - raw);
+    const uint32_t sK = base, sV = base + C::KV_BYTES, sStage = base + 2 * C::KV_BYTES;
+    auto stage_q = [&](int s) { return sStage + s * C::STAGE_BYTES; };
+    auto stage_do = [&](int s) { return sStage + s * C::STAGE_BYTES + C::QT_BYTES; };
+    auto stage_lsd = [&](int s) {
+        return reinterpret_cast<const float2 *>(sm + 2 * C::KV_BYTES + s * C::STAGE_BYTES + 2 * C::QT_BYTES);
+    };
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 2 * C::KV_BYTES + ST * C::STAGE_BYTES);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const uint32_t bar0 = smem_addr(bars);
+    const uint32_t KV_LOADED = bar0;
+    auto Q_FULL = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto Q_EMPTY = [&](int s) { return bar0 + 8u * (1 + ST + s); };
+    auto S_FULL = [&](int x) { return bar0 + 8u * (1 + 2 * ST + x); };
+    auto P_FULL = [&](int x) { return bar0 + 8u * (3 + 2 * ST + x); };
+    const uint32_t DONE = bar0 + 8u * (5 + 2 * ST);
+    auto FIN = [&](int r) { return bar0 + 8u * (r == 0 ? 6 + 2 * ST : 11 + 2 * ST); };  // per issuer
+    auto S_FREE = [&](int x) { return bar0 + 8u * (7 + 2 * ST + x); };
+    auto G_DONE = [&](int x) { return bar0 + 8u * (9 + 2 * ST + x); };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    int kt, hl, b;
+    if (!dkdv_order(p, kt, hl, b)) return;
+    const SeqGeom sg = seq_geom(p, b);
+    const int c0 = kt * BN;
+    if (c0 >= sg.Lk) return;  // past the end of this sequence of a packed batch
+    const Win w = make_win(p.S, p.N, p.G, p.W, (long long)hl + p.kv_head_offset);
+    const int delta_pos = sg.Lk - sg.Lq;
+
+    // the query tiles that see this key tile, from the same closed form as
+    // the schedule builder
+    const TileRanges tr = key_tile_ranges(c0, min(c0 + BN, sg.Lk) - 1, sg.Lq, sg.Lk, w, BM);
+    const int nr = tr.n;
+    const int lo0 = tr.lo0, lo1 = tr.lo1, lo2 = tr.lo2;
+    const int len0 = tr.len0, len1 = tr.len1, len2 = tr.len2;
+    const int nq = (nr > 0 ? len0 : 0) + (nr > 1 ? len1 : 0) + (nr > 2 ? len2 : 0);
+    const int ntask = nq * p.g;
+    auto task = [&](int u, int &hq, int &qt) {
+        hq = hl * p.g + u / nq;
+        int t = u % nq;
+        if (t < len0 || nr == 1) { qt = lo0 + t; return; }
+        t -= len0;
+        if (t < len1 || nr == 2) { qt = lo1 + t; return; }
+        qt = lo2 + t - len1;
+    };
+
+    if (tid == 0) {
+        mbar_init(KV_LOADED, 1);
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(Q_FULL(s), 1);
+            mbar_init(Q_EMPTY(s), 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(S_FULL(x), 1);
+            mbar_init(P_FULL(x), 128);
+            mbar_init(S_FREE(x), 4);  // one arrival per warp
+            mbar_init(G_DONE(x), 1);
+        }
+        mbar_init(DONE, 1);
+        mbar_init(FIN(0), 1);
+        mbar_init(FIN(1), 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_addr(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tmap(&a.tq);
+        prefetch_tmap(&a.tk);
+        prefetch_tmap(&a.tv);
+        prefetch_tmap(&a.tdo);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ TMA
+        if (lane == 0) {
+            mbar_expect_tx(KV_LOADED, 2 * C::KV_BYTES);
+            for (int kb = 0; kb < KB; ++kb) {
+                tma_load_4d(sK + kb * BN * 128, &a.tk, KV_LOADED, kb * 64, sg.koff + c0, hl, sg.tb);
+                tma_load_4d(sV + kb * BN * 128, &a.tv, KV_LOADED, kb * 64, sg.koff + c0, hl, sg.tb);
+            }
+            int issued = 0;
+            for (int u = 0; u < ntask; ++u) {
+                const int s = u % ST;
+                if (u >= ST && !mbar_wait(Q_EMPTY(s), ((u / ST) - 1) & 1, p.err, abort_flag)) break;
+                int hq, qt;
+                task(u, hq, qt);
+                // a listed query tile holds rows; its row pairs lie in the workspace
+                if (!dcheck(qt >= 0 && qt * BM < sg.Lq && (qt + 1) * BM <= a.lq_pad && hq >= hl * p.g &&
+                                hq < (hl + 1) * p.g,
+                            p.err)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                mbar_expect_tx(Q_FULL(s), 2 * C::QT_BYTES + C::LSD_BYTES);
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_4d(stage_q(s) + kb * BM * 128, &a.tq, Q_FULL(s), kb * 64, sg.qoff + qt * BM, hq, sg.tb);
+                    tma_load_4d(stage_do(s) + kb * BM * 128, &a.tdo, Q_FULL(s), kb * 64, sg.qoff + qt * BM, hq, sg.tb);
+                }
+                bulk_load(stage_q(s) + 2 * C::QT_BYTES,
+                          a.lsd + ((long long)b * p.Hq + hq) * a.lq_pad + (long long)qt * BM, C::LSD_BYTES,
+                          Q_FULL(s));
+                issued = u + 1;
+            }
+            mbar_wait(KV_LOADED, 0, p.err, abort_flag);
+            for (int u = issued > ST ? issued - ST : 0; u < issued; ++u)
+                mbar_wait(Q_FULL(u % ST), (u / ST) & 1, p.err, abort_flag);
+        }
+    } else if (warp == 9 || warp == 10) {
+        // ------------------------------------------------------------ MMA
+        // the whole warp runs the loop; one elected lane issues.  Warp 9
+        // issues the score MMAs, warp 10 the gradient MMAs.
+        const uint32_t FULL = 0xffffffffu;
+        const int role = warp - 9;
+        bool ok = __all_sync(FULL, mbar_wait(KV_LOADED, 0, p.err, abort_flag));
+        const uint64_t dk0 = sdesc(sK, 16, 1024), dv0 = sdesc(sV, 16, 1024);
+        const uint64_t dq0 = sdesc(stage_q(0), 16, 1024), ddo0 = sdesc(stage_do(0), 16, 1024);
+        const uint64_t dqm0 = sdesc(stage_q(0), BM * 128, 1024), ddom0 = sdesc(stage_do(0), BM * 128, 1024);
+        auto sdp = [&](int u) -> bool {  // S^T, dP^T of task u into buffer u % 2
+            const int s = u % ST, x = u & 1;
+            if (!__all_sync(FULL, mbar_wait(Q_FULL(s), (u / ST) & 1, p.err, abort_flag))) return false;
+            tc_fence_after();
+            const uint32_t tb = tmem + C::T_BUF + x * C::BUF;
+            const uint32_t so = (uint32_t)s * C::STAGE_BYTES;
+            if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ko = (kk >> 2) * BN * 128 + (kk & 3) * 32;
+                    const uint32_t qo = so + (kk >> 2) * BM * 128 + (kk & 3) * 32;
+                    mma_ss(tb, sdesc_add(dk0, ko), sdesc_add(dq0, qo), C::IDESC_S, kk > 0);
+                    mma_ss(tb + BM, sdesc_add(dv0, ko), sdesc_add(ddo0, qo), C::IDESC_S, kk > 0);
+                }
+                mma_commit(S_FULL(x));
+            }
+            __syncwarp();
+            return true;
+        };
+        auto grad = [&](int u) -> bool {  // dV += P^T dO, dK += dS^T Q
+            const int s = u % ST, x = u & 1;
+            if (!__all_sync(FULL, mbar_wait(P_FULL(x), (u >> 1) & 1, p.err, abort_flag))) return false;
+            tc_fence_after();
+            const uint32_t tb = tmem + C::T_BUF + x * C::BUF;
+            const uint32_t so = (uint32_t)s * C::STAGE_BYTES;
+            if (elect_one()) {
+#pragma unroll
+                for (int k2 = 0; k2 < BM / 16; ++k2) {
+                    const uint32_t acc = (u > 0 || k2 > 0) ? 1u : 0u;
+                    mma_ts(tmem + C::T_DV, tb + 2 * BM + k2 * 8, sdesc_add(ddom0, so + k2 * 2048), C::IDESC_G, acc);
+                    mma_ts(tmem + C::T_DK, tb + 2 * BM + BM / 2 + k2 * 8, sdesc_add(dqm0, so + k2 * 2048), C::IDESC_G,
+                           acc);
+                }
+                mma_commit(Q_EMPTY(s));
+                mma_commit(G_DONE(x));
+            }
+            __syncwarp();
+            return true;
+        };
+        if (role == 0) {
+            for (int u = 0; ok && u < ntask; ++u) {
+                if (u >= 2) {
+                    // warpgroup u % 2 has read S^T and dP^T of task u-2
+                    if (!(ok = __all_sync(FULL, mbar_wait(S_FREE(u & 1), ((u - 2) >> 1) & 1, p.err, abort_flag))))
+                        break;
+                    tc_fence_after();
+                }
+                ok = sdp(u);
+            }
+        } else {
+            for (int u = 0; ok && u < ntask; ++u) ok = grad(u);
+            if (elect_one()) mma_commit(DONE);  // every gradient MMA; the score MMAs completed before them
+            __syncwarp();
+        }
+        if (elect_one()) mma_commit(FIN(role));
+        __syncwarp();
+        mbar_wait(FIN(role), 0, p.err, abort_flag);
+    } else {
+        // ---------------------------------------------- P^T and dS^T per key
+        const int x = warp >> 2;
+        const int jl = (warp & 3) * 32 + lane;  // key row within the tile
+        const int jg = c0 + jl;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tb = tmem + C::T_BUF + x * C::BUF + lane_off;
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        // the aligned positions that see key jg (sink, near, long), as runs
+        // formed once: a task's columns need no mask when one run holds them
+        const Runs3 kr = key_pos_runs(jg, w, sg.Lk - 1);
+        // this warpgroup's tasks u = x, x+2, ...: query head gi of the group
+        // and position t in the key tile's query-tile list, advanced without
+        // division
+        int gi = nq > 0 ? x / nq : 0, tq = nq > 0 ? x % nq : 0;
+        bool ok = true;
+        // MALA block decisions of this key's column for the group's first
+        // query head (nullptr for CoWA)
+        const uint8_t *kbase = p.keep ? p.keep + ((long long)b * p.Hq + hl * p.g) * p.keep_nqt * p.keep_nkt +
+                                            jg / kMalaBN
+                                      : nullptr;
+        for (int k = 0;; ++k) {
+            const int u = 2 * k + x;
+            if (u >= ntask) break;
+            // task set-up, independent of the scores: done while they land
+            const int qt = tq < len0 || nr == 1 ? lo0 + tq
+                           : (tq - len0 < len1 || nr == 2 ? lo1 + tq - len0 : lo2 + tq - len0 - len1);
+            // MALA: a key of a skipped block has dP = 0 and no dV share
+            const bool skip = kbase && !kbase[(gi * p.keep_nqt + qt * BM / kMalaBM) * p.keep_nkt];
+            tq += 2;
+            while (tq >= nq) {
+                tq -= nq;
+                ++gi;
+            }
+            const int q0 = qt * BM;
+            const int nrows = min(BM, sg.Lq - q0);
+            const int pa = q0 + delta_pos, pb = pa + nrows - 1;
+            // no mask when every key of the warp sees every in-range column
+            const bool full = __all_sync(0xffffffffu, runs_cover(kr, pa, pb));
+            uint32_t vis[BM / 32];
+            if (!full) {
+#pragma unroll
+                for (int c = 0; c < BM / 32; ++c)  // columns p = pa + c*32 + bit, in range up to pb
+                    vis[c] = runs_bits(kr, pa + c * 32) & span_bits(0, pb - pa - c * 32);
+            }
+            const float2 *lsd = stage_lsd(u % ST);
+            ok = __all_sync(0xffffffffu, mbar_wait(S_FULL(x), k & 1, p.err, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < BM / 32; ++c) {
+                uint32_t sr[32], dr[32];
+                tmem_ld32(tb + c * 32, sr);
+                tmem_ld32(tb + BM + c * 32, dr);
+                tmem_wait_ld();
+                if (c == BM / 32 - 1) {
+                    // all of S^T and dP^T read: S^T/dP^T of task u+2 may land
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(S_FREE(x));
+                }
+                if (!full) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (!((vis[c] >> e) & 1u)) sr[e] = __float_as_uint(-CUDART_INF_F);
+                }
+                if (skip) {  // MALA skipped block: dP = 0
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) dr[e] = 0u;
+                }
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float4 ld = *reinterpret_cast<const float4 *>(lsd + c * 32 + 2 * e);  // (-lse2, -delta) x2
+                    const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
+                                                 sc2, make_float2(ld.x, ld.z));
+                    const float2 pr = make_float2(fast_ex2(xa.x), fast_ex2(xa.y));
+                    const float2 t = __fadd2_rn(make_float2(__uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1])),
+                                                make_float2(ld.y, ld.w));
+                    const float2 ds = __fmul2_rn(pr, t);
+                    pk[e] = pack2(pr.x, pr.y);
+                    dk[e] = pack2(ds.x, ds.y);
+                }
+                if (c == 0 && k > 0) {
+                    // the gradient MMAs of task u-2 read P^T/dS^T of this buffer
+                    // (G_DONE(x) has completed k-1 or k phases)
+                    ok = __all_sync(0xffffffffu, mbar_wait(G_DONE(x), (k - 1) & 1, p.err, abort_flag));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                if (skip) {  // and no share of dV
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                }
+                tmem_st16(tb + 2 * BM + c * 16, pk);
+                tmem_st16(tb + 2 * BM + BM / 2 + c * 16, dk);
+            }
+            if (!ok) break;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(P_FULL(x));
+        }
+        // epilogue: warpgroup 0 writes dK (scaled), warpgroup 1 writes dV
+        ok = __all_sync(0xffffffffu, mbar_wait(DONE, 0, p.err, abort_flag) && ok);
+        tc_fence_after();
+        const bool have = ok && ntask > 0;
+        const float f = x == 0 ? p.scale : 1.f;
+        const uint32_t tg = tmem + (x == 0 ? C::T_DK : C::T_DV) + lane_off;
+        __nv_bfloat16 *grow_ = x == 0
+            ? reinterpret_cast<__nv_bfloat16 *>(p.dk) + sg.tb * p.ks[0] + (long long)(sg.koff + jg) * p.ks[1] +
+                  hl * p.ks[2]
+            : reinterpret_cast<__nv_bfloat16 *>(p.dv) + sg.tb * p.vs[0] + (long long)(sg.koff + jg) * p.vs[1] +
+                  hl * p.vs[2];
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+            uint32_t g[16];
+            if (have) {
+                tmem_ld16(tg + c * 16, g);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) g[e] = 0u;
+            }
+            uint32_t pk[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pk[e] = pack2(__uint_as_float(g[2 * e]) * f, __uint_as_float(g[2 * e + 1]) * f);
+            if (jg < sg.Lk && dcheck(sg.koff + jg < (p.cu_q ? p.total_k : p.Lk), p.err)) {
+                uint4 *dst = reinterpret_cast<uint4 *>(grow_ + c * 16);
+                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
 // --------------------------------------------------------------------- dQ --
 template <int D>
 struct DqCfg {
@@ -556,12 +935,11 @@ __global__ void __launch_bounds__(352, 1) dq_sm100_kernel(const __grid_constant_
     auto S_FREE = [&](int x) { return bar0 + 8u * (8 + 2 * ST + x); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const TilePos pos = tile_pos(p.Hkv * a.npair, p.B);
-    const int qt = p.nqt - 1 - pos.step;  // long rows first
-    const int hl = pos.slot / a.npair, pair = pos.slot % a.npair;
+    int qt, slot, b;  // long rows first
+    if (!query_tile_item(p, p.Hkv * a.npair, a.npair, qt, slot, b)) return;
+    const int hl = slot / a.npair, pair = slot % a.npair;
     const int hq0 = hl * p.g + NSLOT * pair;
     const int nslot = min(NSLOT, p.g - NSLOT * pair);
-    const int b = pos.b;
     const SeqGeom sg = seq_geom(p, b);
     const int i0 = qt * BM;
     if (i0 >= sg.Lq) return;  // past the end of this sequence of a packed batch
@@ -882,10 +1260,9 @@ __global__ void __launch_bounds__(352, 1) dq_tm_kernel(const __grid_constant__ B
     const uint32_t QD_TM = bar0 + 8u * (9 + 2 * ST);  // Q and dO are in tensor memory
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const TilePos pos = tile_pos(p.Hq, p.B);
-    const int qt = p.nqt - 1 - pos.step;  // long rows first
-    const int hq = pos.slot, hl = hq / p.g;
-    const int b = pos.b;
+    int qt, hq, b;  // long rows first
+    if (!query_tile_item(p, p.Hq, p.g, qt, hq, b)) return;
+    const int hl = hq / p.g;
     const SeqGeom sg = seq_geom(p, b);
     const int i0 = qt * BM;
     if (i0 >= sg.Lq) return;  // past the end of this sequence of a packed batch
@@ -1145,16 +1522,21 @@ __global__ void __launch_bounds__(352, 1) dq_tm_kernel(const __grid_constant__ B
 // ----------------------------------------------------------------- host ----
 template <int D>
 static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, int nqt_dq, int nkt_kv,
-                                 cudaStream_t st)
+                                 const int2 *work_q, int work_q_n, const int2 *work_k, int work_k_n, cudaStream_t st)
 {
-    using K = KvCfg<D>;
+    using K = typename std::conditional<D == 128, KvCfg<128>, KvSsCfg<64>>::type;
     using Q = DqCfg<D>;
     static std::atomic<bool> configured[64];
     cudaError_t e = once_per_device(configured, [] {
-        cudaError_t r = cudaFuncSetAttribute(dkdv_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
-        if (r != cudaSuccess) return r;
-        return D == 128 ? cudaFuncSetAttribute(dq_tm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DqTmCfg::SMEM)
-                        : cudaFuncSetAttribute(dq_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Q::SMEM);
+        if constexpr (D == 128) {
+            cudaError_t r = cudaFuncSetAttribute(dkdv_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
+            if (r != cudaSuccess) return r;
+            return cudaFuncSetAttribute(dq_tm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DqTmCfg::SMEM);
+        } else {
+            cudaError_t r = cudaFuncSetAttribute(dkdv_sm100_ss_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
+            if (r != cudaSuccess) return r;
+            return cudaFuncSetAttribute(dq_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, Q::SMEM);
+        }
     });
     if (e != cudaSuccess) return e;
     const long long rows = (long long)p.B * p.Hq * lq_pad;
@@ -1182,11 +1564,16 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, i
         !make_bshd_map(&a.tv, p.v, D, Lk_map, p.Hkv, B_map, p.vs, K::BN))
         return cudaErrorInvalidValue;
     a.p.nkt = nkt_kv;
+    a.p.work = work_k;  // packed batch: the key-major work list
+    a.p.work_n = work_k_n;
     if (nkt_kv > 0) {
-        const unsigned g1 = tile_grid_blocks(nkt_kv, p.Hkv, p.B);
+        const unsigned g1 = work_k ? tile_grid_blocks(work_k_n, p.Hkv, 1) : tile_grid_blocks(nkt_kv, p.Hkv, p.B);
         if (!g1) return cudaErrorInvalidConfiguration;
         launch_begin("dkdv_sm100", st);
-        dkdv_sm100_kernel<D><<<g1, 352, K::SMEM, st>>>(a);
+        if constexpr (D == 128)
+            dkdv_sm100_kernel<128><<<g1, 352, K::SMEM, st>>>(a);
+        else
+            dkdv_sm100_ss_kernel<64><<<g1, 352, K::SMEM, st>>>(a);
         launch_end(st);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
@@ -1199,36 +1586,36 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, i
         !make_bshd_map(&a.tv, p.v, D, Lk_map, p.Hkv, B_map, p.vs, dq_bn))
         return cudaErrorInvalidValue;
     a.p.nqt = nqt_dq;
-    if (D == 128) {
-        // one query head per CTA, Q and dO resident in tensor memory
-        if (nqt_dq > 0) {
-            const unsigned g2 = tile_grid_blocks(nqt_dq, p.Hq, p.B);
+    a.p.work = work_q;  // packed batch: the query-major work list
+    a.p.work_n = work_q_n;
+    if (nqt_dq > 0) {
+        if constexpr (D == 128) {
+            // one query head per CTA, Q and dO resident in tensor memory
+            const unsigned g2 = work_q ? tile_grid_blocks(work_q_n, p.Hq, 1) : tile_grid_blocks(nqt_dq, p.Hq, p.B);
             if (!g2) return cudaErrorInvalidConfiguration;
             launch_begin("dq_sm100", st);
             dq_tm_kernel<<<g2, 352, DqTmCfg::SMEM, st>>>(a);
             launch_end(st);
-            e = cudaGetLastError();
+        } else {
+            a.npair = (p.g + Q::NSLOT - 1) / Q::NSLOT;
+            const unsigned g2 = work_q ? tile_grid_blocks(work_q_n, (long long)p.Hkv * a.npair, 1)
+                                       : tile_grid_blocks(nqt_dq, (long long)p.Hkv * a.npair, p.B);
+            if (!g2) return cudaErrorInvalidConfiguration;
+            launch_begin("dq_sm100", st);
+            dq_sm100_kernel<64><<<g2, 352, Q::SMEM, st>>>(a);
+            launch_end(st);
         }
-        return e;
-    }
-    a.npair = (p.g + Q::NSLOT - 1) / Q::NSLOT;
-    if (nqt_dq > 0) {
-        const unsigned g2 = tile_grid_blocks(nqt_dq, (long long)p.Hkv * a.npair, p.B);
-        if (!g2) return cudaErrorInvalidConfiguration;
-        launch_begin("dq_sm100", st);
-        dq_sm100_kernel<D><<<g2, 352, Q::SMEM, st>>>(a);
-        launch_end(st);
         e = cudaGetLastError();
     }
     return e;
 }
 
 cudaError_t launch_bwd_sm100(const AttnParams &p, int D, float2 *lsd, int lq_pad, int nqt_dq, int nkt_kv,
-                             cudaStream_t st)
+                             cudaStream_t st, const int2 *work_q, int work_q_n, const int2 *work_k, int work_k_n)
 {
     if (p.B == 0 || p.Hq == 0) return cudaSuccess;
-    return D == 128 ? launch_bwd5_d<128>(p, lsd, lq_pad, nqt_dq, nkt_kv, st)
-                    : launch_bwd5_d<64>(p, lsd, lq_pad, nqt_dq, nkt_kv, st);
+    return D == 128 ? launch_bwd5_d<128>(p, lsd, lq_pad, nqt_dq, nkt_kv, work_q, work_q_n, work_k, work_k_n, st)
+                    : launch_bwd5_d<64>(p, lsd, lq_pad, nqt_dq, nkt_kv, work_q, work_q_n, work_k, work_k_n, st);
 }
 
 }  // namespace cowa

@@ -116,12 +116,11 @@ __global__ void __launch_bounds__(352, 1) fwd_sm100_kernel(const __grid_constant
     auto TURN = [&](int x, int qd) { return bar0 + 8u * (12 + 2 * ST + 4 * x + qd); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const TilePos pos = tile_pos(p.Hkv * a.npair, p.B);
-    const int qt = p.nqt - 1 - pos.step;  // long rows first
-    const int hl = pos.slot / a.npair, pair = pos.slot % a.npair;
+    int qt, slot, b;  // long rows first
+    if (!query_tile_item(p, p.Hkv * a.npair, a.npair, qt, slot, b)) return;
+    const int hl = slot / a.npair, pair = slot % a.npair;
     const int hq0 = hl * p.g + 2 * pair;
     const int nslot = (2 * pair + 1 < p.g) ? 2 : 1;  // an odd group leaves the last head alone
-    const int b = pos.b;
     const SeqGeom sg = seq_geom(p, b);
     const int i0 = qt * BM;
     if (i0 >= sg.Lq) return;  // past the end of this sequence of a packed batch
@@ -523,7 +522,8 @@ static cudaError_t launch_fwd5_d(const AttnParams &p, cudaStream_t st)
         !make_bshd_map(&a.tk, p.k, D, Lk_map, p.Hkv, B_map, p.ks, C::BN) ||
         !make_bshd_map(&a.tv, p.v, D, Lk_map, p.Hkv, B_map, p.vs, C::BN))
         return cudaErrorInvalidValue;
-    const unsigned blocks = tile_grid_blocks(p.nqt, (long long)p.Hkv * a.npair, p.B);
+    const unsigned blocks = p.work ? tile_grid_blocks(p.work_n, (long long)p.Hkv * a.npair, 1)
+                                   : tile_grid_blocks(p.nqt, (long long)p.Hkv * a.npair, p.B);
     if (!blocks) return cudaErrorInvalidConfiguration;
     launch_begin("fwd_sm100", st);
     fwd_sm100_kernel<D><<<blocks, 352, C::SMEM, st>>>(a);

@@ -71,7 +71,43 @@ struct AttnParams {
     // and contributes nothing to dV (only -P * delta remains in dS)
     const uint8_t *keep;
     int keep_nqt, keep_nkt;
+    // Packed batch: the (sequence, tile) items of the launch's tiling, heavy
+    // tiles first (worklist.cu), work_n entries (the last ones (-1, -1));
+    // the grid is work_n x head slots.  nullptr for a uniform batch.
+    const int2 *work;
+    int work_n;
 };
+
+// The tile, head slot and batch entry of a CTA of a query-major pass
+// (forward, dQ), whose head slots are numbered KV head by KV head (spk slots
+// each).  A uniform batch's 1-D grid runs over groups of two KV heads
+// (one for an odd count), and within a group over (head slot, batch)
+// fastest and the tile step slowest, the last query tile first: the CTAs
+// resident together then read the K/V windows of two KV heads only, which
+// L2 holds (all KV heads' windows at 128K are about 100 MB), and each
+// group's long CTAs start before its short ones.  A packed batch's CTA
+// takes item blockIdx.x / nslot of the work list.  False when the CTA has
+// no item.
+__device__ __forceinline__ bool query_tile_item(const AttnParams &p, int nslot, int spk, int &qt, int &slot, int &b)
+{
+    if (p.work) {
+        const int2 it = p.work[blockIdx.x / (unsigned)nslot];
+        slot = (int)(blockIdx.x % (unsigned)nslot);
+        b = it.x;
+        qt = it.y;
+        return it.x >= 0;
+    }
+    const unsigned gs = (unsigned)spk * ((p.Hkv % 2 == 0) ? 2u : 1u);  // head slots per group
+    const unsigned per = gs * (unsigned)p.B, lin = blockIdx.x;
+    const unsigned grp_n = per * (unsigned)p.nqt;
+    const unsigned grp = lin / grp_n, rg = lin - grp * grp_n;
+    const int step = (int)(rg / per);
+    const unsigned r = rg - (unsigned)step * per;
+    b = (int)(r / gs);
+    slot = (int)(grp * gs + (r - (unsigned)b * gs));
+    qt = p.nqt - 1 - step;
+    return true;
+}
 
 // Lengths and row offsets of sequence b, and its batch coordinate (b for a
 // uniform batch, 0 for a packed one, whose rows are offsets into batch 0).
@@ -166,6 +202,15 @@ bool make_bshd_map(CUtensorMap *m, const void *base, int d, long long L, long lo
 constexpr int kMalaBM = 128, kMalaBN = 64;
 cudaError_t launch_mala_fwd(const AttnParams &p, int D, uint8_t *keep, float tau, cudaStream_t st);
 
+// worklist.cu: the (sequence, tile) items of a packed batch for tiles of
+// `tile` rows of the offsets cu [B + 1] (descending: the query-major order,
+// last tile of each sequence first; else ascending: the key-major order),
+// max_items entries (>= sum of the sequences' tile counts; the rest
+// (-1, -1)); scratch: 3 * (max_tiles + 1) ints, max_tiles >= any
+// sequence's tile count
+cudaError_t launch_varlen_worklist(const int *cu, int B, int tile, int max_tiles, bool descending, int2 *list,
+                                   int max_items, int *scratch, int *err, cudaStream_t st);
+
 // fill.cu: constant outputs of the shapes the tcgen05 kernels do not take
 // (zero rows of a strided [B, L, H, D] bf16 tensor; a constant fp32 array)
 cudaError_t launch_zero_rows(void *t, const long long st[3], int B, int L, int H, int D, cudaStream_t s);
@@ -173,20 +218,21 @@ cudaError_t launch_fill_f32(float *p, long long n, float v, cudaStream_t s);
 
 
 // bwd_sm100.cu (tcgen05 backward: preprocess, dK/dV pass, dQ pass)
+// work_q / work_k: the query- and key-major work lists of a packed batch
+// (nullptr for a uniform batch)
 cudaError_t launch_bwd_sm100(const AttnParams &p, int D, float2 *lsd, int lq_pad, int nqt_dq, int nkt_kv,
-                             cudaStream_t st);
+                             cudaStream_t st, const int2 *work_q = nullptr, int work_q_n = 0,
+                             const int2 *work_k = nullptr, int work_k_n = 0);
 constexpr int kBwd5KeyTile = 128;   // keys per dK/dV CTA (tensor-memory lanes)
 constexpr int kBwd5QTile = 128;     // queries per dQ CTA
 __host__ __device__ constexpr int bwd5_kv_bm(int D) { return D == 128 ? 32 : 64; }    // queries per dK/dV task
 __host__ __device__ constexpr int bwd5_dq_bn(int D) { return D == 128 ? 128 : 64; }   // keys per dQ tile
 inline long long bwd5_lq_pad(long long Lq) { return (Lq + 63) / 64 * 64; }
 
-// Launch order of the query-major tcgen05 kernels (forward, dQ): a 1-D grid
-// whose block index runs over (head slot, batch) fastest and over the tile
-// step slowest.  The kernels map step 0 to the heaviest tile of every head
-// (the last query tile), so the long CTAs start in the first waves and the
-// short ones fill the tail.  (The key-major dK/dV pass orders its own grid:
-// sink tiles first, then key tiles ascending head by head.)
+// 1-D grid position of the MALA forward: (query head, batch) fastest, the
+// tile step slowest (its kernel maps step 0 to the last query tile).  The
+// CoWA passes use query_tile_item above and the dK/dV pass its own order
+// (sink tiles first, then key tiles ascending head by head).
 struct TilePos {
     int step, slot, b;
 };

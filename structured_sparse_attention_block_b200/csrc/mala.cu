@@ -23,7 +23,11 @@
 //           O += P V runs, a skipped tile issues no PV MMA.
 // The decisions are written to keep[b][hq][query tile][key tile] (1 kept,
 // 0 skipped or beyond the causal diagonal) for the backward.
-// Warps: 0-3 softmax (thread = query row), 4 TMA producer, 5 MMA issuer.
+// Warps: 0-7 softmax, two warpgroups on every tile, warpgroup x on key
+// columns [32x, 32x + 32) of each 64-key tile (thread = query row): pass 1
+// keeps a max and exp-sum per half and merges the halves once at its end;
+// pass 2 adds the two halves' row masses through shared memory before the
+// decision; 8 TMA producer, 9 MMA issuer.
 // Tensor memory: S in two 64-column buffers (pass item i in buffer i % 2, so
 // S of the next tile is computed while the current one is read), P in two
 // 32-column buffers (tile t in buffer t % 2), O (d columns).  Every mbarrier
@@ -56,13 +60,13 @@ struct MalaCfg {
     static constexpr int T_S = 0, T_P = 2 * BN, T_O = 3 * BN;  // S x2, P x2 (BN/2 each), O
     static_assert(T_O + D <= 512, "tensor-memory plan");
     static constexpr int NBAR = 10 + 2 * ST;
-    static constexpr int SMEM = 1024 + Q_BYTES + ST * STAGE_BYTES + 8 * NBAR + 64;
+    static constexpr int SMEM = 1024 + Q_BYTES + ST * STAGE_BYTES + 8 * NBAR + 16 + 64 + 2048 + 1024;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
     static constexpr uint32_t IDESC_O = idesc_bf16(128, D, 0, 1);
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1) mala_fwd_kernel(const __grid_constant__ MalaArgs a)
+__global__ void __launch_bounds__(320, 1) mala_fwd_kernel(const __grid_constant__ MalaArgs a)
 {
     using C = MalaCfg<D>;
     constexpr int BM = C::BM, BN = C::BN, ST = C::ST, KB = C::KB;
@@ -76,7 +80,9 @@ __global__ void __launch_bounds__(192, 1) mala_fwd_kernel(const __grid_constant_
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *kflag = reinterpret_cast<volatile int *>(tmem_slot + 2);  // [2] decision of tile t in t % 2
-    float *red = reinterpret_cast<float *>(tmem_slot + 4);                  // [2][4] per-warp largest mass
+    float *red = reinterpret_cast<float *>(tmem_slot + 4);                  // [2][8] per-warp largest mass
+    float *half = red + 16;                                                 // [2][2][128] row mass per half
+    float2 *stat = reinterpret_cast<float2 *>(half + 512);                  // [128] (max, sum) of columns 32..63
     const uint32_t bar0 = smem_addr(bars);
     const uint32_t BAR_Q = bar0;
     auto KV_FULL = [&](int s) { return bar0 + 8u * (1 + s); };
@@ -106,19 +112,19 @@ __global__ void __launch_bounds__(192, 1) mala_fwd_kernel(const __grid_constant_
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(S_FULL(x), 1);
-            mbar_init(S_FREE(x), 4);  // one arrival per softmax warp
-            mbar_init(P_FULL(x), 128);
+            mbar_init(S_FREE(x), 8);  // one arrival per softmax warp
+            mbar_init(P_FULL(x), 256);
             mbar_init(P_DONE(x), 1);
         }
         mbar_init(FIN, 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(smem_addr(tmem_slot), 512);
         tmem_relinquish();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == 8 && lane == 0) {
         prefetch_tmap(&a.tq);
         prefetch_tmap(&a.tk);
         prefetch_tmap(&a.tv);
@@ -129,7 +135,7 @@ __global__ void __launch_bounds__(192, 1) mala_fwd_kernel(const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     const int nitems = 2 * nt;  // pass 1 tiles, then pass 2 tiles
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------------------ TMA
         if (lane == 0) {
             mbar_expect_tx(BAR_Q, C::Q_BYTES);
@@ -156,7 +162,7 @@ __global__ void __launch_bounds__(192, 1) mala_fwd_kernel(const __grid_constant_
             for (int i = issued > ST ? issued - ST : 0; i < issued; ++i)
                 mbar_wait(KV_FULL(i % ST), (i / ST) & 1, p.err, abort_flag);
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------ MMA
         // the whole warp runs the loop; one elected lane issues
         const uint32_t FULL = 0xffffffffu;
@@ -211,88 +217,117 @@ __global__ void __launch_bounds__(192, 1) mala_fwd_kernel(const __grid_constant_
         mbar_wait(FIN, 0, p.err, abort_flag);
     } else {
         // -------------------------------------------------------- softmax
-        const int r = warp * 32 + lane;  // row of the query tile
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        constexpr int HB = BN / 2;       // columns per warpgroup
+        const int xg = warp >> 2;        // warpgroup: key columns [xg*HB, xg*HB + HB) of a tile
+        const int r = (warp & 3) * 32 + lane;  // row of the query tile
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const int prow = pa + r;
         const bool valid = r < nrows;  // a query row of the sequence
         const float c = p.scale_log2;
         float m = -CUDART_INF_F, l = 0.f;
         bool ok = true;
-        auto load_s = [&](int i, uint32_t (&sr)[BN]) -> bool {
+        auto sync_wgs = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };  // the 8 softmax warps
+        auto load_s = [&](int i, uint32_t (&sr)[HB]) -> bool {
             const int x = i & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(S_FULL(x), (i >> 1) & 1, p.err, abort_flag))) return false;
             tc_fence_after();
-            tmem_ld32(tmem + C::T_S + x * BN + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld32(tmem + C::T_S + x * BN + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            tmem_ld32(tmem + C::T_S + x * BN + xg * HB + lane_off, sr);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(S_FREE(x));
             // causal mask on the tiles that reach past the row's position or
             // past the keys (a whole tile at or before pa is visible)
-            const int j0 = (i < nt ? i : i - nt) * BN;
-            if (j0 + BN - 1 > pa || j0 + BN > p.Lk) {
+            const int j0 = (i < nt ? i : i - nt) * BN + xg * HB;
+            if (j0 + HB - 1 > pa || j0 + HB > p.Lk) {
 #pragma unroll
-                for (int e = 0; e < BN; ++e)
+                for (int e = 0; e < HB; ++e)
                     if (j0 + e > prow || j0 + e >= p.Lk) sr[e] = __float_as_uint(-CUDART_INF_F);
             }
             return true;
         };
-        // pass 1: the row's max and exp-sum over every causal key
+        // pass 1: the row's max and exp-sum over this warpgroup's half of
+        // every causal key tile
         for (int t = 0; ok && t < nt; ++t) {
-            uint32_t sr[BN];
+            uint32_t sr[HB];
             if (!(ok = load_s(t, sr))) break;
             float mx = -CUDART_INF_F;
 #pragma unroll
-            for (int e = 0; e < BN; e += 2) mx = max3(mx, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+            for (int e = 0; e < HB; e += 2) mx = max3(mx, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
             const float mn = fmaxf(m, mx * c);
             if (mn != -CUDART_INF_F) {
                 float sum = 0.f;
 #pragma unroll
-                for (int e = 0; e < BN; ++e) sum += fast_ex2(__uint_as_float(sr[e]) * c - mn);
+                for (int e = 0; e < HB; ++e) sum += fast_ex2(__uint_as_float(sr[e]) * c - mn);
                 l = l * fast_ex2(m - mn) + sum;
                 m = mn;
             }
         }
+        // the two halves' statistics merged (every warp passes this barrier:
+        // a failed wait leaves ok false but the warp still arrives)
+        if (xg == 1) stat[r] = make_float2(m, l);
+        sync_wgs();
+        if (xg == 0) {
+            const float2 o2 = stat[r];
+            const float mn = fmaxf(m, o2.x);
+            if (mn != -CUDART_INF_F) {
+                l = l * fast_ex2(m - mn) + o2.y * fast_ex2(o2.x - mn);
+                m = mn;
+            }
+            stat[r] = make_float2(m, l);
+        }
+        sync_wgs();
+        if (xg == 1) {
+            const float2 mine = stat[r];
+            m = mine.x;
+            l = mine.y;
+        }
+        ok = __all_sync(0xffffffffu, ok && !*abort_flag);
         const float lse2 = (valid && l > 0.f) ? m + __log2f(l) : CUDART_INF_F;  // +inf: P = 0
-        // pass 2: P against the full statistic, the tile decision, P of kept tiles
+        // pass 2: P against the full statistic, the block decision, P of kept blocks
         bool any = false;
         uint8_t *krow = a.keep + (((long long)b * p.Hq + hq) * p.nqt + qt) * p.nkt;
-        for (int t = 0; ok && t < nt; ++t) {
-            uint32_t sr[BN];
-            if (!(ok = load_s(nt + t, sr))) break;
+        for (int t = 0; t < nt; ++t) {
+            uint32_t sr[HB];
+            const bool got = ok && load_s(nt + t, sr);
+            ok = got;
             float mass = 0.f;
 #pragma unroll
-            for (int e = 0; e < BN; ++e) {
-                const float pe = fast_ex2(__uint_as_float(sr[e]) * c - lse2);
+            for (int e = 0; e < HB; ++e) {
+                const float pe = got ? fast_ex2(__uint_as_float(sr[e]) * c - lse2) : 0.f;
                 mass += pe;
                 sr[e] = __float_as_uint(pe);
             }
-            float wmax = valid ? mass : 0.f;
+            const int y = t & 1;
+            // row mass = the two halves' sums; the largest over the 128 rows
+            half[(y * 2 + xg) * 128 + r] = mass;
+            sync_wgs();
+            const float rowm = half[y * 256 + r] + half[y * 256 + 128 + r];
+            float wmax = valid ? rowm : 0.f;
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, off));
-            const int y = t & 1;
-            if (lane == 0) red[y * 4 + warp] = wmax;
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            const float cmax = fmaxf(fmaxf(red[y * 4], red[y * 4 + 1]), fmaxf(red[y * 4 + 2], red[y * 4 + 3]));
+            if (lane == 0) red[y * 8 + warp] = wmax;
+            sync_wgs();
+            float cmax = red[y * 8];
+#pragma unroll
+            for (int w2 = 1; w2 < 8; ++w2) cmax = fmaxf(cmax, red[y * 8 + w2]);
             const bool keep = cmax >= a.tau;
+            if (!ok) continue;  // every warp keeps meeting the barriers above; nothing else is waited for
             if (t >= 2) {
                 // PV of tile t-2 read this P buffer (P_DONE(y) has completed
                 // phase (t >> 1) - 1 or is about to; never phase t >> 1)
                 if (!(ok = __all_sync(0xffffffffu, mbar_wait(P_DONE(y), ((t >> 1) - 1) & 1, p.err, abort_flag))))
-                    break;
+                    continue;
                 tc_fence_after();
             }
             if (keep) {
-                uint32_t pk[BN / 2];
+                uint32_t pk[HB / 2];
 #pragma unroll
-                for (int e = 0; e < BN / 2; ++e) pk[e] = pack2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
-                const uint32_t tp = tmem + C::T_P + y * (BN / 2) + lane_off;
-                tmem_st16(tp, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-                tmem_st16(tp + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+                for (int e = 0; e < HB / 2; ++e) pk[e] = pack2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
+                tmem_st16(tmem + C::T_P + y * (BN / 2) + xg * (HB / 2) + lane_off, pk);
                 tmem_wait_st();
             }
-            if (r == 0) {
+            if (r == 0 && xg == 0) {
                 kflag[y] = keep ? 1 : 0;
                 krow[t] = keep ? 1 : 0;
             }
@@ -301,18 +336,19 @@ __global__ void __launch_bounds__(192, 1) mala_fwd_kernel(const __grid_constant_
             any = any || keep;
         }
         // tiles past the causal diagonal are never kept
-        for (int t = nt + r; t < p.nkt; t += BM) krow[t] = 0;
-        // epilogue: O = the kept tiles' P V (P is already normalised), LSE
+        for (int t = nt + xg * 128 + r; t < p.nkt; t += 256) krow[t] = 0;
+        // epilogue: O = the kept tiles' P V (P is already normalised), LSE;
+        // warpgroup x writes columns [x*D/2, x*D/2 + D/2)
         ok = __all_sync(0xffffffffu, ok && mbar_wait(FIN, 0, p.err, abort_flag));
         tc_fence_after();
         const bool have = ok && any;
         __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + b * p.os[0] + (long long)(i0 + r) * p.os[1] +
-                              hq * p.os[2];
+                              hq * p.os[2] + xg * (D / 2);
 #pragma unroll
-        for (int cc = 0; cc < D / 16; ++cc) {
+        for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[16];
             if (have) {
-                tmem_ld16(tmem + C::T_O + cc * 16 + lane_off, o);
+                tmem_ld16(tmem + C::T_O + xg * (D / 2) + cc * 16 + lane_off, o);
                 tmem_wait_ld();
             } else {
 #pragma unroll
@@ -327,7 +363,7 @@ __global__ void __launch_bounds__(192, 1) mala_fwd_kernel(const __grid_constant_
                 dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
         }
-        if (valid)
+        if (valid && xg == 0)
             p.lse[((long long)b * p.Hq + hq) * p.lse_ld + i0 + r] =
                 l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
     }
@@ -335,7 +371,7 @@ __global__ void __launch_bounds__(192, 1) mala_fwd_kernel(const __grid_constant_
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem, 512);
+    if (warp == 9) tmem_dealloc(tmem, 512);
 }
 
 template <int D>
@@ -359,7 +395,7 @@ static cudaError_t launch_mala_fwd_d(const AttnParams &p, uint8_t *keep, float t
     const unsigned blocks = tile_grid_blocks(p.nqt, p.Hq, p.B);
     if (!blocks) return cudaErrorInvalidConfiguration;
     launch_begin("mala_fwd", st);
-    mala_fwd_kernel<D><<<blocks, 192, C::SMEM, st>>>(a);
+    mala_fwd_kernel<D><<<blocks, 320, C::SMEM, st>>>(a);
     launch_end(st);
     return cudaGetLastError();
 }
