@@ -113,9 +113,12 @@ struct BwdArgs {
 // together are neighbouring key tiles of one head, which read the same query
 // rows (measured at 32K, d = 128: DRAM reads 9.0 -> 1.6 GB per launch, L2 hit
 // rate 63 -> 91 %); the long sink CTAs start in the first wave.
-// A packed batch's CTA takes item blockIdx.x / Hkv of the key-major work
-// list instead; false when it has no item.
-__device__ __forceinline__ bool dkdv_order(const AttnParams &p, int &kt, int &hl, int &b)
+// With by_head false the order is tile step slowest and (KV head, batch)
+// fastest, every head's sink tile first (at d = 64 this measured faster:
+// recall8k 0.334 against 0.360 ms; its query rows fit L2 either way).  A
+// packed batch's CTA takes item blockIdx.x / Hkv of the key-major work list
+// instead; false when it has no item.
+__device__ __forceinline__ bool dkdv_order(const AttnParams &p, int &kt, int &hl, int &b, bool by_head)
 {
     if (p.work) {
         const int2 it = p.work[blockIdx.x / (unsigned)p.Hkv];
@@ -123,6 +126,13 @@ __device__ __forceinline__ bool dkdv_order(const AttnParams &p, int &kt, int &hl
         b = it.x;
         kt = it.y;
         return it.x >= 0;
+    }
+    if (!by_head) {
+        const TilePos t = tile_pos(p.Hkv, p.B);
+        kt = t.step;
+        hl = t.slot;
+        b = t.b;
+        return true;
     }
     const unsigned hb_n = (unsigned)p.Hkv * (unsigned)p.B, lin = blockIdx.x;
     if (lin < hb_n) {
@@ -169,7 +179,7 @@ struct KvCfg {
     static constexpr uint32_t IDESC_G = idesc_bf16(128, D, 0, 1);
 };
 
-template <int D>
+template <int D, bool MALA>
 __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constant__ BwdArgs a)
 {
     using C = KvCfg<D>;
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int kt, hl, b;
-    if (!dkdv_order(p, kt, hl, b)) return;
+    if (!dkdv_order(p, kt, hl, b, true)) return;
     const SeqGeom sg = seq_geom(p, b);
     const int c0 = kt * BN;
     if (c0 >= sg.Lk) return;  // past the end of this sequence of a packed batch
@@ -405,7 +415,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
         int gi = nq > 0 ? x / nq : 0, tq = nq > 0 ? x % nq : 0;
         // MALA block decisions of this key's column for the group's first
         // query head (nullptr for CoWA)
-        const uint8_t *kbase = p.keep ? p.keep + ((long long)b * p.Hq + hl * p.g) * p.keep_nqt * p.keep_nkt +
+        const uint8_t *kbase = MALA ? p.keep + ((long long)b * p.Hq + hl * p.g) * p.keep_nqt * p.keep_nkt +
                                             jg / kMalaBN
                                       : nullptr;
         for (int k = 0; ok; ++k) {
@@ -415,7 +425,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
             const int qt = tq < len0 || nr == 1 ? lo0 + tq
                            : (tq - len0 < len1 || nr == 2 ? lo1 + tq - len0 : lo2 + tq - len0 - len1);
             // MALA: a key of a skipped block has dP = 0 and no dV share
-            const bool skip = kbase && !kbase[(gi * p.keep_nqt + qt * BM / kMalaBM) * p.keep_nkt];
+            const bool skip = MALA && !kbase[(gi * p.keep_nqt + qt * BM / kMalaBM) * p.keep_nkt];
             tq += 2;
             while (tq >= nq) {
                 tq -= nq;
@@ -557,7 +567,7 @@ struct KvSsCfg {
     static constexpr uint32_t IDESC_G = idesc_bf16(128, D, 0, 1);
 };
 
-template <int D>
+template <int D, bool MALA>
 __global__ void __launch_bounds__(352, 1) dkdv_sm100_ss_kernel(const __grid_constant__ BwdArgs a)
 {
     using C = KvSsCfg<D>;
@@ -589,7 +599,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_ss_kernel(const __grid_cons
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int kt, hl, b;
-    if (!dkdv_order(p, kt, hl, b)) return;
+    if (!dkdv_order(p, kt, hl, b, false)) return;
     const SeqGeom sg = seq_geom(p, b);
     const int c0 = kt * BN;
     if (c0 >= sg.Lk) return;  // past the end of this sequence of a packed batch
@@ -766,7 +776,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_ss_kernel(const __grid_cons
         bool ok = true;
         // MALA block decisions of this key's column for the group's first
         // query head (nullptr for CoWA)
-        const uint8_t *kbase = p.keep ? p.keep + ((long long)b * p.Hq + hl * p.g) * p.keep_nqt * p.keep_nkt +
+        const uint8_t *kbase = MALA ? p.keep + ((long long)b * p.Hq + hl * p.g) * p.keep_nqt * p.keep_nkt +
                                             jg / kMalaBN
                                       : nullptr;
         for (int k = 0;; ++k) {
@@ -776,7 +786,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_ss_kernel(const __grid_cons
             const int qt = tq < len0 || nr == 1 ? lo0 + tq
                            : (tq - len0 < len1 || nr == 2 ? lo1 + tq - len0 : lo2 + tq - len0 - len1);
             // MALA: a key of a skipped block has dP = 0 and no dV share
-            const bool skip = kbase && !kbase[(gi * p.keep_nqt + qt * BM / kMalaBM) * p.keep_nkt];
+            const bool skip = MALA && !kbase[(gi * p.keep_nqt + qt * BM / kMalaBM) * p.keep_nkt];
             tq += 2;
             while (tq >= nq) {
                 tq -= nq;
@@ -908,7 +918,7 @@ struct DqCfg {
     static constexpr uint32_t IDESC_Q = idesc_bf16(128, D, 0, 1);
 };
 
-template <int D>
+template <int D, bool MALA>
 __global__ void __launch_bounds__(352, 1) dq_sm100_kernel(const __grid_constant__ BwdArgs a)
 {
     using C = DqCfg<D>;
@@ -1113,7 +1123,7 @@ __global__ void __launch_bounds__(352, 1) dq_sm100_kernel(const __grid_constant_
             const int j0 = tile_of(t) * BN;
             // MALA: a skipped block's pairs have dP = 0 (query tiles of this
             // pass are the blocks' rows, key tiles their keys)
-            const bool skip = p.keep && !p.keep[(((long long)b * p.Hq + hq) * p.keep_nqt + qt) * p.keep_nkt +
+            const bool skip = MALA && !p.keep[(((long long)b * p.Hq + hq) * p.keep_nqt + qt) * p.keep_nkt +
                                                 j0 / kMalaBN];
             const bool full = __all_sync(0xffffffffu, runs_cover(rr, j0, j0 + BN - 1));
             uint32_t vis[BN / 32];
@@ -1235,6 +1245,7 @@ struct DqTmCfg {
     static constexpr uint32_t IDESC_Q = idesc_bf16(128, D, 0, 1);
 };
 
+template <bool MALA>
 __global__ void __launch_bounds__(352, 1) dq_tm_kernel(const __grid_constant__ BwdArgs a)
 {
     using C = DqTmCfg;
@@ -1439,7 +1450,7 @@ __global__ void __launch_bounds__(352, 1) dq_tm_kernel(const __grid_constant__ B
             // tile set-up, independent of the scores: done while they land
             const int j0 = tile_of(t) * BN + x * 32;
             // MALA: a skipped block's pairs have dP = 0
-            const bool skip = p.keep && !p.keep[(((long long)b * p.Hq + hq) * p.keep_nqt + qt) * p.keep_nkt +
+            const bool skip = MALA && !p.keep[(((long long)b * p.Hq + hq) * p.keep_nqt + qt) * p.keep_nkt +
                                                 j0 / kMalaBN];
             const bool full = __all_sync(0xffffffffu, runs_cover(rr, j0, j0 + 31));
             const uint32_t vis = full ? 0xffffffffu : runs_bits(rr, j0);
@@ -1520,7 +1531,7 @@ __global__ void __launch_bounds__(352, 1) dq_tm_kernel(const __grid_constant__ B
 }
 
 // ----------------------------------------------------------------- host ----
-template <int D>
+template <int D, bool MALA>
 static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, int nqt_dq, int nkt_kv,
                                  const int2 *work_q, int work_q_n, const int2 *work_k, int work_k_n, cudaStream_t st)
 {
@@ -1529,13 +1540,13 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, i
     static std::atomic<bool> configured[64];
     cudaError_t e = once_per_device(configured, [] {
         if constexpr (D == 128) {
-            cudaError_t r = cudaFuncSetAttribute(dkdv_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
+            cudaError_t r = cudaFuncSetAttribute(dkdv_sm100_kernel<128, MALA>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
             if (r != cudaSuccess) return r;
-            return cudaFuncSetAttribute(dq_tm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DqTmCfg::SMEM);
+            return cudaFuncSetAttribute(dq_tm_kernel<MALA>, cudaFuncAttributeMaxDynamicSharedMemorySize, DqTmCfg::SMEM);
         } else {
-            cudaError_t r = cudaFuncSetAttribute(dkdv_sm100_ss_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
+            cudaError_t r = cudaFuncSetAttribute(dkdv_sm100_ss_kernel<64, MALA>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
             if (r != cudaSuccess) return r;
-            return cudaFuncSetAttribute(dq_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, Q::SMEM);
+            return cudaFuncSetAttribute(dq_sm100_kernel<64, MALA>, cudaFuncAttributeMaxDynamicSharedMemorySize, Q::SMEM);
         }
     });
     if (e != cudaSuccess) return e;
@@ -1571,9 +1582,9 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, i
         if (!g1) return cudaErrorInvalidConfiguration;
         launch_begin("dkdv_sm100", st);
         if constexpr (D == 128)
-            dkdv_sm100_kernel<128><<<g1, 352, K::SMEM, st>>>(a);
+            dkdv_sm100_kernel<128, MALA><<<g1, 352, K::SMEM, st>>>(a);
         else
-            dkdv_sm100_ss_kernel<64><<<g1, 352, K::SMEM, st>>>(a);
+            dkdv_sm100_ss_kernel<64, MALA><<<g1, 352, K::SMEM, st>>>(a);
         launch_end(st);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
@@ -1594,7 +1605,7 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, i
             const unsigned g2 = work_q ? tile_grid_blocks(work_q_n, p.Hq, 1) : tile_grid_blocks(nqt_dq, p.Hq, p.B);
             if (!g2) return cudaErrorInvalidConfiguration;
             launch_begin("dq_sm100", st);
-            dq_tm_kernel<<<g2, 352, DqTmCfg::SMEM, st>>>(a);
+            dq_tm_kernel<MALA><<<g2, 352, DqTmCfg::SMEM, st>>>(a);
             launch_end(st);
         } else {
             a.npair = (p.g + Q::NSLOT - 1) / Q::NSLOT;
@@ -1602,7 +1613,7 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, i
                                        : tile_grid_blocks(nqt_dq, (long long)p.Hkv * a.npair, p.B);
             if (!g2) return cudaErrorInvalidConfiguration;
             launch_begin("dq_sm100", st);
-            dq_sm100_kernel<64><<<g2, 352, Q::SMEM, st>>>(a);
+            dq_sm100_kernel<64, MALA><<<g2, 352, Q::SMEM, st>>>(a);
             launch_end(st);
         }
         e = cudaGetLastError();
@@ -1614,8 +1625,13 @@ cudaError_t launch_bwd_sm100(const AttnParams &p, int D, float2 *lsd, int lq_pad
                              cudaStream_t st, const int2 *work_q, int work_q_n, const int2 *work_k, int work_k_n)
 {
     if (p.B == 0 || p.Hq == 0) return cudaSuccess;
-    return D == 128 ? launch_bwd5_d<128>(p, lsd, lq_pad, nqt_dq, nkt_kv, work_q, work_q_n, work_k, work_k_n, st)
-                    : launch_bwd5_d<64>(p, lsd, lq_pad, nqt_dq, nkt_kv, work_q, work_q_n, work_k, work_k_n, st);
+    // MALA's block decisions are a separate instantiation, so the CoWA
+    // kernels carry none of their code
+    if (p.keep)
+        return D == 128 ? launch_bwd5_d<128, true>(p, lsd, lq_pad, nqt_dq, nkt_kv, work_q, work_q_n, work_k, work_k_n, st)
+                        : launch_bwd5_d<64, true>(p, lsd, lq_pad, nqt_dq, nkt_kv, work_q, work_q_n, work_k, work_k_n, st);
+    return D == 128 ? launch_bwd5_d<128, false>(p, lsd, lq_pad, nqt_dq, nkt_kv, work_q, work_q_n, work_k, work_k_n, st)
+                    : launch_bwd5_d<64, false>(p, lsd, lq_pad, nqt_dq, nkt_kv, work_q, work_q_n, work_k, work_k_n, st);
 }
 
 }  // namespace cowa
