@@ -1,4 +1,6 @@
-// CoWA training / prefill forward on the 5th-generation tensor cores.
+// CoWA training / prefill forward on the 5th-generation tensor cores, d = 64
+// (d = 128 runs the kernel of fwd_d128.cu, built on the same plan with 128-key
+// tiles).
 //
 // One CTA per (query tile of 128 rows, pair of query heads of one GQA group,
 // batch).  Two query heads of a group have the same KV head, hence the same
@@ -32,11 +34,10 @@
 //              by exactly the weights it accumulated.  The O row is
 //              rescaled in tensor memory only when the max grows by more than
 //              2^8 (until then the stale max is a valid reference point).
-// Key tiles are 96 wide for d = 64 and 64 wide for d = 128: a softmax thread
-// reads its whole row of S_x with one tensor-memory round trip and keeps it
-// in registers.  Tensor-memory columns (O_x is d + 16 wide: O, then the bf16
-// row sums) for d = 64: S_x at 96x, P_x at 192 + 64x, O_x at 320 + 96x; for
-// d = 128: S_x at 64x, P_x at 128 + 32x, O_x at 192 + 160x.
+// Key tiles are 96 wide: a softmax thread reads its whole row of S_x with one
+// tensor-memory round trip and keeps it in registers.  Tensor-memory columns
+// (O_x is d + 16 wide: O, then the bf16 row sums): S_x at 96x, P_x at
+// 192 + 64x, O_x at 320 + 96x.
 // Softmax x rewrites P_x and rescales O_x for tile t only after O_DONE_x says
 // PV_x(t-1) is complete.
 // The exponential loops of the two slots alternate per lane quadrant (the two
@@ -66,17 +67,17 @@ struct FwdArgs {
 
 template <int D>
 struct FwdCfg {
+    static_assert(D == 64, "d = 128 has its own kernel");
     static constexpr int BM = 128, BN = fwd5_bn(D);
     static constexpr int STAGES = 4;  // tiles t, t+1, t+2 are resident at once
     // tensor-memory column of S_x, P_x, O_x
-    static constexpr __host__ __device__ int t_s(int x) { return D == 128 ? 64 * x : 96 * x; }
-    static constexpr __host__ __device__ int t_p(int x) { return D == 128 ? 128 + 32 * x : 192 + 64 * x; }
-    static constexpr __host__ __device__ int t_o(int x) { return D == 128 ? 192 + 160 * x : 320 + 96 * x; }
+    static constexpr __host__ __device__ int t_s(int x) { return 96 * x; }
+    static constexpr __host__ __device__ int t_p(int x) { return 192 + 64 * x; }
+    static constexpr __host__ __device__ int t_o(int x) { return 320 + 96 * x; }
     static constexpr int OW = D + 16;                 // O columns, then the bf16 row sums
-    // exponentials on the FMA pipe: one pair in four for d = 64, where the
-    // softmax paces the kernel (measured against none, one in two and one in
-    // three); none for d = 128, where it measured slower
-    static constexpr int POLY_EVERY = D == 64 ? 4 : 0;
+    // exponentials on the FMA pipe: one pair in four, where the softmax paces
+    // the kernel (measured against none, one in two and one in three)
+    static constexpr int POLY_EVERY = 4;
     static constexpr int KB = D / 64;                 // 128-byte blocks along d
     static constexpr int Q_BYTES = BM * D * 2;        // one head's query tile
     static constexpr int KV_BYTES = BN * D * 2;       // one of K or V
@@ -534,7 +535,7 @@ static cudaError_t launch_fwd5_d(const AttnParams &p, cudaStream_t st)
 cudaError_t launch_fwd_sm100(const AttnParams &p, int D, cudaStream_t st)
 {
     if (p.nqt == 0 || p.Hq == 0 || p.B == 0) return cudaSuccess;
-    return D == 128 ? launch_fwd5_d<128>(p, st) : launch_fwd5_d<64>(p, st);
+    return D == 128 ? launch_fwd_d128(p, st) : launch_fwd5_d<64>(p, st);
 }
 
 }  // namespace cowa

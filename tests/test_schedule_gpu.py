@@ -36,10 +36,9 @@ SMALL = [  # Lq, Lk, Hkv, quad
 ]
 
 
-# the tilings the kernels use: forward 128x96 (d=64) and 128x64 (d=128);
-# backward dQ 128x64 (d=64) and 128x128 (d=128), dK/dV key-tile major over
-# 128 keys with 64 (d=64) or 32 (d=128) query rows per task; the warp-level
-# kernels' 64x64 and key-major 32/64 x 64
+# the tilings the kernels use: forward 128x96 (d=64) and 128x128 (d=128);
+# backward dQ 128x64, dK/dV key-tile major over 128 keys with 64 (d=64) or
+# 32 (d=128) query rows per task; MALA blocks 128x64; and smaller tilings
 TILINGS = [(128, 96, False), (128, 64, False), (128, 128, False), (64, 128, True), (32, 128, True),
            (64, 64, False), (32, 64, True), (64, 64, True)]
 
