@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(S_FULL(x), 1);
-            mbar_init(P_FULL(x), 128);
+            mbar_init(P_FULL(x), 4);  // one arrival per warp
             mbar_init(S_FREE(x), 4);  // one arrival per warp
             mbar_init(G_DONE(x), 1);
         }
@@ -501,7 +501,8 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_kernel(const __grid_constan
             if (!ok) break;
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(P_FULL(x));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(P_FULL(x));
         }
         // epilogue: warpgroup 0 writes dK (scaled), warpgroup 1 writes dV
         ok = __all_sync(0xffffffffu, mbar_wait(DONE, 0, p.err, abort_flag) && ok);
@@ -631,7 +632,7 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_ss_kernel(const __grid_cons
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(S_FULL(x), 1);
-            mbar_init(P_FULL(x), 128);
+            mbar_init(P_FULL(x), 4);  // one arrival per warp
             mbar_init(S_FREE(x), 4);  // one arrival per warp
             mbar_init(G_DONE(x), 1);
         }
@@ -858,7 +859,8 @@ __global__ void __launch_bounds__(352, 1) dkdv_sm100_ss_kernel(const __grid_cons
             if (!ok) break;
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(P_FULL(x));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(P_FULL(x));
         }
         // epilogue: warpgroup 0 writes dK (scaled), warpgroup 1 writes dV
         ok = __all_sync(0xffffffffu, mbar_wait(DONE, 0, p.err, abort_flag) && ok);
@@ -980,7 +982,7 @@ __global__ void __launch_bounds__(352, 1) dq_sm100_kernel(const __grid_constant_
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(S_FULL(x), 1);
-            mbar_init(DS_FULL(x), 128);
+            mbar_init(DS_FULL(x), 4);  // one arrival per warp
             mbar_init(DONE(x), 1);
             mbar_init(S_FREE(x), 4);  // one arrival per warp
             mbar_init(FIN(x), 1);
@@ -1179,7 +1181,8 @@ __global__ void __launch_bounds__(352, 1) dq_sm100_kernel(const __grid_constant_
             if (!ok) break;
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(DS_FULL(x));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(DS_FULL(x));
         }
         if (active && ok && ntiles > 0)
             ok = __all_sync(0xffffffffu, mbar_wait(DONE(x), (ntiles - 1) & 1, p.err, abort_flag));
@@ -1305,7 +1308,7 @@ __global__ void __launch_bounds__(352, 1) dq_tm_kernel(const __grid_constant__ B
         mbar_init(S_FULL, 1);
         mbar_init(S_FREE, 8);  // one arrival per elementwise warp
         for (int y = 0; y < 2; ++y) {
-            mbar_init(DS_FULL(y), 256);
+            mbar_init(DS_FULL(y), 8);  // one arrival per warp
             mbar_init(DONE(y), 1);
             mbar_init(FIN(y), 1);
         }
@@ -1493,7 +1496,8 @@ __global__ void __launch_bounds__(352, 1) dq_tm_kernel(const __grid_constant__ B
             tmem_st16(tmem + C::t_ds(y) + x * 16 + lane_off, pk);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(DS_FULL(y));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(DS_FULL(y));
         }
         // the last dQ MMA: DONE of the last tile's parity
         if (ok && ntiles > 0)

@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(384, 1) fwd_sm100_d128_kernel(const __grid_con
         for (int x = 0; x < 2; ++x) {
             mbar_init(S_FULL(x), 1);
             mbar_init(S_FREE(x), 4);  // one arrival per softmax warp
-            mbar_init(P_FULL(x), 128);
+            mbar_init(P_FULL(x), 4);  // one arrival per softmax warp
             mbar_init(O_DONE(x), 1);
             mbar_init(FIN(x), 1);
         }
@@ -400,7 +400,8 @@ __global__ void __launch_bounds__(384, 1) fwd_sm100_d128_kernel(const __grid_con
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(P_FULL(x));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(P_FULL(x));
         }
         // every MMA of this slot has completed (FIN follows the last PV)
         if (active) ok = __all_sync(0xffffffffu, ok && mbar_wait(FIN(x), 0, p.err, abort_flag));

@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(352, 1) fwd_sm100_kernel(const __grid_constant
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(S_FULL(x), 1);
-            mbar_init(P_FULL(x), 128);
+            mbar_init(P_FULL(x), 4);  // one arrival per softmax warp
             mbar_init(O_DONE(x), 1);
             mbar_init(S_FREE(x), 4);  // one arrival per softmax warp
             for (int qd = 0; qd < 4; ++qd) mbar_init(TURN(x, qd), 1);
@@ -409,7 +409,8 @@ __global__ void __launch_bounds__(352, 1) fwd_sm100_kernel(const __grid_constant
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(P_FULL(x));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(P_FULL(x));
         }
         if (active && ok && ntiles > 0) {
             // PV_x(ntiles-2) was waited for at the last tile, so O_DONE(x) has

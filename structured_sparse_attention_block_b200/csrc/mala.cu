@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(320, 1) mala_fwd_kernel(const __grid_constant_
         for (int x = 0; x < 2; ++x) {
             mbar_init(S_FULL(x), 1);
             mbar_init(S_FREE(x), 8);  // one arrival per softmax warp
-            mbar_init(P_FULL(x), 256);
+            mbar_init(P_FULL(x), 8);  // one arrival per softmax warp
             mbar_init(P_DONE(x), 1);
         }
         mbar_init(FIN, 1);
@@ -332,7 +332,8 @@ __global__ void __launch_bounds__(320, 1) mala_fwd_kernel(const __grid_constant_
                 krow[t] = keep ? 1 : 0;
             }
             tc_fence_before();
-            mbar_arrive(P_FULL(y));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(P_FULL(y));
             any = any || keep;
         }
         // tiles past the causal diagonal are never kept

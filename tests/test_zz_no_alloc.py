@@ -4,8 +4,9 @@ Such callers (a plugin inside a runtime that owns all device memory and hands
 over only input and output buffers, or a serving loop where cudaMalloc is not
 allowed) get a decode whose split scratch is a fixed array inside the
 library.  These tests call it through the C ABI and compare it with
-cowa_decode, which takes a caller workspace, on two calls in a row (the
-second call finds the first call's partials still in the array), check that
+cowa_decode, which takes a caller workspace, and with the fp64 oracle, on two
+calls in a row (the second call finds the first call's partials still in the
+array), check that
 a call leaves device memory as it found it (neither torch's allocator nor the
 driver's free-memory count moves), call it once through the Python wrapper,
 and check that a shape too large for the array is refused before anything
@@ -16,7 +17,9 @@ import ctypes
 import pytest
 import torch
 
-from helpers import LSE_ABS, assert_o, to64
+import numpy as np
+
+from helpers import LSE_ABS, assert_lse, assert_o, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -29,9 +32,9 @@ def noalloc_status(cowa, q, kc, vc, sl, quad, out, lse):
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-def test_noalloc_matches_decode_on_two_calls_in_a_row():
+def test_noalloc_matches_decode_on_two_calls_in_a_row(oracle_mod):
     import structured_sparse_attention_block_b200 as cowa
-    from structured_sparse_attention_block_b200.inputs import decode_inputs
+    from structured_sparse_attention_block_b200.inputs import bf16_bits, decode_inputs
     quad = (64, 512, 0, 896)
     runs = [(0, [4096, 4000, 129, 1]), (1, [77, 4096, 2048, 3000])]
     for seed, seqlens in runs:
@@ -45,6 +48,10 @@ def test_noalloc_matches_decode_on_two_calls_in_a_row():
         assert_o(out[:, 0], to64(o_ref[:, 0]), what="noalloc O")
         diff = (lse - lse_ref).abs().max().item()
         assert diff <= LSE_ABS
+        # and against the oracle's decode of the same inputs
+        o64, lse64 = oracle_mod.decode(bf16_bits(q[:, 0]), bf16_bits(kc), bf16_bits(vc), np.array(seqlens), quad)
+        assert_o(out[:, 0], o64, what="noalloc O vs oracle")
+        assert_lse(lse, lse64)
 
 
 def test_noalloc_leaves_device_memory_unchanged():
