@@ -227,7 +227,7 @@ KERNEL_SOURCES = {
     "bwd_prep": ["bwd_sm100.cu"],
     "decode_split": ["decode.cu"],
     "decode_combine": ["decode.cu"],
-    "mala_fwd": ["mala.cu"],
+    "mala_fwd": ["mala.cu", "mala_d128.cu"],
     "varlen_worklist": ["worklist.cu"],
 }
 SHARED_SOURCES = ["common.cuh", "kernels.cuh", "sm100.cuh"]

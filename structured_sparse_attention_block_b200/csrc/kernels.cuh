@@ -203,6 +203,8 @@ bool make_bshd_map(CUtensorMap *m, const void *base, int d, long long L, long lo
 // together; keep[b][hq][qt][kt] receives the decisions
 constexpr int kMalaBM = 128, kMalaBN = 64;
 cudaError_t launch_mala_fwd(const AttnParams &p, int D, uint8_t *keep, float tau, cudaStream_t st);
+// mala_d128.cu: the d = 128 MALA forward, called by launch_mala_fwd
+cudaError_t launch_mala_fwd_d128(const AttnParams &p, uint8_t *keep, float tau, cudaStream_t st);
 
 // worklist.cu: the (sequence, tile) items of a packed batch for tiles of
 // `tile` rows of the offsets cu [B + 1] (descending: the query-major order,

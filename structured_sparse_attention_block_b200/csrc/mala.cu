@@ -1,4 +1,5 @@
-// MassAlloc Attention (MALA) forward on the 5th-generation tensor cores.
+// MassAlloc Attention (MALA) forward on the 5th-generation tensor cores, d = 64
+// (d = 128 runs the kernel of mala_d128.cu: two heads per CTA, 128-key tiles).
 //
 // "Two new attention models slash redundancy..." (first section) and the
 // abstract of "CoWindow Attention: Full Causal Coverage Is a Collective
@@ -404,7 +405,7 @@ static cudaError_t launch_mala_fwd_d(const AttnParams &p, uint8_t *keep, float t
 cudaError_t launch_mala_fwd(const AttnParams &p, int D, uint8_t *keep, float tau, cudaStream_t st)
 {
     if (p.nqt == 0 || p.Hq == 0 || p.B == 0) return cudaSuccess;
-    return D == 128 ? launch_mala_fwd_d<128>(p, keep, tau, st) : launch_mala_fwd_d<64>(p, keep, tau, st);
+    return D == 128 ? launch_mala_fwd_d128(p, keep, tau, st) : launch_mala_fwd_d<64>(p, keep, tau, st);
 }
 
 }  // namespace cowa

@@ -18,6 +18,8 @@ CASES = [  # B, Lq, Lk, Hq, Hkv, d, quad
     (1, 130, 130, 2, 2, 64, (0, 0, 0, 0)),           # nothing visible
     (1, 1, 700, 4, 2, 128, (32, 100, 0, 300)),       # a single query row
     (3, 1000, 1000, 16, 8, 64, (1, 1, 0, 125)),       # many heads, 1-wide windows
+    (2, 700, 700, 6, 2, 128, (8, 150, 0, 330)),      # g = 3: head pairs and a lone head in one launch
+    (1, 1500, 1500, 4, 1, 128, (64, 256, 3, 512)),   # many 128-key tiles per query tile: the K/V rings wrap
 ]
 
 

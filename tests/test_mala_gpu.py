@@ -52,6 +52,7 @@ CASES = [  # B, Lq, Lk, Hq, Hkv, d, spread of q (sharper softmax)
     (2, 200, 200, 2, 1, 128, 1.5),
     (1, 130, 400, 4, 4, 128, 2.0),   # chunked prefill: Lq < Lk
     (1, 257, 257, 8, 2, 64, 3.0),
+    (1, 700, 700, 6, 2, 128, 2.0),   # g = 3: head pairs and a lone head; several 128-key tiles
 ]
 
 
