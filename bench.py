@@ -221,7 +221,7 @@ def load_peaks():
 # Source files each kernel is built from: its traffic record is valid only
 # while their hash matches the one stored beside the counters.
 KERNEL_SOURCES = {
-    "fwd_sm100": ["fwd_sm100.cu", "fwd_d128.cu"],
+    "fwd_sm100": ["fwd_sm100.cu"],
     "dkdv_sm100": ["bwd_sm100.cu"],
     "dq_sm100": ["bwd_sm100.cu"],
     "bwd_prep": ["bwd_sm100.cu"],

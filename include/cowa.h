@@ -331,8 +331,7 @@ COWA_API int cowa_decode_noalloc(const cowa_shape_t *shape, cowa_quad_t quad, fl
  * Visible-tile classes of one KV head, as the training kernels see them, for
  * checking the schedule: writes out[qt * nkt + kt] (device, uint8) for the
  * tiling BM x BN, BM in {32, 64, 128} and BN in {64, 96, 128} (the forward
- * uses query tiles of 128 with key tiles of 96 for d = 64 and 128 for
- * d = 128; the dQ pass query tiles of 128 with key tiles of 64; the dK/dV
+ * uses query tiles of 128 with key tiles of 128; the dQ pass query tiles of 128 with key tiles of 64; the dK/dV
  * pass, key-tile major, key tiles of 128 with query tiles of 64 for d = 64
  * and 32 for d = 128),
  * nqt = ceil(Lq/BM), nkt = ceil(Lk/BN):

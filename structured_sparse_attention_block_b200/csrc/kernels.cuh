@@ -189,12 +189,10 @@ cudaError_t launch_tile_classes(const int *sched, uint8_t *out, int kv_head, int
 
 // fwd_sm100.cu (tcgen05 forward)
 cudaError_t launch_fwd_sm100(const AttnParams &p, int D, cudaStream_t st);
-// fwd_d128.cu: the d = 128 forward (128-key tiles), called by launch_fwd_sm100
-cudaError_t launch_fwd_d128(const AttnParams &p, cudaStream_t st);
 constexpr int kFwd5BM = 128;
-// key-tile width of the tcgen05 forward: 96 for d = 64, 128 for d = 128 (a
-// softmax thread holds one row of a tile in registers)
-__host__ __device__ constexpr int fwd5_bn(int D) { return D == 128 ? 128 : 96; }
+// key-tile width of the tcgen05 forward (a softmax thread holds one row of
+// a tile in registers)
+__host__ __device__ constexpr int fwd5_bn(int) { return 128; }
 // [B, L, H, d] bf16 tensor as a 4-D TMA map, 64-element x `rows` boxes, 128-byte swizzle
 bool make_bshd_map(CUtensorMap *m, const void *base, int d, long long L, long long H, long long B,
                    const long long st[3], int rows);

@@ -14,7 +14,7 @@
 // block decisions (the four warps of a head slot meet once per tile through
 // shared memory), and writes P of the kept blocks (bf16) for
 // O += P V, whose MMAs run only over kept blocks' keys.
-// Tensor memory as in fwd_d128.cu: one 128-column S region shared by the
+// Tensor memory as in fwd_sm100.cu: one 128-column S region shared by the
 // two slots (S_0(i), S_1(i), S_0(i+1), ... each issued once the other slot's
 // softmax holds the previous one), P_x (64 columns), O_x (128 columns).
 // K has a ring of three stages (both passes), V of two (pass 2 only).

@@ -36,7 +36,7 @@ SMALL = [  # Lq, Lk, Hkv, quad
 ]
 
 
-# the tilings the kernels use: forward 128x96 (d=64) and 128x128 (d=128);
+# the tilings the kernels use: forward 128x128 (an earlier d=64 forward used 128x96);
 # backward dQ 128x64, dK/dV key-tile major over 128 keys with 64 (d=64) or
 # 32 (d=128) query rows per task; MALA blocks 128x64; and smaller tilings
 TILINGS = [(128, 96, False), (128, 64, False), (128, 128, False), (64, 128, True), (32, 128, True),
