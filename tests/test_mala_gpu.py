@@ -131,3 +131,50 @@ def test_mala_rejects_bad_arguments():
     for tau in (-0.1, float("nan"), float("inf")):
         with pytest.raises(cowa.CowaError):
             cowa.cowa_mala_fwd(q, k, v, tau)
+
+
+def test_mala_workload_sampled_blocks():
+    """The bench's MALA workload at full size (the 14B-like 32K shape, tau =
+    2^-8, the same seed) in the launch configuration the bench times; sampled
+    query blocks of 128 rows, one head each, against the oracle run on just
+    those rows and their causal keys (rows [i0, i0 + 128) with keys
+    [0, i0 + 128) keep the bottom-right alignment of the full problem).
+    Decisions must agree wherever the oracle's block mass is not within 0.1 %
+    of tau; O, LSE and the rows' dQ use the operator's tolerances (compared
+    only when no decision of the block is that close)."""
+    import structured_sparse_attention_block_b200 as cowa
+    from oracle import mala
+    from structured_sparse_attention_block_b200.inputs import WORKLOADS, bf16_bits, workload_inputs
+    wl = WORKLOADS["llm14b_32k"]
+    tau = 2.0 ** -8
+    q, k, v, do = workload_inputs(wl, seed=11)
+    o, lse, keep = cowa.cowa_mala_fwd(q, k, v, tau)
+    dq, _, _ = cowa.cowa_mala_bwd(q, k, v, o, lse, keep, do)
+    torch.cuda.synchronize()
+    assert cowa.lib().cowa_get_device_error(None) == 0
+    g = wl.Hq // wl.Hkv
+    nqt = -(-wl.Lq // BM)
+    compared = 0
+    for qb, hq in [(nqt - 1, 0), (nqt // 2, 21), (3, 39), (nqt - 2, 17)]:
+        i0 = qb * BM
+        rows = slice(i0, min(i0 + BM, wl.Lq))
+        nk = min(i0 + BM, wl.Lk)
+        h = hq // g
+        q1 = bf16_bits(q[:, rows, hq:hq + 1])
+        k1, v1 = bf16_bits(k[:, :nk, h:h + 1]), bf16_bits(v[:, :nk, h:h + 1])
+        do1 = bf16_bits(do[:, rows, hq:hq + 1])
+        o_ref, lse_ref, keep_ref, _ = mala.fwd(q1, k1, v1, tau, BM, BN)
+        masses = block_masses(q1, k1)[0, 0, 0]
+        got = keep[0, hq, qb].cpu().numpy().astype(bool)
+        nb = keep_ref.shape[-1]
+        near = np.abs(masses - tau) <= 1e-3 * tau
+        assert np.array_equal(got[:nb][~near], keep_ref[0, 0, 0][~near]), "block decisions differ (block %d, head %d)" % (qb, hq)
+        assert not got[nb:].any(), "a block past the causal diagonal is kept"
+        if near.any():
+            continue
+        assert_o(o[:, rows, hq:hq + 1], o_ref)
+        assert_lse(lse[:, hq:hq + 1, rows], lse_ref)
+        rq, _, _ = mala.bwd(q1, k1, v1, do1, tau, BM, BN)
+        assert_grad(dq[:, rows, hq:hq + 1], rq, "dQ")
+        compared += 1
+    assert compared >= 2
