@@ -116,13 +116,29 @@ struct BwdArgs {
 // With by_head false the order is tile step slowest and (KV head, batch)
 // fastest, every head's sink tile first (at d = 64 this measured faster:
 // recall8k 0.334 against 0.360 ms; its query rows fit L2 either way).  A
-// packed batch's CTA takes item blockIdx.x / Hkv of the key-major work list
-// instead; false when it has no item.
+// packed batch's grid runs over the key-major work list's items instead, in
+// the matching order (below); false when the CTA has no item.
 __device__ __forceinline__ bool dkdv_order(const AttnParams &p, int &kt, int &hl, int &b, bool by_head)
 {
     if (p.work) {
-        const int2 it = p.work[blockIdx.x / (unsigned)p.Hkv];
-        hl = (int)(blockIdx.x % (unsigned)p.Hkv);
+        // the list holds rank 0 (each sequence's first key tile, the sink)
+        // first: with by_head, those of every KV head go first, then each
+        // head's remaining items in list order, head after head
+        const unsigned H = (unsigned)p.Hkv, n = (unsigned)p.work_n, lin = blockIdx.x;
+        const unsigned n0 = by_head ? min((unsigned)p.work_n0, n) : 0u;
+        unsigned item;
+        if (!by_head) {
+            item = lin / H;
+            hl = (int)(lin % H);
+        } else if (lin < H * n0) {
+            item = lin / H;
+            hl = (int)(lin % H);
+        } else {
+            const unsigned r = lin - H * n0, per = n - n0;  // per > 0: lin < H * n
+            hl = (int)(r / per);
+            item = n0 + (r - (unsigned)hl * per);
+        }
+        const int2 it = p.work[item];
         b = it.x;
         kt = it.y;
         return it.x >= 0;
@@ -1581,6 +1597,7 @@ static cudaError_t launch_bwd5_d(const AttnParams &p, float2 *lsd, int lq_pad, i
     a.p.nkt = nkt_kv;
     a.p.work = work_k;  // packed batch: the key-major work list
     a.p.work_n = work_k_n;
+    a.p.work_n0 = p.B;  // rank 0 comes first: at most one item per sequence
     if (nkt_kv > 0) {
         const unsigned g1 = work_k ? tile_grid_blocks(work_k_n, p.Hkv, 1) : tile_grid_blocks(nkt_kv, p.Hkv, p.B);
         if (!g1) return cudaErrorInvalidConfiguration;

@@ -76,6 +76,7 @@ struct AttnParams {
     // the grid is work_n x head slots.  nullptr for a uniform batch.
     const int2 *work;
     int work_n;
+    int work_n0;  // key-major list: its first work_n0 items are the tiles of rank 0 (at most one per sequence)
 };
 
 // The tile, head slot and batch entry of a CTA of a query-major pass
@@ -85,19 +86,23 @@ struct AttnParams {
 // fastest and the tile step slowest, the last query tile first: the CTAs
 // resident together then read the K/V windows of two KV heads only, which
 // L2 holds (all KV heads' windows at 128K are about 100 MB), and each
-// group's long CTAs start before its short ones.  A packed batch's CTA
-// takes item blockIdx.x / nslot of the work list.  False when the CTA has
-// no item.
+// group's long CTAs start before its short ones.  A packed batch's grid
+// has the same grouping over the work list's items (heaviest first) in
+// place of the tile steps.  False when the CTA has no item.
 __device__ __forceinline__ bool query_tile_item(const AttnParams &p, int nslot, int spk, int &qt, int &slot, int &b)
 {
+    const unsigned gs = (unsigned)spk * ((p.Hkv % 2 == 0) ? 2u : 1u);  // head slots per group
     if (p.work) {
-        const int2 it = p.work[blockIdx.x / (unsigned)nslot];
-        slot = (int)(blockIdx.x % (unsigned)nslot);
+        // the same grouping over the list's items (heaviest first)
+        const unsigned per = gs * (unsigned)p.work_n, lin = blockIdx.x;
+        const unsigned grp = lin / per, rg = lin - grp * per;
+        const unsigned item = rg / gs;
+        slot = (int)(grp * gs + (rg - item * gs));
+        const int2 it = p.work[item];
         b = it.x;
         qt = it.y;
         return it.x >= 0;
     }
-    const unsigned gs = (unsigned)spk * ((p.Hkv % 2 == 0) ? 2u : 1u);  // head slots per group
     const unsigned per = gs * (unsigned)p.B, lin = blockIdx.x;
     const unsigned grp_n = per * (unsigned)p.nqt;
     const unsigned grp = lin / grp_n, rg = lin - grp * grp_n;
