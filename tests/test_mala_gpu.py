@@ -53,6 +53,8 @@ CASES = [  # B, Lq, Lk, Hq, Hkv, d, spread of q (sharper softmax)
     (1, 130, 400, 4, 4, 128, 2.0),   # chunked prefill: Lq < Lk
     (1, 257, 257, 8, 2, 64, 3.0),
     (1, 700, 700, 6, 2, 128, 2.0),   # g = 3: head pairs and a lone head; several 128-key tiles
+    (1, 300, 130, 4, 2, 128, 2.0),   # Lq > Lk: the first rows see no key (O = 0, LSE = -inf)
+    (2, 260, 100, 2, 1, 64, 2.0),    # the same at d = 64
 ]
 
 
