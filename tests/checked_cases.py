@@ -1,7 +1,7 @@
 """Small ragged parity cases of every kernel, run in a process of their own
-(see test_debug_gpu.py): forward, backward, decode, packed batches and the
-windowed decode cache, each against the fp64 oracle, with the device error
-word read after every case.  Prints "checked ok <library>" at the end."""
+(see test_debug_gpu.py): forward, backward, decode, packed batches, the
+windowed decode cache and MALA, each against the fp64 oracle, with the
+device error word read after every case.  Prints "checked ok <library>" at the end."""
 import os
 import sys
 
@@ -88,6 +88,28 @@ def main():
     no_device_error("windowed decode")
     o_ref, lse_ref = oracle.decode(bf16_bits(qd[:, 0]), bf16_bits(kc), bf16_bits(vc), [700, 400], quad)
     assert_o(od[:, 0], o_ref)
+    # MALA at both ends of tau, where no decision is close to the threshold:
+    # tau = 0 keeps every causal block (dense causal attention), tau > 1
+    # keeps none (O = 0, zero gradients)
+    from oracle import mala
+    for d in (64, 128):
+        q, k, v, do = training_inputs(1, 300, 300, 4, 2, d, seed=d + 5)
+        qb, kb, vb, db = (bf16_bits(x) for x in (q, k, v, do))
+        for tau in (0.0, 1.5):
+            o, lse, keep = cowa.cowa_mala_fwd(q, k, v, tau)
+            dq, dk, dv = cowa.cowa_mala_bwd(q, k, v, o, lse, keep, do)
+            torch.cuda.synchronize()
+            no_device_error("MALA d=%d tau=%g" % (d, tau))
+            o_ref, lse_ref, _, _ = mala.fwd(qb, kb, vb, tau, 128, 64)
+            assert_o(o, o_ref, what="MALA O")
+            assert_lse(lse, lse_ref)
+            if tau == 0.0:
+                rq, rk, rv = mala.bwd(qb, kb, vb, db, tau, 128, 64)
+                assert_grad(dq, rq, "MALA dQ")
+                assert_grad(dk, rk, "MALA dK")
+                assert_grad(dv, rv, "MALA dV")
+            else:
+                assert int(keep.sum()) == 0 and bool(torch.all(dq == 0)) and bool(torch.all(dk == 0))
     print("checked ok %s" % cowa.library_path())
 
 
